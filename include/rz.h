@@ -1,0 +1,182 @@
+/*
+ * rz.h -- C ABI of librz: batch-invariant token logprobs and the REINFORCE Zero
+ * loss / gradient on one NVIDIA B200 (sm_100a).
+ *
+ * What the library computes is defined on the page "vLLM says aligned kernels make
+ * asynchronous RL stable at lag 64" (ainewsbites.com), section "REINFORCE Zero removes
+ * the mismatch first", and the batch-invariance contract on "vLLM Train-Inference
+ * Consistency Release Notes" (agentlenshq.com), section "Achieving Bitwise Consistency":
+ *
+ *   z[t,v]  = sum_k H[t,k] W[v,k]                      (LM head, no bias, temperature 1)
+ *   lse[t]  = log sum_v exp z[t,v];   lp[t] = z[t, y_t] - lse[t]
+ *   w_t     = exp(lp[t] - lp_rollout[t])               (unclipped importance ratio)
+ *   A_i     = r_i - mean_{j in group(i)} r_j           (group-mean advantage)
+ *   loss    = -(1/N) sum_i (A_i / L_i) sum_{t in i} w_t (token mean per response, N responses)
+ *   kappa_t = -A_i w_t / (N L_i) = d loss / d lp_t
+ *   dZ[t,v] = kappa_t ([v == y_t] - exp(z[t,v] - lse[t]))
+ *   dH      = dZ W,   dW = dZ^T H
+ *
+ * Batch invariance: the bits of lp[t] and lse[t] depend only on (H[t,:], y_t, W), never
+ * on n_tok, on the row's position, on the other rows of the call, or on how a sequence
+ * is split into calls (prefill chunks vs one-token decode calls).  rz_loss_fwd_bwd's
+ * lp_out is bitwise equal to rz_token_logprobs' lp_out for the same rows.  All outputs
+ * are deterministic: the same call on the same inputs gives the same bits.
+ *
+ * Conventions for every entry point:
+ *   - Array pointers are DEVICE pointers owned by the caller, dense row-major, and must
+ *     not alias one another (outputs never alias inputs).
+ *   - bf16 arrays are passed as their 16-bit patterns (rz_bf16 = uint16_t).
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls enqueue work
+ *     on it and return without synchronising; argument checks happen on the host first
+ *     and, on error, nothing is enqueued.
+ *   - `workspace` is caller-allocated device memory of at least the size the matching
+ *     rz_workspace_bytes_* query returns, 256-byte aligned.  Its first word is the
+ *     device status of the most recent call that used it (read with
+ *     rz_read_device_status).  A workspace must not be shared by calls that may run
+ *     concurrently.  The library allocates no memory.
+ *   - Shapes: d % 64 == 0 (64 <= d <= 32768); 1 <= V <= 2^31 - 1; 0 <= n_tok < 2^31.
+ *     H, W, dH, dW must be 16-byte aligned; other arrays 4-byte aligned (8 for int64).
+ *   - Device-checked inputs (a violation sets a bit of the device status and never
+ *     traps): 0 <= token_ids[t] < V (the row's lp becomes NaN); seg_offsets[0] = 0,
+ *     seg_offsets strictly increasing, seg_offsets[n_resp] = n_tok; 0 <= group_ids < n_groups.
+ */
+#ifndef RZ_H_
+#define RZ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t rz_bf16; /* bit pattern of a bfloat16 value */
+
+typedef enum {
+  RZ_OK = 0,
+  RZ_ERR_INVALID_ARG = 1,         /* null pointer, bad size, misaligned pointer            */
+  RZ_ERR_UNSUPPORTED_SHAPE = 2,   /* d not a multiple of 64, or a size beyond the limits  */
+  RZ_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes below the rz_workspace_bytes_* query         */
+  RZ_ERR_CUDA = 4,                /* a CUDA runtime/driver call failed (launch, memset…)   */
+  RZ_ERR_DEVICE_CHECK = 5,        /* device-side input check failed (ids, segments, groups)*/
+  RZ_ERR_DEVICE_TIMEOUT = 6       /* a kernel wait gave up (bounded wait limit reached)    */
+} rz_status;
+
+/* Device status bits (the first int32 of a workspace). */
+#define RZ_DEV_BAD_TOKEN_ID 1
+#define RZ_DEV_BAD_SEGMENTS 2
+#define RZ_DEV_BAD_GROUP_ID 4
+#define RZ_DEV_WAIT_TIMEOUT 8
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* rz_status_string(rz_status s);
+
+/* Workspace bytes for rz_token_logprobs(n_tok, d, V); 0 if the shape is unsupported. */
+size_t rz_workspace_bytes_logprobs(int64_t n_tok, int32_t d, int32_t V);
+
+/* Workspace bytes for rz_loss_fwd_bwd; 0 if the shape is unsupported. */
+size_t rz_workspace_bytes_loss(int64_t n_tok, int32_t n_resp, int32_t n_groups, int32_t d, int32_t V);
+
+/* Workspace bytes for rz_segment_loss; 0 if the sizes are unsupported. */
+size_t rz_workspace_bytes_segment_loss(int64_t n_tok, int32_t n_resp, int32_t n_groups);
+
+/*
+ * Token logprobs (the learner's own probability of each sampled token; page
+ * "vLLM says aligned kernels…", section "REINFORCE Zero removes the mismatch first").
+ *
+ *   H          [n_tok, d] bf16   final hidden states
+ *   W_head     [V, d]     bf16   LM head (nn.Linear weight layout, no bias)
+ *   token_ids  [n_tok]    int32  sampled tokens
+ *   lp_out     [n_tok]    fp32   out: lp[t] = z[t,y_t] - lse[t]
+ *   lse_out    [n_tok]    fp32   out, nullable: log-sum-exp of row t's logits
+ *
+ * Logits are never written to memory: a fused tensor-core kernel computes H W^T tile by
+ * tile and keeps an online log-sum-exp per row over fixed vocabulary segments, then a
+ * second kernel merges the segments in fixed order.  n_tok == 0 is a no-op.
+ */
+rz_status rz_token_logprobs(const rz_bf16* H, const rz_bf16* W_head, const int32_t* token_ids, int64_t n_tok,
+                            int32_t d, int32_t V, float* lp_out, float* lse_out, void* workspace,
+                            size_t ws_bytes, void* stream);
+
+/*
+ * Forward, REINFORCE Zero loss and backward in one call.
+ *
+ *   H, W_head, token_ids  as in rz_token_logprobs
+ *   lp_rollout [n_tok]      fp32   logprobs the rollout recorded for the same tokens
+ *   rewards    [n_resp]     fp32   one reward per response
+ *   seg_offsets[n_resp+1]   int64  response i owns tokens seg_offsets[i] .. seg_offsets[i+1]-1
+ *   group_ids  [n_resp]     int32  group of each response, in [0, n_groups)
+ *   loss       [1]          fp32   out: the scalar loss (to be minimised)
+ *   dH         [n_tok, d]   bf16   out: d loss / d H
+ *   dW         [V, d]       fp32   out: d loss / d W_head (overwritten, not accumulated)
+ *   lp_out     [n_tok]      fp32   out, nullable: token logprobs (bitwise equal to
+ *                                   rz_token_logprobs on the same rows)
+ *   kappa_out  [n_tok]      fp32   out, nullable: kappa_t = d loss / d lp_t
+ *
+ * The gradient of the ratio surrogate is exact; it equals the REINFORCE gradient with
+ * the ratio w_t held constant.  No clipping, no value model, no rejection gates.
+ * Requires n_tok >= 1, n_resp >= 1, n_groups >= 1.
+ */
+rz_status rz_loss_fwd_bwd(const rz_bf16* H, const rz_bf16* W_head, const int32_t* token_ids,
+                          const float* lp_rollout, const float* rewards, const int64_t* seg_offsets,
+                          const int32_t* group_ids, int64_t n_tok, int32_t n_resp, int32_t n_groups, int32_t d,
+                          int32_t V, float* loss, rz_bf16* dH, float* dW, float* lp_out, float* kappa_out,
+                          void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * The loss stage alone, from logprobs the caller already has (same definitions and the
+ * same kernels rz_loss_fwd_bwd uses after its forward).
+ *
+ *   lp, lp_rollout [n_tok] fp32;  rewards, seg_offsets, group_ids as above
+ *   loss       [1]     fp32  out
+ *   kappa_out  [n_tok] fp32  out: -A_i w_t / (N L_i)
+ *   w_out      [n_tok] fp32  out, nullable: unclipped ratio exp(lp - lp_rollout)
+ */
+rz_status rz_segment_loss(const float* lp, const float* lp_rollout, const float* rewards,
+                          const int64_t* seg_offsets, const int32_t* group_ids, int64_t n_tok, int32_t n_resp,
+                          int32_t n_groups, float* loss, float* kappa_out, float* w_out, void* workspace,
+                          size_t ws_bytes, void* stream);
+
+/* Kernel kinds reported per launch by rz_loss_fwd_bwd_timed. */
+#define RZ_KERNEL_LMHEAD_LSE 0    /* fused LM head + online log-sum-exp + gather (tensor cores) */
+#define RZ_KERNEL_MERGE_LSE 1     /* fixed-order merge of the vocabulary-segment partials       */
+#define RZ_KERNEL_RESPONSE_COEF 2 /* group means and -A_i / (N L_i)                             */
+#define RZ_KERNEL_TOKEN_KAPPA 3   /* ratio and kappa per token, per-block loss partials          */
+#define RZ_KERNEL_LOSS_FINAL 4    /* fixed-order sum of the loss partials                        */
+#define RZ_KERNEL_DZ 5            /* recomputed logits -> dZ chunk (tensor cores)                */
+#define RZ_KERNEL_DH 6            /* dH chunk = dZ W (tensor cores)                              */
+#define RZ_KERNEL_DW 7            /* dW (+)= dZ^T H (tensor cores)                               */
+
+/* Number of kernel launches one rz_loss_fwd_bwd call makes for n_tok tokens (0 if n_tok < 1). */
+int32_t rz_num_launches_loss(int64_t n_tok);
+
+/*
+ * rz_loss_fwd_bwd with per-launch timing: identical arguments and results, plus
+ *   launch_events [2*capacity] cudaEvent_t created by the caller (timing enabled); the
+ *                  library records events[2i] before and events[2i+1] after launch i
+ *                  on `stream`
+ *   launch_kinds  [capacity] host int32, out: RZ_KERNEL_* kind of launch i
+ *   n_launches    host int32, out: launches recorded (at most capacity)
+ * Launches past `capacity` still run but are not recorded.
+ */
+rz_status rz_loss_fwd_bwd_timed(const rz_bf16* H, const rz_bf16* W_head, const int32_t* token_ids,
+                                const float* lp_rollout, const float* rewards, const int64_t* seg_offsets,
+                                const int32_t* group_ids, int64_t n_tok, int32_t n_resp, int32_t n_groups,
+                                int32_t d, int32_t V, float* loss, rz_bf16* dH, float* dW, float* lp_out,
+                                float* kappa_out, void* workspace, size_t ws_bytes, void* stream,
+                                void* const* launch_events, int32_t* launch_kinds, int32_t capacity,
+                                int32_t* n_launches);
+
+/*
+ * Synchronises `stream`, then reads the device status word of `workspace`.
+ * Returns RZ_OK, RZ_ERR_DEVICE_CHECK (bad ids / segments / groups),
+ * RZ_ERR_DEVICE_TIMEOUT (a bounded wait gave up) or RZ_ERR_CUDA.
+ * bits_out (nullable) receives the raw RZ_DEV_* bits.
+ */
+rz_status rz_read_device_status(const void* workspace, void* stream, int32_t* bits_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RZ_H_ */

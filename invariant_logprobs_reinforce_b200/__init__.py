@@ -1,0 +1,255 @@
+"""Batch-invariant token logprobs and the REINFORCE Zero loss/gradient on B200.
+
+Thin Python binding over librz.so (include/rz.h).  Every step of the path runs in the
+library's CUDA kernels; this module only marshals torch tensors (device memory, streams)
+into the C calls, which keep their C names.  There is no CPU or PyTorch fallback: if
+librz.so is missing or no CUDA device is present, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+from .build import LIB as _LIB_PATH
+
+__all__ = [
+    "RZ_OK", "RZError", "lib", "rz_status_string", "rz_workspace_bytes_logprobs", "rz_workspace_bytes_loss",
+    "rz_workspace_bytes_segment_loss", "rz_token_logprobs", "rz_loss_fwd_bwd", "rz_segment_loss",
+    "rz_read_device_status", "EXPORTED_SYMBOLS",
+]
+
+RZ_OK = 0
+STATUS_NAMES = {
+    0: "RZ_OK", 1: "RZ_ERR_INVALID_ARG", 2: "RZ_ERR_UNSUPPORTED_SHAPE", 3: "RZ_ERR_WORKSPACE_TOO_SMALL",
+    4: "RZ_ERR_CUDA", 5: "RZ_ERR_DEVICE_CHECK", 6: "RZ_ERR_DEVICE_TIMEOUT",
+}
+EXPORTED_SYMBOLS = (
+    "rz_status_string", "rz_workspace_bytes_logprobs", "rz_workspace_bytes_loss", "rz_workspace_bytes_segment_loss",
+    "rz_token_logprobs", "rz_loss_fwd_bwd", "rz_segment_loss", "rz_read_device_status", "rz_num_launches_loss",
+    "rz_loss_fwd_bwd_timed",
+)
+KERNEL_KINDS = ("lmhead_lse", "merge_lse", "response_coef", "token_kappa", "loss_final", "dz", "dh", "dw")
+
+_lib = None
+
+
+class RZError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {STATUS_NAMES.get(code, code)}")
+        self.code = code
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded librz.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise ImportError(f"librz.so not built at {_LIB_PATH}; run invariant_logprobs_reinforce_b200.build.build()")
+        L = ctypes.CDLL(_LIB_PATH)
+        P, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+        L.rz_status_string.argtypes = [ctypes.c_int]
+        L.rz_status_string.restype = ctypes.c_char_p
+        L.rz_workspace_bytes_logprobs.argtypes = [i64, i32, i32]
+        L.rz_workspace_bytes_logprobs.restype = sz
+        L.rz_workspace_bytes_loss.argtypes = [i64, i32, i32, i32, i32]
+        L.rz_workspace_bytes_loss.restype = sz
+        L.rz_workspace_bytes_segment_loss.argtypes = [i64, i32, i32]
+        L.rz_workspace_bytes_segment_loss.restype = sz
+        L.rz_token_logprobs.argtypes = [P, P, P, i64, i32, i32, P, P, P, sz, P]
+        L.rz_token_logprobs.restype = ctypes.c_int
+        L.rz_loss_fwd_bwd.argtypes = [P, P, P, P, P, P, P, i64, i32, i32, i32, i32, P, P, P, P, P, P, sz, P]
+        L.rz_loss_fwd_bwd.restype = ctypes.c_int
+        L.rz_segment_loss.argtypes = [P, P, P, P, P, i64, i32, i32, P, P, P, P, sz, P]
+        L.rz_segment_loss.restype = ctypes.c_int
+        L.rz_loss_fwd_bwd_timed.argtypes = [P, P, P, P, P, P, P, i64, i32, i32, i32, i32, P, P, P, P, P, P, sz, P,
+                                             P, P, i32, ctypes.POINTER(ctypes.c_int32)]
+        L.rz_loss_fwd_bwd_timed.restype = ctypes.c_int
+        L.rz_num_launches_loss.argtypes = [i64]
+        L.rz_num_launches_loss.restype = i32
+        L.rz_read_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
+        L.rz_read_device_status.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def rz_status_string(code: int) -> str:
+    return lib().rz_status_string(code).decode()
+
+
+def rz_workspace_bytes_logprobs(n_tok: int, d: int, V: int) -> int:
+    return int(lib().rz_workspace_bytes_logprobs(n_tok, d, V))
+
+
+def rz_workspace_bytes_loss(n_tok: int, n_resp: int, n_groups: int, d: int, V: int) -> int:
+    return int(lib().rz_workspace_bytes_loss(n_tok, n_resp, n_groups, d, V))
+
+
+def rz_workspace_bytes_segment_loss(n_tok: int, n_resp: int, n_groups: int) -> int:
+    return int(lib().rz_workspace_bytes_segment_loss(n_tok, n_resp, n_groups))
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream):
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t, dtype, name, device=None):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _workspace(nbytes, workspace, device):
+    torch = _torch()
+    if workspace is None:
+        return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+    _need(workspace, torch.uint8, "workspace", device)
+    return workspace
+
+
+def _check(code, what):
+    if code != RZ_OK:
+        raise RZError(code, what)
+
+
+# ----------------------------------------------------------------------------- entry points
+
+def rz_token_logprobs(H, W_head, token_ids, lp_out=None, lse_out=None, workspace=None, stream=None,
+                      want_lse=True):
+    """Token logprobs of the sampled tokens (bf16 H [n,d], bf16 W [V,d], int32 ids [n]).
+
+    Returns (lp, lse) as fp32 CUDA tensors (lse is None when want_lse is False and no
+    lse_out is given).
+    """
+    torch = _torch()
+    _need(H, torch.bfloat16, "H")
+    dev = H.device
+    _need(W_head, torch.bfloat16, "W_head", dev)
+    _need(token_ids, torch.int32, "token_ids", dev)
+    n, d = H.shape
+    V = W_head.shape[0]
+    if W_head.shape[1] != d or token_ids.shape != (n,):
+        raise ValueError("shape mismatch")
+    lp = lp_out if lp_out is not None else torch.empty(n, dtype=torch.float32, device=dev)
+    lse = lse_out if lse_out is not None else (torch.empty(n, dtype=torch.float32, device=dev) if want_lse else None)
+    ws_bytes = rz_workspace_bytes_logprobs(n, d, V)
+    ws = _workspace(ws_bytes, workspace, dev)
+    code = lib().rz_token_logprobs(_ptr(H), _ptr(W_head), _ptr(token_ids), n, d, V, _ptr(lp), _ptr(lse), _ptr(ws),
+                                   ws.numel(), _stream_handle(stream))
+    _check(code, "rz_token_logprobs")
+    return lp, lse
+
+
+def rz_loss_fwd_bwd(H, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids, n_groups, loss=None,
+                    dH=None, dW=None, lp_out=None, kappa_out=None, workspace=None, stream=None, want_lp=True,
+                    want_kappa=True):
+    """Forward + REINFORCE Zero loss + backward.  Returns dict(loss, dH, dW, lp, kappa, workspace)."""
+    torch = _torch()
+    _need(H, torch.bfloat16, "H")
+    dev = H.device
+    _need(W_head, torch.bfloat16, "W_head", dev)
+    _need(token_ids, torch.int32, "token_ids", dev)
+    _need(lp_rollout, torch.float32, "lp_rollout", dev)
+    _need(rewards, torch.float32, "rewards", dev)
+    _need(seg_offsets, torch.int64, "seg_offsets", dev)
+    _need(group_ids, torch.int32, "group_ids", dev)
+    n, d = H.shape
+    V = W_head.shape[0]
+    R = rewards.shape[0]
+    if seg_offsets.shape != (R + 1,) or group_ids.shape != (R,) or lp_rollout.shape != (n,):
+        raise ValueError("shape mismatch")
+    loss = loss if loss is not None else torch.empty(1, dtype=torch.float32, device=dev)
+    dH = dH if dH is not None else torch.empty((n, d), dtype=torch.bfloat16, device=dev)
+    dW = dW if dW is not None else torch.empty((V, d), dtype=torch.float32, device=dev)
+    if lp_out is None and want_lp:
+        lp_out = torch.empty(n, dtype=torch.float32, device=dev)
+    if kappa_out is None and want_kappa:
+        kappa_out = torch.empty(n, dtype=torch.float32, device=dev)
+    ws_bytes = rz_workspace_bytes_loss(n, R, n_groups, d, V)
+    ws = _workspace(ws_bytes, workspace, dev)
+    code = lib().rz_loss_fwd_bwd(_ptr(H), _ptr(W_head), _ptr(token_ids), _ptr(lp_rollout), _ptr(rewards),
+                                 _ptr(seg_offsets), _ptr(group_ids), n, R, n_groups, d, V, _ptr(loss), _ptr(dH),
+                                 _ptr(dW), _ptr(lp_out), _ptr(kappa_out), _ptr(ws), ws.numel(),
+                                 _stream_handle(stream))
+    _check(code, "rz_loss_fwd_bwd")
+    return dict(loss=loss, dH=dH, dW=dW, lp=lp_out, kappa=kappa_out, workspace=ws)
+
+
+def rz_num_launches_loss(n_tok: int) -> int:
+    return int(lib().rz_num_launches_loss(n_tok))
+
+
+def rz_loss_fwd_bwd_timed(events, H, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids, n_groups,
+                          loss, dH, dW, lp_out, kappa_out, workspace, stream=None):
+    """rz_loss_fwd_bwd recording a CUDA event pair around every kernel launch.
+
+    ``events`` is a list of 2*capacity torch.cuda.Event(enable_timing=True) objects that
+    have been recorded once (so their handles exist).  Returns the kernel kind of each
+    recorded launch (indices into KERNEL_KINDS).
+    """
+    n, d = H.shape
+    V = W_head.shape[0]
+    R = rewards.shape[0]
+    cap = len(events) // 2
+    handles = (ctypes.c_void_p * (2 * cap))(*[ctypes.c_void_p(e.cuda_event) for e in events[:2 * cap]])
+    kinds = (ctypes.c_int32 * max(cap, 1))()
+    count = ctypes.c_int32(0)
+    code = lib().rz_loss_fwd_bwd_timed(_ptr(H), _ptr(W_head), _ptr(token_ids), _ptr(lp_rollout), _ptr(rewards),
+                                       _ptr(seg_offsets), _ptr(group_ids), n, R, n_groups, d, V, _ptr(loss), _ptr(dH),
+                                       _ptr(dW), _ptr(lp_out), _ptr(kappa_out), _ptr(workspace), workspace.numel(),
+                                       _stream_handle(stream), handles, kinds, cap, ctypes.byref(count))
+    _check(code, "rz_loss_fwd_bwd_timed")
+    return [int(kinds[i]) for i in range(count.value)]
+
+
+def rz_segment_loss(lp, lp_rollout, rewards, seg_offsets, group_ids, n_groups, loss=None, kappa_out=None,
+                    w_out=None, want_w=False, workspace=None, stream=None):
+    """The loss stage alone from given logprobs.  Returns dict(loss, kappa, w, workspace)."""
+    torch = _torch()
+    _need(lp, torch.float32, "lp")
+    dev = lp.device
+    _need(lp_rollout, torch.float32, "lp_rollout", dev)
+    _need(rewards, torch.float32, "rewards", dev)
+    _need(seg_offsets, torch.int64, "seg_offsets", dev)
+    _need(group_ids, torch.int32, "group_ids", dev)
+    n = lp.shape[0]
+    R = rewards.shape[0]
+    loss = loss if loss is not None else torch.empty(1, dtype=torch.float32, device=dev)
+    kappa_out = kappa_out if kappa_out is not None else torch.empty(n, dtype=torch.float32, device=dev)
+    if w_out is None and want_w:
+        w_out = torch.empty(n, dtype=torch.float32, device=dev)
+    ws = _workspace(rz_workspace_bytes_segment_loss(n, R, n_groups), workspace, dev)
+    code = lib().rz_segment_loss(_ptr(lp), _ptr(lp_rollout), _ptr(rewards), _ptr(seg_offsets), _ptr(group_ids), n,
+                                 R, n_groups, _ptr(loss), _ptr(kappa_out), _ptr(w_out), _ptr(ws), ws.numel(),
+                                 _stream_handle(stream))
+    _check(code, "rz_segment_loss")
+    return dict(loss=loss, kappa=kappa_out, w=w_out, workspace=ws)
+
+
+def rz_read_device_status(workspace, stream=None):
+    """Synchronise the stream and return (status code, raw RZ_DEV_* bits) of a workspace."""
+    bits = ctypes.c_int32(0)
+    code = lib().rz_read_device_status(_ptr(workspace), _stream_handle(stream), ctypes.byref(bits))
+    return int(code), int(bits.value)

@@ -1,0 +1,456 @@
+// rz_api.cu -- the C ABI declared in include/rz.h: argument checks, workspace carving,
+// TMA descriptor creation and the launch sequence of each entry point.
+//
+// Launch sequence of rz_loss_fwd_bwd (all on the caller's stream, no host sync):
+//   1. forward  : fused LM head + online log-sum-exp per (128-row block, 2048-column
+//                 vocabulary segment) -> per-segment partials; merge -> lp, lse
+//   2. loss     : per-response coefficient -A_i/(N L_i); per-token kappa and ratio; loss
+//   3. backward : for each chunk of 16384 tokens, in order:
+//                 dZ chunk (recomputed logits, bf16)  ->  dH rows = dZ W  ->  dW (+)= dZ^T H
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/rz.h"
+#include "rz_kernels.cuh"
+
+namespace rz {
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr int kMaxDevices = 64;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool shape_ok(int32_t d, int32_t V) { return d >= 64 && d <= 32768 && d % 64 == 0 && V >= 1; }
+
+int num_segments(int32_t V) { return static_cast<int>(ceil_div(V, kSegWidth)); }
+
+int64_t padded_vocab(int32_t V) { return align_up(static_cast<size_t>(V), 8); }
+
+// Workspace layout (byte offsets from the workspace base, each 256-byte aligned).
+struct Layout {
+  size_t status = 0;
+  size_t part_m = 0, part_s = 0, zy = 0;  // forward partials
+  size_t lp = 0, lse = 0, kappa = 0;      // per-token scratch
+  size_t coef = 0, gsum = 0, gcnt = 0, bsum = 0;
+  size_t dz = 0;
+  size_t total = 0;
+};
+
+int kappa_blocks(int64_t n) {
+  return static_cast<int>(ceil_div(n, static_cast<int64_t>(kKappaThreads) * kKappaTokensPerThread));
+}
+
+Layout make_layout(int64_t n, int32_t R, int32_t G, int32_t d, int32_t V, bool fwd, bool loss, bool bwd) {
+  Layout L;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, kAlign);
+    return at;
+  };
+  L.status = take(16);
+  if (fwd) {
+    const int S = num_segments(V);
+    L.part_m = take(sizeof(float) * static_cast<size_t>(S) * n);
+    L.part_s = take(sizeof(float) * static_cast<size_t>(S) * n);
+    L.zy = take(sizeof(float) * n);
+  }
+  if (loss) {
+    L.lp = take(sizeof(float) * n);
+    L.lse = take(sizeof(float) * n);
+    L.kappa = take(sizeof(float) * n);
+    L.coef = take(sizeof(float) * R);
+    L.gsum = take(sizeof(double) * G);
+    L.gcnt = take(sizeof(int) * G);
+    L.bsum = take(sizeof(double) * kappa_blocks(n));
+  }
+  if (bwd) {
+    const int64_t rows = std::min<int64_t>(align_up(n, BM), kChunkTokens);
+    L.dz = take(sizeof(uint16_t) * static_cast<size_t>(rows) * padded_vocab(V));
+  }
+  (void)d;
+  L.total = off;
+  return L;
+}
+
+template <class T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+// ---------------------------------------------------------------- driver entry point
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2D bf16 tensor map: dims {inner, outer}, row stride in bytes, box {64, box_outer},
+// 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_stride_bytes,
+              uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {64, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- launch recorder
+
+// Optional per-launch CUDA events (rz_loss_fwd_bwd_timed): an event pair around each
+// kernel launch, in launch order, with the kernel kind of each launch.
+struct Recorder {
+  cudaEvent_t* events;  // [2 * cap]
+  int32_t* kinds;       // [cap]
+  int32_t cap;
+  int32_t count;
+  bool open;
+};
+
+void rec_begin(Recorder* r, int kind, cudaStream_t s) {
+  if (r == nullptr) return;
+  r->open = r->count < r->cap;
+  if (!r->open) return;
+  r->kinds[r->count] = kind;
+  cudaEventRecord(r->events[2 * r->count], s);
+}
+
+void rec_end(Recorder* r, cudaStream_t s) {
+  if (r == nullptr || !r->open) return;
+  cudaEventRecord(r->events[2 * r->count + 1], s);
+  ++r->count;
+  r->open = false;
+}
+
+// ---------------------------------------------------------------- launches
+
+int sm_count() {
+  static int cache[kMaxDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev < kMaxDevices && cache[dev] > 0) return cache[dev];
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev < kMaxDevices) cache[dev] = sms;
+  return sms;
+}
+
+template <bool A_MN, bool B_MN, class Epi>
+cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmSched& s, const OperandPos& p,
+                        const Epi& e, int* status, cudaStream_t stream) {
+  auto kernel = gemm_tc_kernel<A_MN, B_MN, Epi>;
+  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes);
+  if (err != cudaSuccess) return err;
+  const int sms = sm_count();
+  if (sms <= 0) return cudaErrorInvalidDevice;
+  const int grid = std::max(1, std::min(s.num_units, sms));
+  kernel<<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(a, b, s, p, e, status);
+  return cudaGetLastError();
+}
+
+GemmSched make_sched(int64_t m_rows, int64_t n_cols, int tiles_per_unit, int group_m, int64_t k) {
+  GemmSched s;
+  s.m_blocks = static_cast<int>(ceil_div(m_rows, BM));
+  s.n_tiles = static_cast<int>(ceil_div(n_cols, BN));
+  s.tiles_per_unit = tiles_per_unit;
+  s.units_n = static_cast<int>(ceil_div(s.n_tiles, tiles_per_unit));
+  s.group_m = std::max(1, std::min(group_m, s.m_blocks));
+  s.num_units = s.m_blocks * s.units_n;
+  s.num_kb = static_cast<int>(ceil_div(k, BK));
+  return s;
+}
+
+// Forward over all n rows: partials, then merge into lp (and lse if requested).
+rz_status run_forward(const rz_bf16* H, const rz_bf16* W, const int32_t* ids, int64_t n, int32_t d, int32_t V,
+                      float* lp, float* lse, void* ws, const Layout& L, cudaStream_t stream, Recorder* rec) {
+  int* status = at<int>(ws, L.status);
+  CUtensorMap mH, mW;
+  if (!make_map(&mH, H, d, n, static_cast<uint64_t>(d) * 2, BM)) return RZ_ERR_CUDA;
+  if (!make_map(&mW, W, d, V, static_cast<uint64_t>(d) * 2, BN)) return RZ_ERR_CUDA;
+  const GemmSched s = make_sched(n, V, kSegTiles, 32, d);
+  EpiLse e;
+  e.ids = ids;
+  e.n = n;
+  e.V = V;
+  e.part_m = at<float>(ws, L.part_m);
+  e.part_s = at<float>(ws, L.part_s);
+  e.zy = at<float>(ws, L.zy);
+  const OperandPos pos{0, 0, 0, 0};
+  rec_begin(rec, RZ_KERNEL_LMHEAD_LSE, stream);
+  if (launch_gemm<false, false>(mH, mW, s, pos, e, status, stream) != cudaSuccess) return RZ_ERR_CUDA;
+  rec_end(rec, stream);
+  const int threads = 256;
+  rec_begin(rec, RZ_KERNEL_MERGE_LSE, stream);
+  merge_lse_kernel<<<static_cast<unsigned>(ceil_div(n, threads)), threads, 0, stream>>>(
+      e.part_m, e.part_s, e.zy, ids, n, V, num_segments(V), lp, lse, status);
+  if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
+  rec_end(rec, stream);
+  return RZ_OK;
+}
+
+rz_status run_loss(const float* lp, const float* lp_roll, const float* rewards, const int64_t* off,
+                   const int32_t* gid, int64_t n, int32_t R, int32_t G, float* loss, float* kappa, float* w_out,
+                   void* ws, const Layout& L, cudaStream_t stream, Recorder* rec) {
+  int* status = at<int>(ws, L.status);
+  float* coef = at<float>(ws, L.coef);
+  rec_begin(rec, RZ_KERNEL_RESPONSE_COEF, stream);
+  response_coef_kernel<<<1, 1024, 0, stream>>>(rewards, off, gid, R, G, n, at<double>(ws, L.gsum),
+                                               at<int>(ws, L.gcnt), coef, status);
+  if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
+  rec_end(rec, stream);
+  const int nb = kappa_blocks(n);
+  const int vec_ok = aligned(lp, 16) && aligned(lp_roll, 16) && aligned(kappa, 16) &&
+                     (w_out == nullptr || aligned(w_out, 16));
+  rec_begin(rec, RZ_KERNEL_TOKEN_KAPPA, stream);
+  token_kappa_kernel<<<nb, kKappaThreads, 0, stream>>>(lp, lp_roll, off, R, coef, n, vec_ok, kappa, w_out,
+                                                       at<double>(ws, L.bsum));
+  if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
+  rec_end(rec, stream);
+  rec_begin(rec, RZ_KERNEL_LOSS_FINAL, stream);
+  loss_final_kernel<<<1, 1024, 0, stream>>>(at<double>(ws, L.bsum), nb, loss);
+  if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
+  rec_end(rec, stream);
+  return RZ_OK;
+}
+
+rz_status run_backward(const rz_bf16* H, const rz_bf16* W, const int32_t* ids, int64_t n, int32_t d, int32_t V,
+                       const float* lse, const float* kappa, rz_bf16* dH, float* dW, void* ws, const Layout& L,
+                       cudaStream_t stream, Recorder* rec) {
+  int* status = at<int>(ws, L.status);
+  __nv_bfloat16* dz = at<__nv_bfloat16>(ws, L.dz);
+  const int64_t ldz = padded_vocab(V);
+  CUtensorMap mWk, mWmn;
+  if (!make_map(&mWk, W, d, V, static_cast<uint64_t>(d) * 2, BN)) return RZ_ERR_CUDA;
+  if (!make_map(&mWmn, W, d, V, static_cast<uint64_t>(d) * 2, 64)) return RZ_ERR_CUDA;
+  for (int64_t c0 = 0; c0 < n; c0 += kChunkTokens) {
+    const int64_t rows = std::min<int64_t>(kChunkTokens, n - c0);
+    // rows of H past the chunk read as zeros, so no other chunk's data enters it
+    CUtensorMap mHk, mHmn, mDzK, mDzMn;
+    if (!make_map(&mHk, H, d, c0 + rows, static_cast<uint64_t>(d) * 2, BM)) return RZ_ERR_CUDA;
+    if (!make_map(&mHmn, H, d, c0 + rows, static_cast<uint64_t>(d) * 2, 64)) return RZ_ERR_CUDA;
+    if (!make_map(&mDzK, dz, V, rows, static_cast<uint64_t>(ldz) * 2, BM)) return RZ_ERR_CUDA;
+    if (!make_map(&mDzMn, dz, V, rows, static_cast<uint64_t>(ldz) * 2, 64)) return RZ_ERR_CUDA;
+
+    // dZ chunk: A = H rows (K-major), B = W (K-major)
+    {
+      EpiDz e;
+      e.ids = ids + c0;
+      e.lse = lse + c0;
+      e.kappa = kappa + c0;
+      e.rows = rows;
+      e.V = V;
+      e.ldz = ldz;
+      e.dz = dz;
+      const GemmSched s = make_sched(rows, V, 1, 32, d);
+      const OperandPos pos{static_cast<int>(c0), 0, 0, 0};
+      rec_begin(rec, RZ_KERNEL_DZ, stream);
+      if (launch_gemm<false, false>(mHk, mWk, s, pos, e, status, stream) != cudaSuccess) return RZ_ERR_CUDA;
+      rec_end(rec, stream);
+    }
+    // dH chunk = dZ W: A = dZ (K-major, K = V), B = W (MN-major: d contiguous)
+    {
+      EpiStoreBf16 e;
+      e.out = reinterpret_cast<__nv_bfloat16*>(dH) + c0 * d;
+      e.ld = d;
+      e.rows = rows;
+      e.ncols = d;
+      const GemmSched s = make_sched(rows, d, 1, 1, V);
+      const OperandPos pos{0, 0, 0, 0};
+      rec_begin(rec, RZ_KERNEL_DH, stream);
+      if (launch_gemm<false, true>(mDzK, mWmn, s, pos, e, status, stream) != cudaSuccess) return RZ_ERR_CUDA;
+      rec_end(rec, stream);
+    }
+    // dW (+)= dZ^T H: A = dZ^T (MN-major: V contiguous), B = H chunk (MN-major: d contiguous)
+    {
+      EpiAccF32 e;
+      e.out = dW;
+      e.ld = d;
+      e.rows = V;
+      e.ncols = d;
+      e.accumulate = c0 > 0 ? 1 : 0;
+      const GemmSched s = make_sched(V, d, 1, 1, rows);
+      const OperandPos pos{0, 0, 0, static_cast<int>(c0)};
+      rec_begin(rec, RZ_KERNEL_DW, stream);
+      if (launch_gemm<true, true>(mDzMn, mHmn, s, pos, e, status, stream) != cudaSuccess) return RZ_ERR_CUDA;
+      rec_end(rec, stream);
+    }
+  }
+  return RZ_OK;
+}
+
+}  // namespace
+}  // namespace rz
+
+using namespace rz;
+
+extern "C" {
+#define RZ_API __attribute__((visibility("default")))
+
+RZ_API const char* rz_status_string(rz_status s) {
+  switch (s) {
+    case RZ_OK: return "RZ_OK";
+    case RZ_ERR_INVALID_ARG: return "RZ_ERR_INVALID_ARG";
+    case RZ_ERR_UNSUPPORTED_SHAPE: return "RZ_ERR_UNSUPPORTED_SHAPE";
+    case RZ_ERR_WORKSPACE_TOO_SMALL: return "RZ_ERR_WORKSPACE_TOO_SMALL";
+    case RZ_ERR_CUDA: return "RZ_ERR_CUDA";
+    case RZ_ERR_DEVICE_CHECK: return "RZ_ERR_DEVICE_CHECK";
+    case RZ_ERR_DEVICE_TIMEOUT: return "RZ_ERR_DEVICE_TIMEOUT";
+  }
+  return "RZ_UNKNOWN_STATUS";
+}
+
+RZ_API size_t rz_workspace_bytes_logprobs(int64_t n_tok, int32_t d, int32_t V) {
+  if (n_tok < 0 || n_tok >= (int64_t{1} << 31) || !shape_ok(d, V)) return 0;
+  return make_layout(n_tok, 0, 0, d, V, true, false, false).total;
+}
+
+RZ_API size_t rz_workspace_bytes_loss(int64_t n_tok, int32_t n_resp, int32_t n_groups, int32_t d, int32_t V) {
+  if (n_tok < 1 || n_tok >= (int64_t{1} << 31) || n_resp < 1 || n_groups < 1 || !shape_ok(d, V)) return 0;
+  return make_layout(n_tok, n_resp, n_groups, d, V, true, true, true).total;
+}
+
+RZ_API size_t rz_workspace_bytes_segment_loss(int64_t n_tok, int32_t n_resp, int32_t n_groups) {
+  if (n_tok < 1 || n_tok >= (int64_t{1} << 31) || n_resp < 1 || n_groups < 1) return 0;
+  return make_layout(n_tok, n_resp, n_groups, 64, 1, false, true, false).total;
+}
+
+RZ_API rz_status rz_token_logprobs(const rz_bf16* H, const rz_bf16* W_head, const int32_t* token_ids, int64_t n_tok,
+                            int32_t d, int32_t V, float* lp_out, float* lse_out, void* workspace,
+                            size_t ws_bytes, void* stream) {
+  if (n_tok < 0 || n_tok >= (int64_t{1} << 31)) return RZ_ERR_INVALID_ARG;
+  if (!shape_ok(d, V)) return RZ_ERR_UNSUPPORTED_SHAPE;
+  if (n_tok == 0) return RZ_OK;
+  if (!H || !W_head || !token_ids || !lp_out || !workspace) return RZ_ERR_INVALID_ARG;
+  if (!aligned(H, 16) || !aligned(W_head, 16) || !aligned(token_ids, 4) || !aligned(lp_out, 4) ||
+      (lse_out && !aligned(lse_out, 4)) || !aligned(workspace, kAlign))
+    return RZ_ERR_INVALID_ARG;
+  const Layout L = make_layout(n_tok, 0, 0, d, V, true, false, false);
+  if (ws_bytes < L.total) return RZ_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(at<int>(workspace, L.status), 0, sizeof(int), st) != cudaSuccess) return RZ_ERR_CUDA;
+  return run_forward(H, W_head, token_ids, n_tok, d, V, lp_out, lse_out, workspace, L, st, nullptr);
+}
+
+RZ_API rz_status rz_segment_loss(const float* lp, const float* lp_rollout, const float* rewards,
+                          const int64_t* seg_offsets, const int32_t* group_ids, int64_t n_tok, int32_t n_resp,
+                          int32_t n_groups, float* loss, float* kappa_out, float* w_out, void* workspace,
+                          size_t ws_bytes, void* stream) {
+  if (n_tok < 1 || n_tok >= (int64_t{1} << 31) || n_resp < 1 || n_groups < 1) return RZ_ERR_INVALID_ARG;
+  if (!lp || !lp_rollout || !rewards || !seg_offsets || !group_ids || !loss || !kappa_out || !workspace)
+    return RZ_ERR_INVALID_ARG;
+  if (!aligned(lp, 4) || !aligned(lp_rollout, 4) || !aligned(rewards, 4) || !aligned(seg_offsets, 8) ||
+      !aligned(group_ids, 4) || !aligned(loss, 4) || !aligned(kappa_out, 4) || (w_out && !aligned(w_out, 4)) ||
+      !aligned(workspace, kAlign))
+    return RZ_ERR_INVALID_ARG;
+  const Layout L = make_layout(n_tok, n_resp, n_groups, 64, 1, false, true, false);
+  if (ws_bytes < L.total) return RZ_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(at<int>(workspace, L.status), 0, sizeof(int), st) != cudaSuccess) return RZ_ERR_CUDA;
+  return run_loss(lp, lp_rollout, rewards, seg_offsets, group_ids, n_tok, n_resp, n_groups, loss, kappa_out, w_out,
+                  workspace, L, st, nullptr);
+}
+
+}  // extern "C"
+
+namespace {
+rz_status loss_fwd_bwd_impl(const rz_bf16* H, const rz_bf16* W_head, const int32_t* token_ids,
+                          const float* lp_rollout, const float* rewards, const int64_t* seg_offsets,
+                          const int32_t* group_ids, int64_t n_tok, int32_t n_resp, int32_t n_groups, int32_t d,
+                          int32_t V, float* loss, rz_bf16* dH, float* dW, float* lp_out, float* kappa_out,
+                          void* workspace, size_t ws_bytes, void* stream, Recorder* rec) {
+  if (n_tok < 1 || n_tok >= (int64_t{1} << 31) || n_resp < 1 || n_groups < 1) return RZ_ERR_INVALID_ARG;
+  if (!shape_ok(d, V)) return RZ_ERR_UNSUPPORTED_SHAPE;
+  if (!H || !W_head || !token_ids || !lp_rollout || !rewards || !seg_offsets || !group_ids || !loss || !dH ||
+      !dW || !workspace)
+    return RZ_ERR_INVALID_ARG;
+  if (!aligned(H, 16) || !aligned(W_head, 16) || !aligned(dH, 16) || !aligned(dW, 16) || !aligned(token_ids, 4) ||
+      !aligned(lp_rollout, 4) || !aligned(rewards, 4) || !aligned(seg_offsets, 8) || !aligned(group_ids, 4) ||
+      !aligned(loss, 4) || (lp_out && !aligned(lp_out, 4)) || (kappa_out && !aligned(kappa_out, 4)) ||
+      !aligned(workspace, kAlign))
+    return RZ_ERR_INVALID_ARG;
+  const Layout L = make_layout(n_tok, n_resp, n_groups, d, V, true, true, true);
+  if (ws_bytes < L.total) return RZ_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(at<int>(workspace, L.status), 0, sizeof(int), st) != cudaSuccess) return RZ_ERR_CUDA;
+  float* lp = lp_out ? lp_out : at<float>(workspace, L.lp);
+  float* lse = at<float>(workspace, L.lse);
+  float* kappa = kappa_out ? kappa_out : at<float>(workspace, L.kappa);
+  rz_status r = run_forward(H, W_head, token_ids, n_tok, d, V, lp, lse, workspace, L, st, rec);
+  if (r != RZ_OK) return r;
+  r = run_loss(lp, lp_rollout, rewards, seg_offsets, group_ids, n_tok, n_resp, n_groups, loss, kappa, nullptr,
+               workspace, L, st, rec);
+  if (r != RZ_OK) return r;
+  return run_backward(H, W_head, token_ids, n_tok, d, V, lse, kappa, dH, dW, workspace, L, st, rec);
+}
+
+}  // namespace
+
+extern "C" {
+
+RZ_API rz_status rz_loss_fwd_bwd(const rz_bf16* H, const rz_bf16* W_head, const int32_t* token_ids,
+                                 const float* lp_rollout, const float* rewards, const int64_t* seg_offsets,
+                                 const int32_t* group_ids, int64_t n_tok, int32_t n_resp, int32_t n_groups,
+                                 int32_t d, int32_t V, float* loss, rz_bf16* dH, float* dW, float* lp_out,
+                                 float* kappa_out, void* workspace, size_t ws_bytes, void* stream) {
+  return loss_fwd_bwd_impl(H, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids, n_tok, n_resp,
+                           n_groups, d, V, loss, dH, dW, lp_out, kappa_out, workspace, ws_bytes, stream, nullptr);
+}
+
+RZ_API int32_t rz_num_launches_loss(int64_t n_tok) {
+  if (n_tok < 1) return 0;
+  return static_cast<int32_t>(5 + 3 * ceil_div(n_tok, kChunkTokens));
+}
+
+RZ_API rz_status rz_loss_fwd_bwd_timed(const rz_bf16* H, const rz_bf16* W_head, const int32_t* token_ids,
+                                       const float* lp_rollout, const float* rewards, const int64_t* seg_offsets,
+                                       const int32_t* group_ids, int64_t n_tok, int32_t n_resp, int32_t n_groups,
+                                       int32_t d, int32_t V, float* loss, rz_bf16* dH, float* dW, float* lp_out,
+                                       float* kappa_out, void* workspace, size_t ws_bytes, void* stream,
+                                       void* const* launch_events, int32_t* launch_kinds, int32_t capacity,
+                                       int32_t* n_launches) {
+  if (!launch_events || !launch_kinds || !n_launches || capacity < 0) return RZ_ERR_INVALID_ARG;
+  Recorder rec{reinterpret_cast<cudaEvent_t*>(const_cast<void**>(launch_events)), launch_kinds, capacity, 0, false};
+  const rz_status r = loss_fwd_bwd_impl(H, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids, n_tok,
+                                        n_resp, n_groups, d, V, loss, dH, dW, lp_out, kappa_out, workspace, ws_bytes,
+                                        stream, &rec);
+  *n_launches = rec.count;
+  return r;
+}
+
+RZ_API rz_status rz_read_device_status(const void* workspace, void* stream, int32_t* bits_out) {
+  if (!workspace) return RZ_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return RZ_ERR_CUDA;
+  int32_t bits = 0;
+  if (cudaMemcpy(&bits, workspace, sizeof(bits), cudaMemcpyDeviceToHost) != cudaSuccess) return RZ_ERR_CUDA;
+  if (bits_out) *bits_out = bits;
+  if (bits & RZ_DEV_WAIT_TIMEOUT) return RZ_ERR_DEVICE_TIMEOUT;
+  if (bits) return RZ_ERR_DEVICE_CHECK;
+  return RZ_OK;
+}
+
+}  // extern "C"
