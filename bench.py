@@ -1,0 +1,441 @@
+"""Benchmark of the REINFORCE Zero logprob / loss / gradient path on B200.
+
+One step = one rz_loss_fwd_bwd call over one batch of the Qwen3-4B-shaped workload
+(d=2560, V=151936, 64 groups x 8 responses, lengths log-uniform 128..2048 tokens):
+fused LM head + online log-sum-exp forward, the REINFORCE Zero loss stage, and the
+backward (dZ chunks, dH, dW).  Prints ONE JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl rz|reference] [--workload NAME]
+
+--impl reference times the fp64 CPU oracle (the only reference this path has) on host
+cores over a bounded sample of the same workload.  With N > 1 (torchrun) every rank runs
+an independent replica (the path does not shard); timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import io
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fwd+bwd logprob/loss tokens/s on 1 B200"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="rz", choices=["rz", "reference"])
+    ap.add_argument("--workload", default="qwen3_4b")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.idx)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r for r in csv.reader(io.StringIO(out)) if len(r) >= 9]
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                smax.append(float(r[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(smax)), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- rz arm
+
+def algorithmic_flops(kind: str, rows: int, d: int, V: int) -> float:
+    """Dense contraction FLOPs of one launch: 2 * rows * d * V for each tensor-core kernel."""
+    if kind in ("lmhead_lse", "dz", "dh", "dw"):
+        return 2.0 * rows * d * V
+    return 0.0
+
+
+def launch_rows(kinds, n_tok, chunk=16384):
+    """Rows (tokens) each recorded launch covers, in launch order."""
+    rows = []
+    c0 = 0
+    for k in kinds:
+        if k in ("lmhead_lse", "merge_lse", "response_coef", "token_kappa", "loss_final"):
+            rows.append(n_tok)
+        else:
+            r = min(chunk, n_tok - c0)
+            rows.append(r)
+            if k == "dw":
+                c0 += chunk
+    return rows
+
+
+def traffic_for(kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the current source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        with open(p) as f:
+            rec = json.load(f)
+        from invariant_logprobs_reinforce_b200.build import source_digest
+        if rec.get("source_digest") != source_digest():
+            return None
+        ent = rec.get("kernels", {}).get(kernel)
+        return None if ent is None else ent.get("bytes_per_launch")
+    except Exception:
+        return None
+
+
+def run_rz(args, rank, world, local_rank):
+    import torch
+    import workloads as wl
+    import invariant_logprobs_reinforce_b200 as rz
+    from invariant_logprobs_reinforce_b200 import build as rzbuild
+
+    rzbuild.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream()
+    cfg = wl.CONFIGS[args.workload]
+    prob = wl.full_config(args.workload, device=str(dev))
+    seg = prob.seg
+    n, d, V = prob.n_tok, prob.d, prob.V
+    R, G = seg.n_resp, seg.n_groups
+    H, W, ids = prob.H, prob.W, prob.ids
+    rewards = torch.from_numpy(seg.rewards).to(dev)
+    off = torch.from_numpy(seg.seg_offsets).to(dev)
+    gid = torch.from_numpy(seg.group_ids).to(dev)
+
+    # recorded rollout logprobs = learner logprobs + the workload's weight-lag noise
+    lp0, _ = rz.rz_token_logprobs(H, W, ids)
+    torch.cuda.synchronize()
+    lp_roll = torch.from_numpy(wl.rollout_logprobs_with_lag(lp0.cpu().numpy(), prob.noise, prob.seed)).to(dev)
+
+    ws = torch.empty(rz.rz_workspace_bytes_loss(n, R, G, d, V), dtype=torch.uint8, device=dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    dH = torch.empty((n, d), dtype=torch.bfloat16, device=dev)
+    dW = torch.empty((V, d), dtype=torch.float32, device=dev)
+    lp = torch.empty(n, dtype=torch.float32, device=dev)
+    kappa = torch.empty(n, dtype=torch.float32, device=dev)
+    n_launch = rz.rz_num_launches_loss(n)
+    events = [torch.cuda.Event(enable_timing=True) for _ in range(2 * n_launch * (args.steps + 1))]
+    for e in events:
+        e.record(stream)  # materialise the handles
+    torch.cuda.synchronize()
+
+    def step(ev=None):
+        if ev is None:
+            rz.rz_loss_fwd_bwd(H, W, ids, lp_roll, rewards, off, gid, G, loss=loss, dH=dH, dW=dW, lp_out=lp,
+                               kappa_out=kappa, workspace=ws, stream=stream)
+            return None
+        return rz.rz_loss_fwd_bwd_timed(ev, H, W, ids, lp_roll, rewards, off, gid, G, loss, dH, dW, lp, kappa, ws,
+                                        stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    code, bits = rz.rz_read_device_status(ws)
+    if code != 0:
+        raise RuntimeError(f"device status {code} bits {bits}")
+
+    dist = world > 1
+    if dist:
+        import torch.distributed as tdist
+    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local_rank)
+    clocks.start()
+    time.sleep(0.5)
+    if dist:
+        tdist.barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    all_kinds = []
+    for s in range(args.steps):
+        evs = events[2 * n_launch * s:2 * n_launch * (s + 1)]
+        kinds = step(evs)
+        all_kinds.append((evs, kinds))
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        tdist.barrier()
+    clk = clocks.stop()
+    ms = t_start.elapsed_time(t_end)
+    code, bits = rz.rz_read_device_status(ws)
+    if code != 0:
+        raise RuntimeError(f"device status {code} bits {bits}")
+
+    # per-kernel durations from the recorded event pairs
+    per = {}
+    for evs, kinds in all_kinds:
+        names = [rz.KERNEL_KINDS[k] for k in kinds]
+        rows = launch_rows(names, n)
+        for i, (name, r) in enumerate(zip(names, rows)):
+            t = evs[2 * i].elapsed_time(evs[2 * i + 1])
+            ent = per.setdefault(name, {"launches": 0, "ms": 0.0, "flops": 0.0})
+            ent["launches"] += 1
+            ent["ms"] += t
+            ent["flops"] += algorithmic_flops(name, r, d, V)
+    launches_total = sum(v["launches"] for v in per.values())
+
+    if dist:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # forward alone (rz_token_logprobs), same inputs
+    lpf = torch.empty(n, dtype=torch.float32, device=dev)
+    wsf = torch.empty(rz.rz_workspace_bytes_logprobs(n, d, V), dtype=torch.uint8, device=dev)
+    for _ in range(2):
+        rz.rz_token_logprobs(H, W, ids, lp_out=lpf, workspace=wsf, stream=stream, want_lse=False)
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    fsteps = max(2, args.steps)
+    for _ in range(fsteps):
+        rz.rz_token_logprobs(H, W, ids, lp_out=lpf, workspace=wsf, stream=stream, want_lse=False)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    fwd_ms = f0.elapsed_time(f1) / fsteps
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(rz, torch, dev, stream, H, W, ids, lp_roll, rewards, off, gid, G, n, d, V, args)
+
+    peaks, peak_src = load_peaks()
+    peak_tflops = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    tens = {k: v for k, v in per.items() if v["flops"] > 0}
+    dom = max(tens, key=lambda k: tens[k]["ms"])
+    ach = tens[dom]["flops"] / (tens[dom]["ms"] * 1e-3) / 1e12
+    kernels = {k: {"launches": v["launches"] // args.steps, "ms_per_step": v["ms"] / args.steps,
+                   "share": v["ms"] / sum(x["ms"] for x in per.values()),
+                   **({"tflops": v["flops"] / (v["ms"] * 1e-3) / 1e12,
+                       "frac_of_peak": v["flops"] / (v["ms"] * 1e-3) / 1e12 / peak_tflops} if v["flops"] else {})}
+               for k, v in per.items()}
+    step_ms = ms / args.steps
+    tok_s = world * n / (step_ms * 1e-3)
+    return dict(
+        value=tok_s, ms_per_step=step_ms, n_tok=n, d=d, V=V, R=R, G=G, clocks=clk, kernels=kernels,
+        dominant=dom, achieved=ach, peak=peak_tflops, peak_src=peak_src, traffic=traffic_for(dom),
+        fwd_ms=fwd_ms, fwd_tok_s=world * n / (fwd_ms * 1e-3), launches=launches_total, e2e=e2e, cfg=cfg,
+    )
+
+
+def run_e2e(rz, torch, dev, stream, H, W, ids, lp_roll, rewards, off, gid, G, n, d, V, args):
+    """The same step through the public call with inputs in pinned host memory: H2D of every
+    input and D2H of the loss and logprobs inside the timed region."""
+    host = {k: t.cpu().pin_memory() for k, t in
+            dict(H=H, W=W, ids=ids, lp_roll=lp_roll, rewards=rewards, off=off, gid=gid).items()}
+    dbuf = {k: torch.empty_like(t, device=dev) for k, t in host.items()}
+    loss_h = torch.empty(1, dtype=torch.float32).pin_memory()
+    lp_h = torch.empty(n, dtype=torch.float32).pin_memory()
+    R = rewards.shape[0]
+    ws = torch.empty(rz.rz_workspace_bytes_loss(n, R, G, d, V), dtype=torch.uint8, device=dev)
+    out = dict(loss=torch.empty(1, dtype=torch.float32, device=dev),
+               dH=torch.empty((n, d), dtype=torch.bfloat16, device=dev),
+               dW=torch.empty((V, d), dtype=torch.float32, device=dev),
+               lp=torch.empty(n, dtype=torch.float32, device=dev))
+
+    def step():
+        for k in host:
+            dbuf[k].copy_(host[k], non_blocking=True)
+        rz.rz_loss_fwd_bwd(dbuf["H"], dbuf["W"], dbuf["ids"], dbuf["lp_roll"], dbuf["rewards"], dbuf["off"],
+                           dbuf["gid"], G, loss=out["loss"], dH=out["dH"], dW=out["dW"], lp_out=out["lp"],
+                           kappa_out=None, want_kappa=False, workspace=ws, stream=stream)
+        loss_h.copy_(out["loss"], non_blocking=True)
+        lp_h.copy_(out["lp"], non_blocking=True)
+
+    for _ in range(1):
+        step()
+    torch.cuda.synchronize()
+    steps = max(2, min(args.steps, 3))
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = loss_h.numel() * 4 + lp_h.numel() * 4
+    return {"value": n / (ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": ms}
+
+
+# --------------------------------------------------------------------------- CPU oracle
+
+def cpu_oracle_sample(workload: str, budget_s: float = 12.0):
+    """The fp64 oracle as it stands, fwd+loss+bwd on a bounded sub-batch of the workload's
+    shape (one group of two responses of k/2 tokens each, the workload's d and V)."""
+    import oracle
+    import workloads as wl
+    oracle.build()
+    cfg = wl.CONFIGS[workload]
+    d, V = cfg["d"], cfg["V"]
+    rng = np.random.Generator(np.random.PCG64(cfg["seed"] + 1))
+    W = wl.bf16_bits(rng.standard_normal((V, d), dtype=np.float32) * np.float32(1.0 / math.sqrt(d)))
+
+    def run(k):
+        H = wl.bf16_bits(rng.standard_normal((k, d), dtype=np.float32))
+        ids = rng.integers(0, V, size=k).astype(np.int32)
+        off = np.array([0, k // 2, k], np.int64)
+        lr = np.full(k, -12.0)
+        t0 = time.perf_counter()
+        oracle.loss_fwd_bwd(H, W, ids, lr, np.array([1.0, 0.0]), off, np.zeros(2, np.int32), 1)
+        return time.perf_counter() - t0
+
+    k = 2
+    t = run(k)
+    k2 = int(max(2, min(256, 2 * round(0.5 * k * budget_s / max(t, 1e-3)))))
+    t2 = run(k2)
+    return {"value": k2 / t2, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{k2} tokens of {workload} (2 responses x {k2 // 2} tokens, d={d}, V={V}): "
+                      f"fp64 lp, loss, dH and dW; {t2:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    import workloads as wl
+    cfg = wl.CONFIGS[args.workload]
+    budget = max(3.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    vals = []
+    last = None
+    for i in range(args.warmup + args.steps):
+        last = cpu_oracle_sample(args.workload, budget_s=budget)
+        if i >= args.warmup:
+            vals.append(last["value"])
+    v = float(np.mean(vals)) if vals else float(last["value"])
+    seg = wl.draw_segments(args.workload)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": seg.n_tok / v * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{args.workload}: d={cfg['d']}, V={cfg['V']}, n_tok={seg.n_tok}, "
+                               f"n_resp={seg.n_resp} (timed on a bounded token sample; tokens/s extrapolates "
+                               f"linearly, the cost is row-linear)"},
+        "cpu_baseline": dict(last, value=v),
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    return line
+
+
+# --------------------------------------------------------------------------- main
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
+
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(local_rank)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                 device_id=torch.device("cuda", local_rank))
+    res = run_rz(args, rank, world, local_rank)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_sample(args.workload)
+    if rank == 0:
+        cfg = res["cfg"]
+        frac = res["achieved"] / res["peak"]
+        line = {
+            "metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {
+                "workload": f"{args.workload}: d={res['d']}, V={res['V']}, {res['G']} groups x "
+                            f"{res['R'] // res['G']} responses, lengths {cfg['lengths'][0]} "
+                            f"{cfg['lengths'][1]}-{cfg['lengths'][2]}, n_tok={res['n_tok']} per GPU",
+                "n_tok": res["n_tok"], "d": res["d"], "V": res["V"], "n_resp": res["R"], "n_groups": res["G"],
+                "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                "l2": "inputs larger than L2 (H %.2f GB, W %.2f GB)" % (res["n_tok"] * res["d"] * 2 / 1e9,
+                                                                      res["V"] * res["d"] * 2 / 1e9),
+            },
+            "roofline": {"bound": "tensor", "kernel": res["dominant"], "achieved": res["achieved"],
+                         "peak": res["peak"], "unit": "TFLOP/s", "frac": frac, "traffic": res["traffic"],
+                         "peak_source": f"bf16_tflops_sustained of {res['peak_src']}"},
+            "tensor_frac_6dV": res["value"] / world * 6 * res["d"] * res["V"] / (res["peak"] * 1e12),
+            "fwd_only": {"tokens_per_s": res["fwd_tok_s"], "ms_per_step": res["fwd_ms"],
+                         "tensor_frac_2dV": res["fwd_tok_s"] / world * 2 * res["d"] * res["V"] / (res["peak"] * 1e12)},
+            "kernels": res["kernels"],
+            "gpu_launches": res["launches"],
+            "clocks": res["clocks"],
+            "e2e": res["e2e"],
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as tdist
+        tdist.barrier()
+        tdist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

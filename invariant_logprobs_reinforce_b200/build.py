@@ -50,3 +50,14 @@ if __name__ == "__main__":
     import sys
     build(force="--force" in sys.argv, verbose=True,
           extra_flags=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else [])
+
+
+def source_digest() -> str:
+    """sha256 over the CUDA sources and the public header (identifies a kernel build)."""
+    import hashlib
+    h = hashlib.sha256()
+    for p in deps():
+        h.update(os.path.basename(p).encode())
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
