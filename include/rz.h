@@ -167,6 +167,37 @@ rz_status rz_loss_fwd_bwd_timed(const rz_bf16* H, const rz_bf16* W_head, const i
                                 void* const* launch_events, int32_t* launch_kinds, int32_t capacity,
                                 int32_t* n_launches);
 
+/* Size of the library-owned scratch array used by rz_token_logprobs_noalloc (32 MiB). */
+#define RZ_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * rz_token_logprobs without a caller workspace and without any allocation.
+ *
+ * The pages have no counterpart to this call; it exists for callers that cannot
+ * allocate device memory: a rollout or serving engine that reserved nearly all of HBM
+ * for its KV cache at start-up and hands out only fixed buffers, a latency-critical
+ * loop where cudaMalloc/cudaFree could synchronise the device, or a plugin that receives
+ * device pointers from a host framework but has no access to its allocator.
+ *
+ * Arguments and results are those of rz_token_logprobs (same kernels, same bits), minus
+ * the workspace.  The scratch is a fixed array of RZ_NOALLOC_SCRATCH_BYTES inside the
+ * library, held by every GPU that loads the library until the process exits.  A call
+ * needs 256 + 4*n_tok*(2*ceil(V/2048) + 1) bytes of it (rounded up to 256-byte pieces):
+ * at V = 151936 that is about 55,000 tokens per call.  Larger calls return
+ * RZ_ERR_WORKSPACE_TOO_SMALL and enqueue nothing; split them into several calls.
+ *
+ * The first call on each device looks up the scratch address (cudaGetSymbolAddress)
+ * and caches it; make that first call before any stream capture begins.  All calls
+ * share the one array: calls whose GPU work can overlap (different streams, or
+ * different host threads) race on it and must be serialised by the caller.  Each call
+ * clears the scratch's status word; out-of-range token ids still give NaN logprobs,
+ * but the status word is internal (rz_read_device_status does not apply).  Nothing
+ * here calls cudaMalloc, cudaFree or any allocating routine.
+ */
+rz_status rz_token_logprobs_noalloc(const rz_bf16* H, const rz_bf16* W_head, const int32_t* token_ids,
+                                    int64_t n_tok, int32_t d, int32_t V, float* lp_out, float* lse_out,
+                                    void* stream);
+
 /*
  * Synchronises `stream`, then reads the device status word of `workspace`.
  * Returns RZ_OK, RZ_ERR_DEVICE_CHECK (bad ids / segments / groups),

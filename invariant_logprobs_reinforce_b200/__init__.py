@@ -26,7 +26,7 @@ STATUS_NAMES = {
 EXPORTED_SYMBOLS = (
     "rz_status_string", "rz_workspace_bytes_logprobs", "rz_workspace_bytes_loss", "rz_workspace_bytes_segment_loss",
     "rz_token_logprobs", "rz_loss_fwd_bwd", "rz_segment_loss", "rz_read_device_status", "rz_num_launches_loss",
-    "rz_loss_fwd_bwd_timed",
+    "rz_loss_fwd_bwd_timed", "rz_token_logprobs_noalloc",
 )
 KERNEL_KINDS = ("lmhead_lse", "merge_lse", "response_coef", "token_kappa", "loss_final", "dz", "dh", "dw")
 
@@ -66,6 +66,8 @@ def lib() -> ctypes.CDLL:
         L.rz_loss_fwd_bwd_timed.restype = ctypes.c_int
         L.rz_num_launches_loss.argtypes = [i64]
         L.rz_num_launches_loss.restype = i32
+        L.rz_token_logprobs_noalloc.argtypes = [P, P, P, i64, i32, i32, P, P, P]
+        L.rz_token_logprobs_noalloc.restype = ctypes.c_int
         L.rz_read_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
         L.rz_read_device_status.restype = ctypes.c_int
         _lib = L

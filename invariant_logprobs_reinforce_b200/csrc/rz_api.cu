@@ -441,6 +441,63 @@ RZ_API rz_status rz_loss_fwd_bwd_timed(const rz_bf16* H, const rz_bf16* W_head, 
   return r;
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------- allocation-free variant
+//
+// Scratch for rz_token_logprobs_noalloc: a fixed device array in this library's module,
+// so callers that cannot allocate device memory still get the forward.  Every device
+// that loads the library holds these RZ_NOALLOC_SCRATCH_BYTES until the process exits.
+// All calls share it, so calls whose GPU work overlaps (other streams, other threads)
+// race on it; the status word at its start is cleared by every call, and every other
+// byte a call reads has been written earlier in that same call.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[RZ_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+// Device address of g_noalloc_scratch on the current device.  Host code only sees a
+// host-side stand-in under that name, so the address is looked up once per device
+// (with that device current) and cached.
+rz_status noalloc_scratch(void** out) {
+  static void* addr[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return RZ_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return RZ_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return RZ_ERR_CUDA;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return RZ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+RZ_API rz_status rz_token_logprobs_noalloc(const rz_bf16* H, const rz_bf16* W_head, const int32_t* token_ids,
+                                           int64_t n_tok, int32_t d, int32_t V, float* lp_out, float* lse_out,
+                                           void* stream) {
+  if (n_tok < 0 || n_tok >= (int64_t{1} << 31)) return RZ_ERR_INVALID_ARG;
+  if (!shape_ok(d, V)) return RZ_ERR_UNSUPPORTED_SHAPE;
+  if (n_tok == 0) return RZ_OK;
+  if (!H || !W_head || !token_ids || !lp_out) return RZ_ERR_INVALID_ARG;
+  if (!aligned(H, 16) || !aligned(W_head, 16) || !aligned(token_ids, 4) || !aligned(lp_out, 4) ||
+      (lse_out && !aligned(lse_out, 4)))
+    return RZ_ERR_INVALID_ARG;
+  const Layout L = make_layout(n_tok, 0, 0, d, V, true, false, false);
+  if (L.total > static_cast<size_t>(RZ_NOALLOC_SCRATCH_BYTES)) return RZ_ERR_WORKSPACE_TOO_SMALL;
+  void* scratch = nullptr;
+  const rz_status r = noalloc_scratch(&scratch);
+  if (r != RZ_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(at<int>(scratch, L.status), 0, sizeof(int), st) != cudaSuccess) return RZ_ERR_CUDA;
+  return run_forward(H, W_head, token_ids, n_tok, d, V, lp_out, lse_out, scratch, L, st, nullptr);
+}
+
 RZ_API rz_status rz_read_device_status(const void* workspace, void* stream, int32_t* bits_out) {
   if (!workspace) return RZ_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
