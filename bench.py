@@ -42,6 +42,9 @@ def parse_args():
     ap.add_argument("--workload", default="qwen3_4b")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-loss-stage", action="store_true")
+    ap.add_argument("--n-tok-cap", type=int, default=None,
+                    help="keep only the leading whole groups that fit (small profiling cases)")
     return ap.parse_args()
 
 
@@ -154,7 +157,7 @@ def run_rz(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     stream = torch.cuda.current_stream()
     cfg = wl.CONFIGS[args.workload]
-    prob = wl.full_config(args.workload, device=str(dev))
+    prob = wl.full_config(args.workload, device=str(dev), n_tok_cap=args.n_tok_cap)
     seg = prob.seg
     n, d, V = prob.n_tok, prob.d, prob.V
     R, G = seg.n_resp, seg.n_groups
@@ -254,6 +257,10 @@ def run_rz(args, rank, world, local_rank):
     torch.cuda.synchronize()
     fwd_ms = f0.elapsed_time(f1) / fsteps
 
+    loss_stage = None
+    if not args.no_loss_stage:
+        loss_stage = run_loss_stage(rz, torch, dev, stream)
+
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(rz, torch, dev, stream, H, W, ids, lp_roll, rewards, off, gid, G, n, d, V, args)
@@ -274,7 +281,59 @@ def run_rz(args, rank, world, local_rank):
         value=tok_s, ms_per_step=step_ms, n_tok=n, d=d, V=V, R=R, G=G, clocks=clk, kernels=kernels,
         dominant=dom, achieved=ach, peak=peak_tflops, peak_src=peak_src, traffic=traffic_for(dom),
         fwd_ms=fwd_ms, fwd_tok_s=world * n / (fwd_ms * 1e-3), launches=launches_total, e2e=e2e, cfg=cfg,
+        loss_stage=loss_stage,
     )
+
+
+def run_loss_stage(rz, torch, dev, stream, n_tok=1 << 26, reps=20):
+    """The loss stage alone (rz_segment_loss) at 2^26 tokens with the moe_head response
+    shape (lengths U{256..4096}, groups of 16, Bernoulli(0.5) rewards): HBM-bound, 12
+    algorithmic bytes per token (read lp and lp_rollout, write kappa) plus 16 per
+    response (reward, offset, group id)."""
+    import workloads as wl
+    cfg = wl.CONFIGS["moe_head"]
+    rng = np.random.Generator(np.random.PCG64(cfg["seed"] + 2))
+    L = rng.integers(256, 4097, size=n_tok // 256 + 1)
+    csum = np.cumsum(L)
+    R = int(np.searchsorted(csum, n_tok)) + 1
+    L = L[:R].copy()
+    L[-1] -= int(csum[R - 1] - n_tok)
+    if L[-1] < 1:
+        L = L[:-1]
+        L[-1] += n_tok - int(L.sum())
+    R = len(L)
+    off = np.zeros(R + 1, np.int64)
+    off[1:] = np.cumsum(L)
+    gid = (np.arange(R) // 16).astype(np.int32)
+    G = int(gid[-1]) + 1
+    rewards = (rng.uniform(size=R) < 0.5).astype(np.float32)
+    g = torch.Generator(device=dev)
+    g.manual_seed(cfg["seed"] + 3)
+    lp = -2.0 * torch.rand(n_tok, generator=g, device=dev) - 0.05
+    lr = lp + 0.05 * torch.randn(n_tok, generator=g, device=dev)
+    t_r = torch.from_numpy(rewards).to(dev)
+    t_off = torch.from_numpy(off).to(dev)
+    t_gid = torch.from_numpy(gid).to(dev)
+    ws = torch.empty(rz.rz_workspace_bytes_segment_loss(n_tok, R, G), dtype=torch.uint8, device=dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    kappa = torch.empty(n_tok, dtype=torch.float32, device=dev)
+    for _ in range(3):
+        rz.rz_segment_loss(lp, lr, t_r, t_off, t_gid, G, loss=loss, kappa_out=kappa, workspace=ws, stream=stream)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        rz.rz_segment_loss(lp, lr, t_r, t_off, t_gid, G, loss=loss, kappa_out=kappa, workspace=ws, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    nbytes = 12 * n_tok + 16 * R
+    peaks, src = load_peaks()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"n_tok": n_tok, "n_resp": R, "n_groups": G, "ms_per_call": ms, "algorithmic_bytes": nbytes,
+            "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+            "bound": "hbm", "peak_source": f"hbm_gbs of {src}",
+            "note": "whole rz_segment_loss call (3 launches); inputs 768 MB > L2"}
 
 
 def run_e2e(rz, torch, dev, stream, H, W, ids, lp_roll, rewards, off, gid, G, n, d, V, args):
@@ -321,7 +380,7 @@ def run_e2e(rz, torch, dev, stream, H, W, ids, lp_roll, rewards, off, gid, G, n,
 
 # --------------------------------------------------------------------------- CPU oracle
 
-def cpu_oracle_sample(workload: str, budget_s: float = 12.0):
+def cpu_oracle_sample(workload: str, budget_s: float = 15.0):
     """The fp64 oracle as it stands, fwd+loss+bwd on a bounded sub-batch of the workload's
     shape (one group of two responses of k/2 tokens each, the workload's d and V)."""
     import oracle
@@ -341,9 +400,9 @@ def cpu_oracle_sample(workload: str, budget_s: float = 12.0):
         oracle.loss_fwd_bwd(H, W, ids, lr, np.array([1.0, 0.0]), off, np.zeros(2, np.int32), 1)
         return time.perf_counter() - t0
 
-    k = 2
+    k = 4
     t = run(k)
-    k2 = int(max(2, min(256, 2 * round(0.5 * k * budget_s / max(t, 1e-3)))))
+    k2 = int(max(2, min(512, 2 * round(0.5 * k * budget_s / max(t, 1e-3)))))
     t2 = run(k2)
     return {"value": k2 / t2, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
             "sample": f"{k2} tokens of {workload} (2 responses x {k2 // 2} tokens, d={d}, V={V}): "
@@ -424,6 +483,7 @@ def main():
             "fwd_only": {"tokens_per_s": res["fwd_tok_s"], "ms_per_step": res["fwd_ms"],
                          "tensor_frac_2dV": res["fwd_tok_s"] / world * 2 * res["d"] * res["V"] / (res["peak"] * 1e12)},
             "kernels": res["kernels"],
+            "loss_stage": res["loss_stage"],
             "gpu_launches": res["launches"],
             "clocks": res["clocks"],
             "e2e": res["e2e"],

@@ -47,7 +47,7 @@ struct Layout {
 };
 
 int kappa_blocks(int64_t n) {
-  return static_cast<int>(ceil_div(n, static_cast<int64_t>(kKappaThreads) * kKappaTokensPerThread));
+  return static_cast<int>(ceil_div(n, static_cast<int64_t>(kKappaBlockTokens)));
 }
 
 Layout make_layout(int64_t n, int32_t R, int32_t G, int32_t d, int32_t V, bool fwd, bool loss, bool bwd) {

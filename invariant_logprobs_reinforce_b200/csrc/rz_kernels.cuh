@@ -124,30 +124,53 @@ __global__ void merge_lse_kernel(const float* __restrict__ part_m, const float* 
 
 // ------------------------------------------------------------------------ loss stage
 
-// One block.  Checks the segments and groups, forms group sums in response-index
-// order (fp64), and the per-response coefficient  coef_i = -A_i / (N L_i).
-__global__ void response_coef_kernel(const float* __restrict__ rewards, const int64_t* __restrict__ off,
-                                     const int32_t* __restrict__ gid, int R, int G, int64_t n,
-                                     double* __restrict__ gsum, int* __restrict__ gcnt, float* __restrict__ coef,
-                                     int* status) {
+// One block.  Checks the segments and groups, forms each group's reward sum in
+// response-index order (fp64), and the per-response coefficient  coef_i = -A_i / (N L_i).
+// When the group ids are non-decreasing (groups are contiguous runs, the usual layout),
+// the first response of each run sums its run: O(R).  Otherwise every group scans all
+// responses: O(R G).  Both add the same rewards in the same (index) order, so both give
+// the same bits.
+__global__ void __launch_bounds__(1024)
+    response_coef_kernel(const float* __restrict__ rewards, const int64_t* __restrict__ off,
+                         const int32_t* __restrict__ gid, int R, int G, int64_t n, double* __restrict__ gsum,
+                         int* __restrict__ gcnt, float* __restrict__ coef, int* status) {
   int bad = 0;
+  int sorted = 1;
   if (threadIdx.x == 0 && (off[0] != 0 || off[R] != n)) bad |= kDevBadSegments;
   for (int i = threadIdx.x; i < R; i += blockDim.x) {
     if (off[i + 1] <= off[i]) bad |= kDevBadSegments;
-    if (gid[i] < 0 || gid[i] >= G) bad |= kDevBadGroupId;
+    const int g = gid[i];
+    if (g < 0 || g >= G) bad |= kDevBadGroupId;
+    if (i + 1 < R && gid[i + 1] < g) sorted = 0;
   }
   if (bad) atomicOr(status, bad);
-  for (int g = threadIdx.x; g < G; g += blockDim.x) {
-    double s = 0.0;
-    int c = 0;
-    for (int i = 0; i < R; ++i) {
-      if (__ldg(gid + i) == g) {
-        s += static_cast<double>(__ldg(rewards + i));
+  sorted = __syncthreads_and(sorted);
+  if (sorted) {
+    for (int i = threadIdx.x; i < R; i += blockDim.x) {
+      const int g = gid[i];
+      if ((i > 0 && gid[i - 1] == g) || g < 0 || g >= G) continue;  // not the start of a valid run
+      double s = 0.0;
+      int c = 0;
+      for (int j = i; j < R && gid[j] == g; ++j) {
+        s += static_cast<double>(rewards[j]);
         ++c;
       }
+      gsum[g] = s;
+      gcnt[g] = c;
     }
-    gsum[g] = s;
-    gcnt[g] = c;
+  } else {
+    for (int g = threadIdx.x; g < G; g += blockDim.x) {
+      double s = 0.0;
+      int c = 0;
+      for (int i = 0; i < R; ++i) {
+        if (__ldg(gid + i) == g) {
+          s += static_cast<double>(__ldg(rewards + i));
+          ++c;
+        }
+      }
+      gsum[g] = s;
+      gcnt[g] = c;
+    }
   }
   __syncthreads();
   const double N = static_cast<double>(R);
@@ -164,7 +187,9 @@ __global__ void response_coef_kernel(const float* __restrict__ rewards, const in
 }
 
 constexpr int kKappaThreads = 256;
-constexpr int kKappaTokensPerThread = 4;
+constexpr int kKappaIters = 4;                                    // float4 groups per thread
+constexpr int kKappaBlockTokens = kKappaThreads * 4 * kKappaIters;  // 4096 tokens per block
+constexpr int kKappaStagedOffsets = 256;                          // responses staged per block
 
 // response owning token t: the largest i with off[i] <= t (clamped to [0, R-1])
 __device__ __forceinline__ int find_response(const int64_t* __restrict__ off, int R, int64_t t) {
@@ -176,18 +201,56 @@ __device__ __forceinline__ int find_response(const int64_t* __restrict__ off, in
   return lo;
 }
 
-// kappa_t = coef_i * exp(lp_t - lp_rollout_t) (ratio unclipped); per-block partial sums
-// of kappa in fp64 with a fixed reduction tree.
+// kappa_t = coef_i * exp(lp_t - lp_rollout_t) (ratio unclipped) for 4096 tokens per block;
+// per-block partial sums of kappa in fp64 with a fixed reduction order.  The segment
+// offsets a block touches are staged in shared memory once per block.
 __global__ void __launch_bounds__(kKappaThreads)
     token_kappa_kernel(const float* __restrict__ lp, const float* __restrict__ lp_roll,
                        const int64_t* __restrict__ off, int R, const float* __restrict__ coef, int64_t n,
                        int vec_ok, float* __restrict__ kappa, float* __restrict__ w_out,
                        double* __restrict__ block_sums) {
-  const int64_t t0 = (static_cast<int64_t>(blockIdx.x) * kKappaThreads + threadIdx.x) * kKappaTokensPerThread;
+  __shared__ int64_t s_off[kKappaStagedOffsets + 1];
+  __shared__ int s_first, s_count;
+  __shared__ double warp_sums[kKappaThreads / 32];
+  const int64_t b0 = static_cast<int64_t>(blockIdx.x) * kKappaBlockTokens;
+  const int64_t b1 = min(n, b0 + kKappaBlockTokens);
+  if (threadIdx.x == 0) {
+    const int i0 = find_response(off, R, b0);
+    const int i1 = find_response(off, R, b1 - 1);
+    s_first = i0;
+    s_count = i1 - i0 + 1;
+  }
+  __syncthreads();
+  const int i0 = s_first;
+  const int cnt = s_count;
+  const bool staged = cnt >= 1 && cnt <= kKappaStagedOffsets;
+  if (staged)
+    for (int k = threadIdx.x; k <= cnt; k += kKappaThreads) s_off[k] = off[i0 + k];
+  __syncthreads();
+
+  // offset of response i+1, from shared memory when staged (past the staged range, which
+  // only malformed offsets can reach, the walk stops)
+  auto next_off = [&](int i) -> int64_t {
+    if (!staged) return __ldg(off + i + 1);
+    return (i + 1 - i0) <= cnt ? s_off[i + 1 - i0] : INT64_MAX;
+  };
+  auto locate = [&](int64_t t) -> int {
+    if (!staged) return find_response(off, R, t);
+    int lo = 0, hi = cnt - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_off[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    return i0 + lo;
+  };
+
   double local = 0.0;
-  if (t0 < n) {
-    int i = find_response(off, R, t0);
-    if (vec_ok && t0 + kKappaTokensPerThread <= n) {
+#pragma unroll 1
+  for (int it = 0; it < kKappaIters; ++it) {
+    const int64_t t0 = b0 + static_cast<int64_t>(it) * (kKappaThreads * 4) + threadIdx.x * 4;
+    if (t0 >= b1) break;
+    int i = locate(t0);
+    if (vec_ok && t0 + 4 <= n) {
       const float4 a = *reinterpret_cast<const float4*>(lp + t0);
       const float4 b = *reinterpret_cast<const float4*>(lp_roll + t0);
       const float la[4] = {a.x, a.y, a.z, a.w};
@@ -195,7 +258,7 @@ __global__ void __launch_bounds__(kKappaThreads)
       float w[4], k[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        while (i + 1 < R && __ldg(off + i + 1) <= t0 + j) ++i;
+        while (i + 1 < R && next_off(i) <= t0 + j) ++i;
         w[j] = expf(la[j] - lb[j]);
         k[j] = __ldg(coef + i) * w[j];
         local += static_cast<double>(k[j]);
@@ -203,9 +266,9 @@ __global__ void __launch_bounds__(kKappaThreads)
       *reinterpret_cast<float4*>(kappa + t0) = make_float4(k[0], k[1], k[2], k[3]);
       if (w_out != nullptr) *reinterpret_cast<float4*>(w_out + t0) = make_float4(w[0], w[1], w[2], w[3]);
     } else {
-      for (int j = 0; j < kKappaTokensPerThread && t0 + j < n; ++j) {
+      for (int j = 0; j < 4 && t0 + j < n; ++j) {
         const int64_t t = t0 + j;
-        while (i + 1 < R && __ldg(off + i + 1) <= t) ++i;
+        while (i + 1 < R && next_off(i) <= t) ++i;
         const float w = expf(lp[t] - lp_roll[t]);
         const float k = __ldg(coef + i) * w;
         kappa[t] = k;
@@ -217,7 +280,6 @@ __global__ void __launch_bounds__(kKappaThreads)
   // fixed-order block reduction: warp butterfly, then warp partials in warp order
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) local += __shfl_xor_sync(0xffffffffu, local, o);
-  __shared__ double warp_sums[kKappaThreads / 32];
   if ((threadIdx.x & 31) == 0) warp_sums[threadIdx.x >> 5] = local;
   __syncthreads();
   if (threadIdx.x == 0) {

@@ -116,9 +116,28 @@ def test_zero_head_gives_minus_log_V(rz):
         assert torch.allclose(lse.double(), torch.full_like(lse.double(), np.log(V)), atol=4e-6, rtol=0)
 
 
-def test_segment_loss_stage_against_oracle(rz, oracle):
+def _segments_for(layout):
+    if layout == "contiguous_groups":  # moe_head shape: 128 groups x 16, lengths U{256..4096}
+        return wl.draw_segments("moe_head")
+    rng = np.random.default_rng(17)
+    if layout == "interleaved_groups":  # group ids not sorted: response i in group i % 37
+        L = rng.integers(1, 300, size=37 * 11)
+        gid = (np.arange(L.size) % 37).astype(np.int32)
+        G = 37
+    else:  # "short_responses": 1..3 tokens each, > 256 responses per 4096-token block
+        L = rng.integers(1, 4, size=20000)
+        gid = (np.arange(L.size) // 5).astype(np.int32)
+        G = int(gid[-1]) + 1
+    off = np.zeros(L.size + 1, np.int64)
+    off[1:] = np.cumsum(L)
+    r = (rng.uniform(size=L.size) < 0.4).astype(np.float32)
+    return wl.Segments(off, gid, r, G)
+
+
+@pytest.mark.parametrize("layout", ["contiguous_groups", "interleaved_groups", "short_responses"])
+def test_segment_loss_stage_against_oracle(rz, oracle, layout):
     """The loss stage alone, fed the same synthetic logprobs on both sides: relative 1e-4."""
-    seg = wl.draw_segments("moe_head")
+    seg = _segments_for(layout)
     rng = np.random.default_rng(9)
     n = seg.n_tok
     lp = (-rng.exponential(2.0, n)).astype(np.float32)
@@ -128,8 +147,34 @@ def test_segment_loss_stage_against_oracle(rz, oracle):
     out = rz.rz_segment_loss(torch.from_numpy(lp).cuda(), torch.from_numpy(lr).cuda(),
                              torch.from_numpy(seg.rewards).cuda(), torch.from_numpy(seg.seg_offsets).cuda(),
                              torch.from_numpy(seg.group_ids).cuda(), seg.n_groups, want_w=True)
+    assert rz.rz_read_device_status(out["workspace"]) == (0, 0)
     A = oracle.advantages(seg.rewards, seg.group_ids, seg.n_groups)
     scale = float(np.mean(np.abs(A) * h.response_means(w_o, seg.seg_offsets)))
     assert abs(out["loss"].item() - loss_o) <= 1e-4 * max(abs(loss_o), scale)
     np.testing.assert_allclose(out["w"].cpu().numpy(), w_o, rtol=1e-6)
     np.testing.assert_allclose(out["kappa"].cpu().numpy(), kappa_o, rtol=1e-5, atol=1e-30)
+
+
+def test_segment_loss_sorted_and_unsorted_groups_agree_bitwise(rz):
+    """Contiguous and scattered group layouts take different kernel paths but add the same
+    rewards in the same order: permuting responses permutes kappa exactly."""
+    seg = _segments_for("contiguous_groups")
+    rng = np.random.default_rng(4)
+    lp = (-rng.exponential(2.0, seg.n_tok)).astype(np.float32)
+    lr = (lp + 0.03).astype(np.float32)
+    a = rz.rz_segment_loss(torch.from_numpy(lp).cuda(), torch.from_numpy(lr).cuda(),
+                           torch.from_numpy(seg.rewards).cuda(), torch.from_numpy(seg.seg_offsets).cuda(),
+                           torch.from_numpy(seg.group_ids).cuda(), seg.n_groups)
+    # reverse the response order (group ids become decreasing: the general path)
+    R = seg.n_resp
+    perm = np.arange(R)[::-1]
+    off = seg.seg_offsets
+    tok = np.concatenate([np.arange(off[i], off[i + 1]) for i in perm])
+    off2 = np.zeros(R + 1, np.int64)
+    off2[1:] = np.cumsum(np.diff(off)[perm])
+    b = rz.rz_segment_loss(torch.from_numpy(lp[tok]).cuda(), torch.from_numpy(lr[tok]).cuda(),
+                           torch.from_numpy(seg.rewards[perm].copy()).cuda(), torch.from_numpy(off2).cuda(),
+                           torch.from_numpy(seg.group_ids[perm].copy()).cuda(), seg.n_groups)
+    ka = a["kappa"].cpu().numpy()
+    kb = b["kappa"].cpu().numpy()
+    assert np.array_equal(ka[tok].view(np.int32), kb.view(np.int32))
