@@ -109,23 +109,30 @@ class ClockSampler:
 
 def algorithmic_flops(kind: str, rows: int, d: int, V: int) -> float:
     """Dense contraction FLOPs of one launch: 2 * rows * d * V for each tensor-core kernel."""
-    if kind in ("lmhead_lse", "dz", "dh", "dw"):
+    if kind in ("lmhead_lse", "dh", "dw"):
         return 2.0 * rows * d * V
     return 0.0
 
 
+def algorithmic_bytes(kind: str, rows: int, d: int, V: int) -> float:
+    """HBM bytes of one launch of the memory-bound kernels (per element read + write)."""
+    if kind == "dz":  # read e (fp16) and write dZ (bf16) in place over [rows, V padded to 8]
+        return 4.0 * rows * (-(-V // 8) * 8)
+    return 0.0
+
+
 def launch_rows(kinds, n_tok, chunk=16384):
-    """Rows (tokens) each recorded launch covers, in launch order."""
+    """Rows (tokens) each recorded launch covers, in launch order: the per-chunk launches
+    (forward, merge, kappa, dZ, dH, dW) cover one chunk, the rest the whole batch."""
     rows = []
-    c0 = 0
+    c0 = -chunk
     for k in kinds:
-        if k in ("lmhead_lse", "merge_lse", "response_coef", "token_kappa", "loss_final"):
+        if k == "lmhead_lse":
+            c0 += chunk
+        if k in ("response_coef", "block_first", "loss_final"):
             rows.append(n_tok)
         else:
-            r = min(chunk, n_tok - c0)
-            rows.append(r)
-            if k == "dw":
-                c0 += chunk
+            rows.append(min(chunk, n_tok - c0))
     return rows
 
 
@@ -231,10 +238,11 @@ def run_rz(args, rank, world, local_rank):
         rows = launch_rows(names, n)
         for i, (name, r) in enumerate(zip(names, rows)):
             t = evs[2 * i].elapsed_time(evs[2 * i + 1])
-            ent = per.setdefault(name, {"launches": 0, "ms": 0.0, "flops": 0.0})
+            ent = per.setdefault(name, {"launches": 0, "ms": 0.0, "flops": 0.0, "bytes": 0.0})
             ent["launches"] += 1
             ent["ms"] += t
             ent["flops"] += algorithmic_flops(name, r, d, V)
+            ent["bytes"] += algorithmic_bytes(name, r, d, V)
     launches_total = sum(v["launches"] for v in per.values())
 
     if dist:
@@ -270,11 +278,17 @@ def run_rz(args, rank, world, local_rank):
     tens = {k: v for k, v in per.items() if v["flops"] > 0}
     dom = max(tens, key=lambda k: tens[k]["ms"])
     ach = tens[dom]["flops"] / (tens[dom]["ms"] * 1e-3) / 1e12
-    kernels = {k: {"launches": v["launches"] // args.steps, "ms_per_step": v["ms"] / args.steps,
-                   "share": v["ms"] / sum(x["ms"] for x in per.values()),
-                   **({"tflops": v["flops"] / (v["ms"] * 1e-3) / 1e12,
-                       "frac_of_peak": v["flops"] / (v["ms"] * 1e-3) / 1e12 / peak_tflops} if v["flops"] else {})}
-               for k, v in per.items()}
+    kernels = {}
+    for k, v in per.items():
+        ent = {"launches": v["launches"] // args.steps, "ms_per_step": v["ms"] / args.steps,
+               "share": v["ms"] / sum(x["ms"] for x in per.values())}
+        if v["flops"]:
+            ent["tflops"] = v["flops"] / (v["ms"] * 1e-3) / 1e12
+            ent["frac_of_peak"] = ent["tflops"] / peak_tflops
+        if v["bytes"]:
+            ent["gbs"] = v["bytes"] / (v["ms"] * 1e-3) / 1e9
+            ent["frac_of_hbm"] = ent["gbs"] / peaks["hbm_gbs"]
+        kernels[k] = ent
     step_ms = ms / args.steps
     tok_s = world * n / (step_ms * 1e-3)
     return dict(

@@ -146,6 +146,7 @@ rz_status rz_segment_loss(const float* lp, const float* lp_rollout, const float*
 #define RZ_KERNEL_DZ 5            /* recomputed logits -> dZ chunk (tensor cores)                */
 #define RZ_KERNEL_DH 6            /* dH chunk = dZ W (tensor cores)                              */
 #define RZ_KERNEL_DW 7            /* dW (+)= dZ^T H (tensor cores)                               */
+#define RZ_KERNEL_BLOCK_FIRST 8   /* first response of each 4096-token block of the loss stage   */
 
 /* Number of kernel launches one rz_loss_fwd_bwd call makes for n_tok tokens (0 if n_tok < 1). */
 int32_t rz_num_launches_loss(int64_t n_tok);

@@ -28,7 +28,8 @@ EXPORTED_SYMBOLS = (
     "rz_token_logprobs", "rz_loss_fwd_bwd", "rz_segment_loss", "rz_read_device_status", "rz_num_launches_loss",
     "rz_loss_fwd_bwd_timed", "rz_token_logprobs_noalloc",
 )
-KERNEL_KINDS = ("lmhead_lse", "merge_lse", "response_coef", "token_kappa", "loss_final", "dz", "dh", "dw")
+KERNEL_KINDS = ("lmhead_lse", "merge_lse", "response_coef", "token_kappa", "loss_final", "dz", "dh", "dw",
+                "block_first")
 
 _lib = None
 

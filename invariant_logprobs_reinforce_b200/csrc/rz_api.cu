@@ -33,24 +33,34 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 bool shape_ok(int32_t d, int32_t V) { return d >= 64 && d <= 32768 && d % 64 == 0 && V >= 1; }
 
 int num_segments(int32_t V) { return static_cast<int>(ceil_div(V, kSegWidth)); }
+int num_vocab_tiles(int32_t V) { return static_cast<int>(ceil_div(V, BN)); }
 
 int64_t padded_vocab(int32_t V) { return align_up(static_cast<size_t>(V), 8); }
 
+int kappa_blocks(int64_t n) { return static_cast<int>(ceil_div(n, static_cast<int64_t>(kKappaBlockTokens))); }
+
+// Rows processed together by the loss path (one backward chunk).
+int64_t chunk_capacity(int64_t n) { return std::min<int64_t>(align_up(n, BM), kChunkTokens); }
+
 // Workspace layout (byte offsets from the workspace base, each 256-byte aligned).
+//  forward only  : status | part_m [S][n] | part_s [S][n] | zy [n]
+//  loss path     : status | part_m [S][C] | part_s [S][C] | zy [C] | lp, lse, kappa [n]
+//                  | coef [R] | gsum [G] | gcnt [G] | bsum, bfirst [blocks] | tile_max [C][tiles]
+//                  | e / dZ buffer [C][V rounded up to 8] (16-bit)
+//  loss stage    : status | lp.. as above without the forward and backward pieces
 struct Layout {
   size_t status = 0;
-  size_t part_m = 0, part_s = 0, zy = 0;  // forward partials
-  size_t lp = 0, lse = 0, kappa = 0;      // per-token scratch
-  size_t coef = 0, gsum = 0, gcnt = 0, bsum = 0;
-  size_t dz = 0;
+  size_t part_m = 0, part_s = 0, zy = 0;
+  int64_t part_ld = 0;
+  size_t lp = 0, lse = 0, kappa = 0;
+  size_t coef = 0, gsum = 0, gcnt = 0, bsum = 0, bfirst = 0;
+  size_t tile_max = 0, dz = 0;
   size_t total = 0;
 };
 
-int kappa_blocks(int64_t n) {
-  return static_cast<int>(ceil_div(n, static_cast<int64_t>(kKappaBlockTokens)));
-}
+enum class Path { Forward, Loss, LossStage };
 
-Layout make_layout(int64_t n, int32_t R, int32_t G, int32_t d, int32_t V, bool fwd, bool loss, bool bwd) {
+Layout make_layout(int64_t n, int32_t R, int32_t G, int32_t V, Path path) {
   Layout L;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -59,13 +69,14 @@ Layout make_layout(int64_t n, int32_t R, int32_t G, int32_t d, int32_t V, bool f
     return at;
   };
   L.status = take(16);
-  if (fwd) {
+  if (path != Path::LossStage) {
     const int S = num_segments(V);
-    L.part_m = take(sizeof(float) * static_cast<size_t>(S) * n);
-    L.part_s = take(sizeof(float) * static_cast<size_t>(S) * n);
-    L.zy = take(sizeof(float) * n);
+    L.part_ld = path == Path::Forward ? n : chunk_capacity(n);
+    L.part_m = take(sizeof(float) * static_cast<size_t>(S) * L.part_ld);
+    L.part_s = take(sizeof(float) * static_cast<size_t>(S) * L.part_ld);
+    L.zy = take(sizeof(float) * L.part_ld);
   }
-  if (loss) {
+  if (path != Path::Forward) {
     L.lp = take(sizeof(float) * n);
     L.lse = take(sizeof(float) * n);
     L.kappa = take(sizeof(float) * n);
@@ -73,12 +84,13 @@ Layout make_layout(int64_t n, int32_t R, int32_t G, int32_t d, int32_t V, bool f
     L.gsum = take(sizeof(double) * G);
     L.gcnt = take(sizeof(int) * G);
     L.bsum = take(sizeof(double) * kappa_blocks(n));
+    L.bfirst = take(sizeof(int) * kappa_blocks(n));
   }
-  if (bwd) {
-    const int64_t rows = std::min<int64_t>(align_up(n, BM), kChunkTokens);
-    L.dz = take(sizeof(uint16_t) * static_cast<size_t>(rows) * padded_vocab(V));
+  if (path == Path::Loss) {
+    const int64_t C = chunk_capacity(n);
+    L.tile_max = take(sizeof(float) * static_cast<size_t>(C) * num_vocab_tiles(V));
+    L.dz = take(sizeof(uint16_t) * static_cast<size_t>(C) * padded_vocab(V));
   }
-  (void)d;
   L.total = off;
   return L;
 }
@@ -103,20 +115,32 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2D bf16 tensor map: dims {inner, outer}, row stride in bytes, box {64, box_outer},
-// 128-byte swizzle, zero fill out of bounds.
-bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_stride_bytes,
-              uint32_t box_outer) {
+// 2D tensor map over a row-major [outer, inner] array with the given row stride (bytes),
+// box {box_inner, box_outer}, zero fill out of bounds.
+bool make_map(CUtensorMap* m, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
+              uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_stride_bytes};
-  cuuint32_t box[2] = {64, box_outer};
+  cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUresult r = fn(m, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// Operand load map: bf16, box {64, box_outer}, 128-byte swizzle (the UMMA stage layout).
+bool make_operand_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_stride_bytes,
+                      uint32_t box_outer) {
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, inner, outer, row_stride_bytes, 64, box_outer,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Epilogue store map: 32 rows x 64 bytes with the 64-byte swizzle of the staging slots.
+bool make_store_map(CUtensorMap* m, CUtensorMapDataType dtype, uint32_t elem_bytes, const void* base,
+                    uint64_t inner, uint64_t outer, uint64_t row_stride_bytes) {
+  return make_map(m, dtype, base, inner, outer, row_stride_bytes, 64 / elem_bytes, 32, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 // ---------------------------------------------------------------- launch recorder
@@ -184,120 +208,168 @@ GemmSched make_sched(int64_t m_rows, int64_t n_cols, int tiles_per_unit, int gro
   return s;
 }
 
-// Forward over all n rows: partials, then merge into lp (and lse if requested).
-rz_status run_forward(const rz_bf16* H, const rz_bf16* W, const int32_t* ids, int64_t n, int32_t d, int32_t V,
-                      float* lp, float* lse, void* ws, const Layout& L, cudaStream_t stream, Recorder* rec) {
+// Forward over rows [r0, r0 + rows): the fused LM head + online log-sum-exp kernel writes
+// per-segment partials (row stride L.part_ld, rows launch-relative); the merge writes lp
+// and lse (nullable) for those rows.  With store_p the kernel also writes the fp16
+// exponentials e = exp(z - tile_max) and the tile maxima for the backward.
+rz_status run_forward(const rz_bf16* H, const rz_bf16* W, const int32_t* ids, int64_t r0, int64_t rows, int32_t d,
+                      int32_t V, float* lp, float* lse, void* ws, const Layout& L, bool store_p, cudaStream_t stream,
+                      Recorder* rec) {
   int* status = at<int>(ws, L.status);
   CUtensorMap mH, mW;
-  if (!make_map(&mH, H, d, n, static_cast<uint64_t>(d) * 2, BM)) return RZ_ERR_CUDA;
-  if (!make_map(&mW, W, d, V, static_cast<uint64_t>(d) * 2, BN)) return RZ_ERR_CUDA;
-  const GemmSched s = make_sched(n, V, kSegTiles, 32, d);
-  EpiLse e;
-  e.ids = ids;
-  e.n = n;
-  e.V = V;
-  e.part_m = at<float>(ws, L.part_m);
-  e.part_s = at<float>(ws, L.part_s);
-  e.zy = at<float>(ws, L.zy);
-  const OperandPos pos{0, 0, 0, 0};
+  // rows past the range read as zeros, so no other rows' data enters the launch
+  if (!make_operand_map(&mH, H, d, r0 + rows, static_cast<uint64_t>(d) * 2, BM)) return RZ_ERR_CUDA;
+  if (!make_operand_map(&mW, W, d, V, static_cast<uint64_t>(d) * 2, BN)) return RZ_ERR_CUDA;
+  const GemmSched s = make_sched(rows, V, kSegTiles, 32, d);
+  const OperandPos pos{static_cast<int>(r0), 0, 0, 0};
+  float* part_m = at<float>(ws, L.part_m);
+  float* part_s = at<float>(ws, L.part_s);
+  float* zy = at<float>(ws, L.zy);
   rec_begin(rec, RZ_KERNEL_LMHEAD_LSE, stream);
-  if (launch_gemm<false, false>(mH, mW, s, pos, e, status, stream) != cudaSuccess) return RZ_ERR_CUDA;
+  if (store_p) {
+    EpiLse<true> e;
+    if (!make_store_map(&e.p_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, at<uint16_t>(ws, L.dz), V, rows,
+                        static_cast<uint64_t>(padded_vocab(V)) * 2))
+      return RZ_ERR_CUDA;
+    e.ids = ids + r0;
+    e.rows = rows;
+    e.V = V;
+    e.n_tiles = num_vocab_tiles(V);
+    e.part_m = part_m;
+    e.part_s = part_s;
+    e.part_ld = L.part_ld;
+    e.zy = zy;
+    e.tile_max = at<float>(ws, L.tile_max);
+    if (launch_gemm<false, false>(mH, mW, s, pos, e, status, stream) != cudaSuccess) return RZ_ERR_CUDA;
+  } else {
+    EpiLse<false> e;
+    std::memset(&e.p_map, 0, sizeof(e.p_map));
+    e.ids = ids + r0;
+    e.rows = rows;
+    e.V = V;
+    e.n_tiles = num_vocab_tiles(V);
+    e.part_m = part_m;
+    e.part_s = part_s;
+    e.part_ld = L.part_ld;
+    e.zy = zy;
+    e.tile_max = nullptr;
+    if (launch_gemm<false, false>(mH, mW, s, pos, e, status, stream) != cudaSuccess) return RZ_ERR_CUDA;
+  }
   rec_end(rec, stream);
   const int threads = 256;
   rec_begin(rec, RZ_KERNEL_MERGE_LSE, stream);
-  merge_lse_kernel<<<static_cast<unsigned>(ceil_div(n, threads)), threads, 0, stream>>>(
-      e.part_m, e.part_s, e.zy, ids, n, V, num_segments(V), lp, lse, status);
+  merge_lse_kernel<<<static_cast<unsigned>(ceil_div(rows, threads)), threads, 0, stream>>>(
+      part_m, part_s, L.part_ld, zy, ids + r0, rows, V, num_segments(V), lp + r0, lse ? lse + r0 : nullptr, status);
   if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
   rec_end(rec, stream);
   return RZ_OK;
 }
 
-rz_status run_loss(const float* lp, const float* lp_roll, const float* rewards, const int64_t* off,
-                   const int32_t* gid, int64_t n, int32_t R, int32_t G, float* loss, float* kappa, float* w_out,
-                   void* ws, const Layout& L, cudaStream_t stream, Recorder* rec) {
+// Loss stage, part 1: checks, group sums, coef_i = -A_i/(N L_i), first response per block.
+rz_status run_loss_setup(const float* rewards, const int64_t* off, const int32_t* gid, int64_t n, int32_t R,
+                         int32_t G, void* ws, const Layout& L, cudaStream_t stream, Recorder* rec) {
   int* status = at<int>(ws, L.status);
-  float* coef = at<float>(ws, L.coef);
   rec_begin(rec, RZ_KERNEL_RESPONSE_COEF, stream);
   response_coef_kernel<<<1, 1024, 0, stream>>>(rewards, off, gid, R, G, n, at<double>(ws, L.gsum),
-                                               at<int>(ws, L.gcnt), coef, status);
+                                               at<int>(ws, L.gcnt), at<float>(ws, L.coef), status);
   if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
   rec_end(rec, stream);
   const int nb = kappa_blocks(n);
-  const int vec_ok = aligned(lp, 16) && aligned(lp_roll, 16) && aligned(kappa, 16) &&
-                     (w_out == nullptr || aligned(w_out, 16));
-  rec_begin(rec, RZ_KERNEL_TOKEN_KAPPA, stream);
-  token_kappa_kernel<<<nb, kKappaThreads, 0, stream>>>(lp, lp_roll, off, R, coef, n, vec_ok, kappa, w_out,
-                                                       at<double>(ws, L.bsum));
-  if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
-  rec_end(rec, stream);
-  rec_begin(rec, RZ_KERNEL_LOSS_FINAL, stream);
-  loss_final_kernel<<<1, 1024, 0, stream>>>(at<double>(ws, L.bsum), nb, loss);
+  rec_begin(rec, RZ_KERNEL_BLOCK_FIRST, stream);
+  block_first_kernel<<<static_cast<unsigned>(ceil_div(nb, 256)), 256, 0, stream>>>(off, R, n, nb,
+                                                                                   at<int>(ws, L.bfirst));
   if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
   rec_end(rec, stream);
   return RZ_OK;
 }
 
-rz_status run_backward(const rz_bf16* H, const rz_bf16* W, const int32_t* ids, int64_t n, int32_t d, int32_t V,
-                       const float* lse, const float* kappa, rz_bf16* dH, float* dW, void* ws, const Layout& L,
-                       cudaStream_t stream, Recorder* rec) {
-  int* status = at<int>(ws, L.status);
-  __nv_bfloat16* dz = at<__nv_bfloat16>(ws, L.dz);
-  const int64_t ldz = padded_vocab(V);
-  CUtensorMap mWk, mWmn;
-  if (!make_map(&mWk, W, d, V, static_cast<uint64_t>(d) * 2, BN)) return RZ_ERR_CUDA;
-  if (!make_map(&mWmn, W, d, V, static_cast<uint64_t>(d) * 2, 64)) return RZ_ERR_CUDA;
-  for (int64_t c0 = 0; c0 < n; c0 += kChunkTokens) {
-    const int64_t rows = std::min<int64_t>(kChunkTokens, n - c0);
-    // rows of H past the chunk read as zeros, so no other chunk's data enters it
-    CUtensorMap mHk, mHmn, mDzK, mDzMn;
-    if (!make_map(&mHk, H, d, c0 + rows, static_cast<uint64_t>(d) * 2, BM)) return RZ_ERR_CUDA;
-    if (!make_map(&mHmn, H, d, c0 + rows, static_cast<uint64_t>(d) * 2, 64)) return RZ_ERR_CUDA;
-    if (!make_map(&mDzK, dz, V, rows, static_cast<uint64_t>(ldz) * 2, BM)) return RZ_ERR_CUDA;
-    if (!make_map(&mDzMn, dz, V, rows, static_cast<uint64_t>(ldz) * 2, 64)) return RZ_ERR_CUDA;
+// Loss stage, part 2: kappa and ratio for the 4096-token blocks [blk0, blk0 + nblk).
+rz_status run_kappa(const float* lp, const float* lp_roll, const int64_t* off, int64_t n, int32_t R, int blk0,
+                    int nblk, float* kappa, float* w_out, void* ws, const Layout& L, cudaStream_t stream,
+                    Recorder* rec) {
+  const int vec_ok = aligned(lp, 16) && aligned(lp_roll, 16) && aligned(kappa, 16) &&
+                     (w_out == nullptr || aligned(w_out, 16));
+  rec_begin(rec, RZ_KERNEL_TOKEN_KAPPA, stream);
+  token_kappa_kernel<<<nblk, kKappaThreads, 0, stream>>>(lp, lp_roll, off, R, at<float>(ws, L.coef),
+                                                         at<int>(ws, L.bfirst), n, blk0, vec_ok, kappa, w_out,
+                                                         at<double>(ws, L.bsum));
+  if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
+  rec_end(rec, stream);
+  return RZ_OK;
+}
 
-    // dZ chunk: A = H rows (K-major), B = W (K-major)
-    {
-      EpiDz e;
-      e.ids = ids + c0;
-      e.lse = lse + c0;
-      e.kappa = kappa + c0;
-      e.rows = rows;
-      e.V = V;
-      e.ldz = ldz;
-      e.dz = dz;
-      const GemmSched s = make_sched(rows, V, 1, 32, d);
-      const OperandPos pos{static_cast<int>(c0), 0, 0, 0};
-      rec_begin(rec, RZ_KERNEL_DZ, stream);
-      if (launch_gemm<false, false>(mHk, mWk, s, pos, e, status, stream) != cudaSuccess) return RZ_ERR_CUDA;
-      rec_end(rec, stream);
-    }
-    // dH chunk = dZ W: A = dZ (K-major, K = V), B = W (MN-major: d contiguous)
-    {
-      EpiStoreBf16 e;
-      e.out = reinterpret_cast<__nv_bfloat16*>(dH) + c0 * d;
-      e.ld = d;
-      e.rows = rows;
-      e.ncols = d;
-      const GemmSched s = make_sched(rows, d, 1, 1, V);
-      const OperandPos pos{0, 0, 0, 0};
-      rec_begin(rec, RZ_KERNEL_DH, stream);
-      if (launch_gemm<false, true>(mDzK, mWmn, s, pos, e, status, stream) != cudaSuccess) return RZ_ERR_CUDA;
-      rec_end(rec, stream);
-    }
-    // dW (+)= dZ^T H: A = dZ^T (MN-major: V contiguous), B = H chunk (MN-major: d contiguous)
-    {
-      EpiAccF32 e;
-      e.out = dW;
-      e.ld = d;
-      e.rows = V;
-      e.ncols = d;
-      e.accumulate = c0 > 0 ? 1 : 0;
-      const GemmSched s = make_sched(V, d, 1, 1, rows);
-      const OperandPos pos{0, 0, 0, static_cast<int>(c0)};
-      rec_begin(rec, RZ_KERNEL_DW, stream);
-      if (launch_gemm<true, true>(mDzMn, mHmn, s, pos, e, status, stream) != cudaSuccess) return RZ_ERR_CUDA;
-      rec_end(rec, stream);
-    }
+// Loss stage, part 3: loss = fixed-order sum of the per-block partials.
+rz_status run_loss_final(int64_t n, float* loss, void* ws, const Layout& L, cudaStream_t stream, Recorder* rec) {
+  rec_begin(rec, RZ_KERNEL_LOSS_FINAL, stream);
+  loss_final_kernel<<<1, 1024, 0, stream>>>(at<double>(ws, L.bsum), kappa_blocks(n), loss);
+  if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
+  rec_end(rec, stream);
+  return RZ_OK;
+}
+
+rz_status run_segment_loss(const float* lp, const float* lp_roll, const float* rewards, const int64_t* off,
+                           const int32_t* gid, int64_t n, int32_t R, int32_t G, float* loss, float* kappa,
+                           float* w_out, void* ws, const Layout& L, cudaStream_t stream, Recorder* rec) {
+  rz_status r = run_loss_setup(rewards, off, gid, n, R, G, ws, L, stream, rec);
+  if (r != RZ_OK) return r;
+  r = run_kappa(lp, lp_roll, off, n, R, 0, kappa_blocks(n), kappa, w_out, ws, L, stream, rec);
+  if (r != RZ_OK) return r;
+  return run_loss_final(n, loss, ws, L, stream, rec);
+}
+
+// Backward of one chunk of rows [c0, c0 + rows), after its forward (e, tile maxima) and
+// its kappa: dZ in place, dH rows = dZ W, dW (+)= dZ^T H.
+rz_status run_backward_chunk(const rz_bf16* H, const rz_bf16* W, const int32_t* ids, int64_t c0, int64_t rows,
+                             int32_t d, int32_t V, const float* lp, const float* lse, const float* kappa,
+                             rz_bf16* dH, float* dW, void* ws, const Layout& L, cudaStream_t stream,
+                             Recorder* rec) {
+  int* status = at<int>(ws, L.status);
+  uint16_t* dz = at<uint16_t>(ws, L.dz);
+  const int64_t ldz = padded_vocab(V);
+
+  rec_begin(rec, RZ_KERNEL_DZ, stream);
+  {
+    const dim3 grid(static_cast<unsigned>(ceil_div(ldz, kDzColsPerBlock)), static_cast<unsigned>(rows));
+    dz_from_p_kernel<<<grid, kDzThreads, 0, stream>>>(lse + c0, lp + c0, kappa + c0, ids + c0,
+                                                      at<float>(ws, L.tile_max), num_vocab_tiles(V), V, ldz, dz);
+    if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
+  }
+  rec_end(rec, stream);
+
+  // dH chunk = dZ W: A = dZ (K-major, K = V), B = W (MN-major: d contiguous)
+  {
+    CUtensorMap mDzK, mWmn;
+    if (!make_operand_map(&mDzK, dz, V, rows, static_cast<uint64_t>(ldz) * 2, BM)) return RZ_ERR_CUDA;
+    if (!make_operand_map(&mWmn, W, d, V, static_cast<uint64_t>(d) * 2, 64)) return RZ_ERR_CUDA;
+    EpiDh e;
+    if (!make_store_map(&e.out_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dH + c0 * d, d, rows,
+                        static_cast<uint64_t>(d) * 2))
+      return RZ_ERR_CUDA;
+    e.out_cols = d;
+    e.out_rows = rows;
+    const GemmSched s = make_sched(rows, d, 1, 1, V);
+    const OperandPos pos{0, 0, 0, 0};
+    rec_begin(rec, RZ_KERNEL_DH, stream);
+    if (launch_gemm<false, true>(mDzK, mWmn, s, pos, e, status, stream) != cudaSuccess) return RZ_ERR_CUDA;
+    rec_end(rec, stream);
+  }
+  // dW (+)= dZ^T H: A = dZ^T (MN-major: V contiguous), B = H chunk (MN-major: d contiguous)
+  {
+    CUtensorMap mDzMn, mHmn;
+    if (!make_operand_map(&mDzMn, dz, V, rows, static_cast<uint64_t>(ldz) * 2, 64)) return RZ_ERR_CUDA;
+    // rows of H past the chunk read as zeros
+    if (!make_operand_map(&mHmn, H, d, c0 + rows, static_cast<uint64_t>(d) * 2, 64)) return RZ_ERR_CUDA;
+    EpiDw e;
+    if (!make_store_map(&e.out_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dW, d, V, static_cast<uint64_t>(d) * 4))
+      return RZ_ERR_CUDA;
+    e.out_cols = d;
+    e.out_rows = V;
+    e.accumulate = c0 > 0 ? 1 : 0;
+    const GemmSched s = make_sched(V, d, 1, 1, rows);
+    const OperandPos pos{0, 0, 0, static_cast<int>(c0)};
+    rec_begin(rec, RZ_KERNEL_DW, stream);
+    if (launch_gemm<true, true>(mDzMn, mHmn, s, pos, e, status, stream) != cudaSuccess) return RZ_ERR_CUDA;
+    rec_end(rec, stream);
   }
   return RZ_OK;
 }
@@ -325,17 +397,17 @@ RZ_API const char* rz_status_string(rz_status s) {
 
 RZ_API size_t rz_workspace_bytes_logprobs(int64_t n_tok, int32_t d, int32_t V) {
   if (n_tok < 0 || n_tok >= (int64_t{1} << 31) || !shape_ok(d, V)) return 0;
-  return make_layout(n_tok, 0, 0, d, V, true, false, false).total;
+  return make_layout(n_tok, 0, 0, V, Path::Forward).total;
 }
 
 RZ_API size_t rz_workspace_bytes_loss(int64_t n_tok, int32_t n_resp, int32_t n_groups, int32_t d, int32_t V) {
   if (n_tok < 1 || n_tok >= (int64_t{1} << 31) || n_resp < 1 || n_groups < 1 || !shape_ok(d, V)) return 0;
-  return make_layout(n_tok, n_resp, n_groups, d, V, true, true, true).total;
+  return make_layout(n_tok, n_resp, n_groups, V, Path::Loss).total;
 }
 
 RZ_API size_t rz_workspace_bytes_segment_loss(int64_t n_tok, int32_t n_resp, int32_t n_groups) {
   if (n_tok < 1 || n_tok >= (int64_t{1} << 31) || n_resp < 1 || n_groups < 1) return 0;
-  return make_layout(n_tok, n_resp, n_groups, 64, 1, false, true, false).total;
+  return make_layout(n_tok, n_resp, n_groups, 1, Path::LossStage).total;
 }
 
 RZ_API rz_status rz_token_logprobs(const rz_bf16* H, const rz_bf16* W_head, const int32_t* token_ids, int64_t n_tok,
@@ -348,11 +420,11 @@ RZ_API rz_status rz_token_logprobs(const rz_bf16* H, const rz_bf16* W_head, cons
   if (!aligned(H, 16) || !aligned(W_head, 16) || !aligned(token_ids, 4) || !aligned(lp_out, 4) ||
       (lse_out && !aligned(lse_out, 4)) || !aligned(workspace, kAlign))
     return RZ_ERR_INVALID_ARG;
-  const Layout L = make_layout(n_tok, 0, 0, d, V, true, false, false);
+  const Layout L = make_layout(n_tok, 0, 0, V, Path::Forward);
   if (ws_bytes < L.total) return RZ_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(at<int>(workspace, L.status), 0, sizeof(int), st) != cudaSuccess) return RZ_ERR_CUDA;
-  return run_forward(H, W_head, token_ids, n_tok, d, V, lp_out, lse_out, workspace, L, st, nullptr);
+  return run_forward(H, W_head, token_ids, 0, n_tok, d, V, lp_out, lse_out, workspace, L, false, st, nullptr);
 }
 
 RZ_API rz_status rz_segment_loss(const float* lp, const float* lp_rollout, const float* rewards,
@@ -366,12 +438,12 @@ RZ_API rz_status rz_segment_loss(const float* lp, const float* lp_rollout, const
       !aligned(group_ids, 4) || !aligned(loss, 4) || !aligned(kappa_out, 4) || (w_out && !aligned(w_out, 4)) ||
       !aligned(workspace, kAlign))
     return RZ_ERR_INVALID_ARG;
-  const Layout L = make_layout(n_tok, n_resp, n_groups, 64, 1, false, true, false);
+  const Layout L = make_layout(n_tok, n_resp, n_groups, 1, Path::LossStage);
   if (ws_bytes < L.total) return RZ_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(at<int>(workspace, L.status), 0, sizeof(int), st) != cudaSuccess) return RZ_ERR_CUDA;
-  return run_loss(lp, lp_rollout, rewards, seg_offsets, group_ids, n_tok, n_resp, n_groups, loss, kappa_out, w_out,
-                  workspace, L, st, nullptr);
+  return run_segment_loss(lp, lp_rollout, rewards, seg_offsets, group_ids, n_tok, n_resp, n_groups, loss, kappa_out,
+                          w_out, workspace, L, st, nullptr);
 }
 
 }  // extern "C"
@@ -392,19 +464,29 @@ rz_status loss_fwd_bwd_impl(const rz_bf16* H, const rz_bf16* W_head, const int32
       !aligned(loss, 4) || (lp_out && !aligned(lp_out, 4)) || (kappa_out && !aligned(kappa_out, 4)) ||
       !aligned(workspace, kAlign))
     return RZ_ERR_INVALID_ARG;
-  const Layout L = make_layout(n_tok, n_resp, n_groups, d, V, true, true, true);
+  const Layout L = make_layout(n_tok, n_resp, n_groups, V, Path::Loss);
   if (ws_bytes < L.total) return RZ_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(at<int>(workspace, L.status), 0, sizeof(int), st) != cudaSuccess) return RZ_ERR_CUDA;
   float* lp = lp_out ? lp_out : at<float>(workspace, L.lp);
   float* lse = at<float>(workspace, L.lse);
   float* kappa = kappa_out ? kappa_out : at<float>(workspace, L.kappa);
-  rz_status r = run_forward(H, W_head, token_ids, n_tok, d, V, lp, lse, workspace, L, st, rec);
+  rz_status r = run_loss_setup(rewards, seg_offsets, group_ids, n_tok, n_resp, n_groups, workspace, L, st, rec);
   if (r != RZ_OK) return r;
-  r = run_loss(lp, lp_rollout, rewards, seg_offsets, group_ids, n_tok, n_resp, n_groups, loss, kappa, nullptr,
-               workspace, L, st, rec);
-  if (r != RZ_OK) return r;
-  return run_backward(H, W_head, token_ids, n_tok, d, V, lse, kappa, dH, dW, workspace, L, st, rec);
+  // chunk by chunk: forward (with the exponentials kept), kappa, backward; the loss
+  // partials are per 4096-token block, so the loss does not depend on the chunking
+  for (int64_t c0 = 0; c0 < n_tok; c0 += kChunkTokens) {
+    const int64_t rows = std::min<int64_t>(kChunkTokens, n_tok - c0);
+    r = run_forward(H, W_head, token_ids, c0, rows, d, V, lp, lse, workspace, L, true, st, rec);
+    if (r != RZ_OK) return r;
+    const int blk0 = static_cast<int>(c0 / kKappaBlockTokens);
+    const int nblk = static_cast<int>(ceil_div(rows, kKappaBlockTokens));
+    r = run_kappa(lp, lp_rollout, seg_offsets, n_tok, n_resp, blk0, nblk, kappa, nullptr, workspace, L, st, rec);
+    if (r != RZ_OK) return r;
+    r = run_backward_chunk(H, W_head, token_ids, c0, rows, d, V, lp, lse, kappa, dH, dW, workspace, L, st, rec);
+    if (r != RZ_OK) return r;
+  }
+  return run_loss_final(n_tok, loss, workspace, L, st, rec);
 }
 
 }  // namespace
@@ -422,7 +504,7 @@ RZ_API rz_status rz_loss_fwd_bwd(const rz_bf16* H, const rz_bf16* W_head, const 
 
 RZ_API int32_t rz_num_launches_loss(int64_t n_tok) {
   if (n_tok < 1) return 0;
-  return static_cast<int32_t>(5 + 3 * ceil_div(n_tok, kChunkTokens));
+  return static_cast<int32_t>(3 + 6 * ceil_div(n_tok, kChunkTokens));
 }
 
 RZ_API rz_status rz_loss_fwd_bwd_timed(const rz_bf16* H, const rz_bf16* W_head, const int32_t* token_ids,
@@ -488,14 +570,14 @@ RZ_API rz_status rz_token_logprobs_noalloc(const rz_bf16* H, const rz_bf16* W_he
   if (!aligned(H, 16) || !aligned(W_head, 16) || !aligned(token_ids, 4) || !aligned(lp_out, 4) ||
       (lse_out && !aligned(lse_out, 4)))
     return RZ_ERR_INVALID_ARG;
-  const Layout L = make_layout(n_tok, 0, 0, d, V, true, false, false);
+  const Layout L = make_layout(n_tok, 0, 0, V, Path::Forward);
   if (L.total > static_cast<size_t>(RZ_NOALLOC_SCRATCH_BYTES)) return RZ_ERR_WORKSPACE_TOO_SMALL;
   void* scratch = nullptr;
   const rz_status r = noalloc_scratch(&scratch);
   if (r != RZ_OK) return r;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(at<int>(scratch, L.status), 0, sizeof(int), st) != cudaSuccess) return RZ_ERR_CUDA;
-  return run_forward(H, W_head, token_ids, n_tok, d, V, lp_out, lse_out, scratch, L, st, nullptr);
+  return run_forward(H, W_head, token_ids, 0, n_tok, d, V, lp_out, lse_out, scratch, L, false, st, nullptr);
 }
 
 RZ_API rz_status rz_read_device_status(const void* workspace, void* stream, int32_t* bits_out) {

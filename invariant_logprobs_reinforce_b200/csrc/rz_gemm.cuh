@@ -34,7 +34,12 @@ constexpr int kStageBytesB = BN * BK * 2;  // 32 KB
 constexpr int kStageBytes = kStageBytesA + kStageBytesB;
 constexpr int kGemmThreads = 192;
 constexpr int kTmemCols = 2 * BN;  // two fp32 accumulators of 128 lanes x 256 columns
-constexpr int kGemmSmemBytes = kStages * kStageBytes + 1024 /*barriers*/ + 1024 /*alignment slack*/;
+// Epilogue staging for TMA stores: per epilogue warp, two slots of 32 rows x 64 bytes.
+constexpr int kStageSlotBytes = 32 * 64;
+constexpr int kEpiWarpStageBytes = 2 * kStageSlotBytes;
+constexpr int kEpiStageBytes = 4 * kEpiWarpStageBytes;  // 16 KB
+constexpr int kGemmSmemBytes =
+    kStages * kStageBytes + kEpiStageBytes + 1024 /*barriers*/ + 1024 /*alignment slack*/;
 
 struct GemmSched {
   int m_blocks;        // number of 128-row blocks
@@ -91,17 +96,52 @@ __host__ __device__ constexpr uint32_t operand_k_step() {
   return MN_MAJOR ? (2048u >> 4) : (32u >> 4);
 }
 
+// Per-epilogue-warp staging for TMA stores: two slots of 32 rows x 64 bytes laid out with
+// the 64-byte swizzle (16-byte piece q of row r sits at piece q ^ ((r >> 1) & 3)), which
+// matches a tensor map with CU_TENSOR_MAP_SWIZZLE_64B and a box of 64 bytes x 32 rows and
+// makes the lanes' 16-byte writes bank-conflict free.  Lane 0 issues the store; each
+// slot is reused only after the store that last read it has finished reading.
+struct WarpStage {
+  uint8_t* base;
+  int slot;
+
+  // Write this lane's 64-byte row into the next slot and store the slot's 32 x 64-byte
+  // box at (x, y) of `map` (reduce-add instead of store when `add` is set).  A box whose
+  // first row is at or past `row_limit` lies wholly outside the map and is skipped
+  // (uniform across the warp: y is the warp's first row).
+  __device__ __forceinline__ void store_rows(const CUtensorMap* map, int lane, const uint4 (&row)[4], int32_t x,
+                                             int32_t y, int64_t row_limit, bool add = false) {
+    if (y >= row_limit) return;
+    uint8_t* buf = base + slot * kStageSlotBytes;
+    if (lane == 0) bulk_wait_group_read<1>();  // the store issued from this slot two rounds ago
+    __syncwarp();
+    uint8_t* r = buf + lane * 64;
+    const int sw = (lane >> 1) & 3;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(r + ((q ^ sw) << 4)) = row[q];
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      if (add) tma_reduce_add_2d(map, buf, x, y); else tma_store_2d(map, buf, x, y);
+      bulk_commit_group();
+    }
+    slot ^= 1;
+  }
+};
+
 template <bool A_MN, bool B_MN, class Epi>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const GemmSched sched, const OperandPos pos, const Epi epi, int* __restrict__ status) {
+                   const GemmSched sched, const OperandPos pos, const __grid_constant__ Epi epi,
+                   int* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte swizzle atoms
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   uint8_t* stage_a = smem;
   uint8_t* stage_b = smem + kStages * kStageBytesA;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint8_t* epi_stage = smem + kStages * kStageBytes;  // 1024-aligned
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes + kEpiStageBytes);
   uint64_t* full = bars;                   // [kStages]  TMA -> MMA
   uint64_t* empty = bars + kStages;        // [kStages]  MMA -> TMA
   uint64_t* acc_full = bars + 2 * kStages; // [2]        MMA -> epilogue
@@ -235,6 +275,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int row_in_tile = quad * 32 + lane;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
     typename Epi::State st;
+    WarpStage stage{epi_stage + quad * kEpiWarpStageBytes, 0};
     uint32_t it = 0;
     for (int u = blockIdx.x; u < sched.num_units && !aborted; u += gridDim.x) {
       int mb, nu;
@@ -250,7 +291,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           break;
         }
         tc_fence_after();
-        epi.tile(st, lane_base + acc * BN, mb, nt, row_in_tile);
+        epi.tile(st, lane_base + acc * BN, mb, nt, row_in_tile, lane, stage);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[acc]);
@@ -262,6 +303,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (lane == 0) atomicOr(status, kDevWaitTimeout);
       *abort_flag = 1;
     }
+    // stores issued from the staging slots complete before the CTA exits
+    if (lane == 0) bulk_wait_group_all();
+    __syncwarp();
   }
 
   tc_fence_before();
