@@ -136,8 +136,9 @@ def launch_rows(kinds, n_tok, chunk=16384):
     return rows
 
 
-def traffic_for(kernel: str):
-    """DRAM bytes per launch from a committed ncu summary, if it matches the current source."""
+def traffic_for(kernel: str, rows_per_launch: float):
+    """DRAM bytes per launch from the committed ncu record (profiles/traffic.json), scaled by
+    the rows a launch covers, while the kernel's sources still match the recorded digest."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
@@ -145,10 +146,10 @@ def traffic_for(kernel: str):
         with open(p) as f:
             rec = json.load(f)
         from invariant_logprobs_reinforce_b200.build import source_digest
-        if rec.get("source_digest") != source_digest():
-            return None
         ent = rec.get("kernels", {}).get(kernel)
-        return None if ent is None else ent.get("bytes_per_launch")
+        if ent is None or ent.get("source_digest") != source_digest(ent.get("family", "gemm")):
+            return None
+        return ent["bytes_per_row"] * rows_per_launch
     except Exception:
         return None
 
@@ -238,8 +239,9 @@ def run_rz(args, rank, world, local_rank):
         rows = launch_rows(names, n)
         for i, (name, r) in enumerate(zip(names, rows)):
             t = evs[2 * i].elapsed_time(evs[2 * i + 1])
-            ent = per.setdefault(name, {"launches": 0, "ms": 0.0, "flops": 0.0, "bytes": 0.0})
+            ent = per.setdefault(name, {"launches": 0, "ms": 0.0, "flops": 0.0, "bytes": 0.0, "rows": 0})
             ent["launches"] += 1
+            ent["rows"] += r
             ent["ms"] += t
             ent["flops"] += algorithmic_flops(name, r, d, V)
             ent["bytes"] += algorithmic_bytes(name, r, d, V)
@@ -293,7 +295,8 @@ def run_rz(args, rank, world, local_rank):
     tok_s = world * n / (step_ms * 1e-3)
     return dict(
         value=tok_s, ms_per_step=step_ms, n_tok=n, d=d, V=V, R=R, G=G, clocks=clk, kernels=kernels,
-        dominant=dom, achieved=ach, peak=peak_tflops, peak_src=peak_src, traffic=traffic_for(dom),
+        dominant=dom, achieved=ach, peak=peak_tflops, peak_src=peak_src,
+        traffic=traffic_for(dom, tens[dom]["rows"] / tens[dom]["launches"]),
         fwd_ms=fwd_ms, fwd_tok_s=world * n / (fwd_ms * 1e-3), launches=launches_total, e2e=e2e, cfg=cfg,
         loss_stage=loss_stage,
     )

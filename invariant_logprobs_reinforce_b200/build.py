@@ -52,11 +52,21 @@ if __name__ == "__main__":
           extra_flags=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else [])
 
 
-def source_digest() -> str:
-    """sha256 over the CUDA sources and the public header (identifies a kernel build)."""
+def source_digest(family: str = "all") -> str:
+    """sha256 prefix over the sources that define a kernel family.
+
+    "gemm": the tensor-core engine, its epilogues and the launch code; "simt": the
+    SIMT kernels and the launch code; "all": every CUDA source and the public header.
+    A recorded measurement of a kernel is only current while its family's digest holds.
+    """
     import hashlib
+    names = {
+        "gemm": ("rz_ptx.cuh", "rz_gemm.cuh", "rz_epilogues.cuh", "rz_api.cu"),
+        "simt": ("rz_ptx.cuh", "rz_epilogues.cuh", "rz_simt.cuh", "rz_api.cu"),
+    }
+    paths = deps() if family == "all" else [os.path.join(CSRC, n) for n in names[family]]
     h = hashlib.sha256()
-    for p in deps():
+    for p in paths:
         h.update(os.path.basename(p).encode())
         with open(p, "rb") as f:
             h.update(f.read())

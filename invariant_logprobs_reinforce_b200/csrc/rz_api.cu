@@ -17,7 +17,7 @@
 #include <mutex>
 
 #include "../../include/rz.h"
-#include "rz_kernels.cuh"
+#include "rz_simt.cuh"
 
 namespace rz {
 namespace {
@@ -269,9 +269,17 @@ rz_status run_forward(const rz_bf16* H, const rz_bf16* W, const int32_t* ids, in
 rz_status run_loss_setup(const float* rewards, const int64_t* off, const int32_t* gid, int64_t n, int32_t R,
                          int32_t G, void* ws, const Layout& L, cudaStream_t stream, Recorder* rec) {
   int* status = at<int>(ws, L.status);
+  int* flags = status + 1;  // cleared together with the status word
+  double* gsum = at<double>(ws, L.gsum);
+  int* gcnt = at<int>(ws, L.gcnt);
+  const unsigned rb = static_cast<unsigned>(ceil_div(R, kCoefThreads));
   rec_begin(rec, RZ_KERNEL_RESPONSE_COEF, stream);
-  response_coef_kernel<<<1, 1024, 0, stream>>>(rewards, off, gid, R, G, n, at<double>(ws, L.gsum),
-                                               at<int>(ws, L.gcnt), at<float>(ws, L.coef), status);
+  coef_runs_kernel<<<rb, kCoefThreads, 0, stream>>>(rewards, off, gid, R, G, n, gsum, gcnt, flags, status);
+  if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
+  coef_groups_kernel<<<static_cast<unsigned>(ceil_div(G, kCoefThreads)), kCoefThreads, 0, stream>>>(
+      rewards, gid, R, G, gsum, gcnt, flags);
+  if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
+  coef_kernel<<<rb, kCoefThreads, 0, stream>>>(rewards, off, gid, R, G, gsum, gcnt, at<float>(ws, L.coef));
   if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
   rec_end(rec, stream);
   const int nb = kappa_blocks(n);
@@ -329,9 +337,8 @@ rz_status run_backward_chunk(const rz_bf16* H, const rz_bf16* W, const int32_t* 
 
   rec_begin(rec, RZ_KERNEL_DZ, stream);
   {
-    const dim3 grid(static_cast<unsigned>(ceil_div(ldz, kDzColsPerBlock)), static_cast<unsigned>(rows));
-    dz_from_p_kernel<<<grid, kDzThreads, 0, stream>>>(lse + c0, lp + c0, kappa + c0, ids + c0,
-                                                      at<float>(ws, L.tile_max), num_vocab_tiles(V), V, ldz, dz);
+    dz_from_p_kernel<<<static_cast<unsigned>(rows), kDzThreads, 0, stream>>>(
+        lse + c0, lp + c0, kappa + c0, ids + c0, at<float>(ws, L.tile_max), num_vocab_tiles(V), V, ldz, dz);
     if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
   }
   rec_end(rec, stream);
@@ -423,7 +430,7 @@ RZ_API rz_status rz_token_logprobs(const rz_bf16* H, const rz_bf16* W_head, cons
   const Layout L = make_layout(n_tok, 0, 0, V, Path::Forward);
   if (ws_bytes < L.total) return RZ_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(at<int>(workspace, L.status), 0, sizeof(int), st) != cudaSuccess) return RZ_ERR_CUDA;
+  if (cudaMemsetAsync(at<int>(workspace, L.status), 0, 16, st) != cudaSuccess) return RZ_ERR_CUDA;
   return run_forward(H, W_head, token_ids, 0, n_tok, d, V, lp_out, lse_out, workspace, L, false, st, nullptr);
 }
 
@@ -441,7 +448,7 @@ RZ_API rz_status rz_segment_loss(const float* lp, const float* lp_rollout, const
   const Layout L = make_layout(n_tok, n_resp, n_groups, 1, Path::LossStage);
   if (ws_bytes < L.total) return RZ_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(at<int>(workspace, L.status), 0, sizeof(int), st) != cudaSuccess) return RZ_ERR_CUDA;
+  if (cudaMemsetAsync(at<int>(workspace, L.status), 0, 16, st) != cudaSuccess) return RZ_ERR_CUDA;
   return run_segment_loss(lp, lp_rollout, rewards, seg_offsets, group_ids, n_tok, n_resp, n_groups, loss, kappa_out,
                           w_out, workspace, L, st, nullptr);
 }
@@ -467,7 +474,7 @@ rz_status loss_fwd_bwd_impl(const rz_bf16* H, const rz_bf16* W_head, const int32
   const Layout L = make_layout(n_tok, n_resp, n_groups, V, Path::Loss);
   if (ws_bytes < L.total) return RZ_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(at<int>(workspace, L.status), 0, sizeof(int), st) != cudaSuccess) return RZ_ERR_CUDA;
+  if (cudaMemsetAsync(at<int>(workspace, L.status), 0, 16, st) != cudaSuccess) return RZ_ERR_CUDA;
   float* lp = lp_out ? lp_out : at<float>(workspace, L.lp);
   float* lse = at<float>(workspace, L.lse);
   float* kappa = kappa_out ? kappa_out : at<float>(workspace, L.kappa);
@@ -576,7 +583,7 @@ RZ_API rz_status rz_token_logprobs_noalloc(const rz_bf16* H, const rz_bf16* W_he
   const rz_status r = noalloc_scratch(&scratch);
   if (r != RZ_OK) return r;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(at<int>(scratch, L.status), 0, sizeof(int), st) != cudaSuccess) return RZ_ERR_CUDA;
+  if (cudaMemsetAsync(at<int>(scratch, L.status), 0, 16, st) != cudaSuccess) return RZ_ERR_CUDA;
   return run_forward(H, W_head, token_ids, 0, n_tok, d, V, lp_out, lse_out, scratch, L, false, st, nullptr);
 }
 

@@ -1,0 +1,209 @@
+// rz_epilogues.cuh -- the epilogues that turn the tensor-core engine into the three
+// contractions of the path:
+//
+//   EpiLse<false>  fused LM head + online log-sum-exp + gather (logits stay on chip)
+//   EpiLse<true>   the same, also keeping exp(z - tile max) (fp16) for the backward
+//   EpiDh          dH = dZ W tile, TMA-stored as bf16
+//   EpiDw          dW (+)= dZ^T H tile, TMA-stored / TMA-reduce-added in chunk order
+//
+// Definitions follow "vLLM says aligned kernels make asynchronous RL stable at lag 64"
+// (ainewsbites.com), section "REINFORCE Zero removes the mismatch first"; the fixed
+// orders follow "vLLM Train-Inference Consistency Release Notes" (agentlenshq.com),
+// section "Achieving Bitwise Consistency" (kernel determinism, batch independence).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "rz_gemm.cuh"
+
+namespace rz {
+
+// Vocabulary segment of the forward: 8 tiles of 256 columns.  A function of nothing:
+// the segment grid over [0, V) is fixed, so every row sees the same reduction order
+// whatever the number of rows in the call.
+constexpr int kSegTiles = 8;
+constexpr int kSegWidth = kSegTiles * BN;  // 2048 vocabulary columns
+
+// Backward chunk: tokens whose dZ rows are materialised at once (a fixed constant, so
+// the order in which token contributions reach dW never depends on n_tok).
+constexpr int kChunkTokens = 16384;
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&p);
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  __half2 p = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&p);
+}
+
+// ------------------------------------------------------------------------ forward
+
+// Forward epilogue.  Per row and per 256-column tile: the tile maximum, then
+// e_v = 2^((z_v - tile_max) log2 e) and their sum, folded into the row's running
+// (max, sum) pair of the current vocabulary segment:
+//   m' = max(m, tile_max);  s' = s 2^((m - m') log2 e) + tile_sum 2^((tile_max - m') log2 e)
+// The sampled token's logit is picked out of the tile that holds it.  With STORE_P the
+// e_v are also written (fp16, TMA store) together with the tile maximum, so the backward
+// can form softmax probabilities without recomputing the logits; the log-sum-exp
+// arithmetic is the same code either way, so both variants give the same lse bits.
+template <bool STORE_P>
+struct EpiLse {
+  CUtensorMap p_map;  // STORE_P: fp16 [rows, V] (box 32 x 32, 64-byte swizzle)
+  const int32_t* ids; // launch-relative
+  int64_t rows;       // rows in this launch
+  int V;
+  int n_tiles;        // 256-column tiles over V
+  float* part_m;      // [S][part_ld] running max of the segment
+  float* part_s;      // [S][part_ld] sum of exp(z - max) over the segment
+  int64_t part_ld;
+  float* zy;          // [rows] logit of the sampled token
+  float* tile_max;    // STORE_P: [rows][n_tiles]
+
+  struct State {
+    float m, s;
+    int y;
+    int64_t row;
+  };
+
+  __device__ __forceinline__ void begin_unit(State& st, int mb, int, int r) const {
+    st.row = static_cast<int64_t>(mb) * BM + r;
+    st.y = st.row < rows ? __ldg(ids + st.row) : -1;
+    st.m = -INFINITY;
+    st.s = 0.0f;
+  }
+
+  __device__ __forceinline__ void tile(State& st, uint32_t taddr, int mb, int nt, int r, int lane,
+                                       WarpStage& stage) const {
+    // pass 1: tile maximum over the valid columns
+    float tmax = -INFINITY;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      const int col0 = nt * BN + c * 32;
+      if (col0 >= V) break;  // uniform across the warp
+      float v[32];
+      __syncwarp();  // the TMEM load is warp-collective: reconverge first
+      tmem_ld_32cols(taddr + c * 32, v);
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (col0 + j < V) tmax = fmaxf(tmax, v[j]);
+    }
+    // pass 2: exponentials relative to the tile maximum, their sum, the gather
+    float tsum = 0.0f;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      const int col0 = nt * BN + c * 32;
+      if (col0 >= V) break;
+      float v[32];
+      __syncwarp();
+      tmem_ld_32cols(taddr + c * 32, v);
+      const unsigned off = static_cast<unsigned>(st.y - col0);
+      if (off < 32u) {
+        float z = v[0];
+#pragma unroll
+        for (int j = 1; j < 32; ++j) z = (static_cast<unsigned>(j) == off) ? v[j] : z;
+        zy[st.row] = z;
+      }
+      float e[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        e[j] = (col0 + j < V) ? ex2_approx((v[j] - tmax) * kLog2e) : 0.0f;
+        tsum += e[j];
+      }
+      if constexpr (STORE_P) {
+        uint4 row[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          row[q] = make_uint4(pack_half2(e[8 * q], e[8 * q + 1]), pack_half2(e[8 * q + 2], e[8 * q + 3]),
+                              pack_half2(e[8 * q + 4], e[8 * q + 5]), pack_half2(e[8 * q + 6], e[8 * q + 7]));
+        stage.store_rows(&p_map, lane, row, col0, mb * BM + (r - lane), rows);
+      }
+    }
+    const float m_new = fmaxf(st.m, tmax);
+    st.s = st.s * ex2_approx((st.m - m_new) * kLog2e) + tsum * ex2_approx((tmax - m_new) * kLog2e);
+    st.m = m_new;
+    if constexpr (STORE_P) {
+      if (st.row < rows) tile_max[st.row * n_tiles + nt] = tmax;
+    }
+  }
+
+  __device__ __forceinline__ void end_unit(const State& st, int, int nu, int) const {
+    if (st.row < rows) {
+      part_m[static_cast<int64_t>(nu) * part_ld + st.row] = st.m;
+      part_s[static_cast<int64_t>(nu) * part_ld + st.row] = st.s;
+    }
+  }
+};
+
+// dH tile: fp32 accumulator -> bf16, TMA-stored into a [rows, d] map of the chunk.
+struct EpiDh {
+  CUtensorMap out_map;  // bf16 [rows, d], box 32 x 32, 64-byte swizzle
+
+  struct State {};
+
+  __device__ __forceinline__ void begin_unit(State&, int, int, int) const {}
+
+  __device__ __forceinline__ void tile(State&, uint32_t taddr, int mb, int nt, int r, int lane,
+                                       WarpStage& stage) const {
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      const int col0 = nt * BN + c * 32;
+      if (col0 >= out_cols) break;
+      float v[32];
+      __syncwarp();
+      tmem_ld_32cols(taddr + c * 32, v);
+      uint4 row[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        row[q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                            pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+      stage.store_rows(&out_map, lane, row, col0, mb * BM + (r - lane), out_rows);
+    }
+  }
+
+  __device__ __forceinline__ void end_unit(const State&, int, int, int) const {}
+
+  int out_cols;
+  int64_t out_rows;
+};
+
+// dW tile: fp32 accumulator TMA-stored (first chunk) or TMA-reduce-added (later chunks,
+// in chunk order) into the [V, d] fp32 map; every element gets exactly one store or add
+// per chunk, so the result is deterministic.
+struct EpiDw {
+  CUtensorMap out_map;  // fp32 [V, d], box 16 x 32, 64-byte swizzle
+  int out_cols;
+  int64_t out_rows;
+  int accumulate;
+
+  struct State {};
+
+  __device__ __forceinline__ void begin_unit(State&, int, int, int) const {}
+
+  __device__ __forceinline__ void tile(State&, uint32_t taddr, int mb, int nt, int r, int lane,
+                                       WarpStage& stage) const {
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      const int col0 = nt * BN + c * 32;
+      if (col0 >= out_cols) break;
+      float v[32];
+      __syncwarp();
+      tmem_ld_32cols(taddr + c * 32, v);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint4 row[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          row[q] = make_uint4(__float_as_uint(v[16 * h + 4 * q]), __float_as_uint(v[16 * h + 4 * q + 1]),
+                              __float_as_uint(v[16 * h + 4 * q + 2]), __float_as_uint(v[16 * h + 4 * q + 3]));
+        stage.store_rows(&out_map, lane, row, col0 + 16 * h, mb * BM + (r - lane), out_rows, accumulate != 0);
+      }
+    }
+  }
+
+  __device__ __forceinline__ void end_unit(const State&, int, int, int) const {}
+};
+
+}  // namespace rz

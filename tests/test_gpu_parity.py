@@ -151,7 +151,8 @@ def test_segment_loss_stage_against_oracle(rz, oracle, layout):
     A = oracle.advantages(seg.rewards, seg.group_ids, seg.n_groups)
     scale = float(np.mean(np.abs(A) * h.response_means(w_o, seg.seg_offsets)))
     assert abs(out["loss"].item() - loss_o) <= 1e-4 * max(abs(loss_o), scale)
-    np.testing.assert_allclose(out["w"].cpu().numpy(), w_o, rtol=1e-6)
+    # the ratio is 2^((lp - lp_rollout) log2 e) on the MUFU ex2 unit: about 2 + 1.2|x| ulp
+    np.testing.assert_allclose(out["w"].cpu().numpy(), w_o, rtol=2e-6)
     np.testing.assert_allclose(out["kappa"].cpu().numpy(), kappa_o, rtol=1e-5, atol=1e-30)
 
 
