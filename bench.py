@@ -105,6 +105,22 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+# --------------------------------------------------------------------------- ranks
+
+def max_over_ranks(value: float, device=None) -> float:
+    """The largest value over all ranks of the default process group (the job's time)."""
+    import torch
+    import torch.distributed as tdist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job tokens/s: every rank processes its own replica batch each step."""
+    return world * tokens_per_rank / (ms_per_step * 1e-3)
+
+
 # --------------------------------------------------------------------------- rz arm
 
 def algorithmic_flops(kind: str, rows: int, d: int, V: int) -> float:
@@ -248,9 +264,7 @@ def run_rz(args, rank, world, local_rank):
     launches_total = sum(v["launches"] for v in per.values())
 
     if dist:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, dev)
 
     # forward alone (rz_token_logprobs), same inputs
     lpf = torch.empty(n, dtype=torch.float32, device=dev)
@@ -292,7 +306,7 @@ def run_rz(args, rank, world, local_rank):
             ent["frac_of_hbm"] = ent["gbs"] / peaks["hbm_gbs"]
         kernels[k] = ent
     step_ms = ms / args.steps
-    tok_s = world * n / (step_ms * 1e-3)
+    tok_s = job_throughput(n, world, step_ms)
     return dict(
         value=tok_s, ms_per_step=step_ms, n_tok=n, d=d, V=V, R=R, G=G, clocks=clk, kernels=kernels,
         dominant=dom, achieved=ach, peak=peak_tflops, peak_src=peak_src,
