@@ -47,8 +47,12 @@ def _load():
         lib.oracle_loss_fwd_bwd.argtypes = [P, P, c_int, P, P, P, P, P, i64, i32, i32, i32, i32,
                                             P, P, P, P, P, P, P]
         lib.oracle_num_threads.argtypes = []
+        lib.oracle_loss_from_lp_ex.argtypes = [P, P, P, P, P, i64, i32, i32, i32, ctypes.c_double, ctypes.c_double,
+                                               ctypes.c_double, P, i32, P, P, P]
+        lib.oracle_ratio_stats.argtypes = [P, P, P, i64, i32, P, P, P]
         for f in ("oracle_lp_rows", "oracle_advantages", "oracle_loss_from_lp", "oracle_dh_rows",
-                  "oracle_dw_rows", "oracle_loss_fwd_bwd", "oracle_num_threads"):
+                  "oracle_dw_rows", "oracle_loss_fwd_bwd", "oracle_num_threads", "oracle_loss_from_lp_ex",
+                  "oracle_ratio_stats"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -199,3 +203,45 @@ def loss_fwd_bwd(H, W, ids, lp_rollout, rewards, seg_offsets, group_ids, n_group
                                    _ptr(g), n, R, n_groups, d, V, _ptr(loss), _ptr(dH), _ptr(dW),
                                    _ptr(lp), _ptr(lse), _ptr(w), _ptr(kappa)), "loss_fwd_bwd")
     return dict(loss=float(loss[0]), lp=lp, lse=lse, w=w, kappa=kappa, dH=dH, dW=dW)
+
+
+CLIP, GATE, MASK = 1, 2, 4
+
+
+def loss_from_lp_ex(lp, lp_rollout, rewards, seg_offsets, group_ids, n_groups, flags=0, clip_max=float("inf"),
+                    gate_lo=0.0, gate_hi=float("inf"), mask=None, n_resp_total=0):
+    """(loss, w, kappa) of the loss-stage variants (truncated IS, sequence gate, token mask,
+    global response count); flags = 0 reproduces loss_from_lp.  Readings in oracle.c."""
+    lib = _load()
+    lp = np.ascontiguousarray(lp, dtype=np.float64)
+    lr = np.ascontiguousarray(lp_rollout, dtype=np.float64)
+    r = np.ascontiguousarray(rewards, dtype=np.float64)
+    off = np.ascontiguousarray(seg_offsets, dtype=np.int64)
+    g = np.ascontiguousarray(group_ids, dtype=np.int32)
+    mk = None if mask is None else np.ascontiguousarray(mask, dtype=np.uint8)
+    n, R = lp.shape[0], r.shape[0]
+    w = np.empty(n, np.float64)
+    kappa = np.empty(n, np.float64)
+    loss = np.zeros(1, np.float64)
+    _check(lib.oracle_loss_from_lp_ex(_ptr(lp), _ptr(lr), _ptr(r), _ptr(off), _ptr(g), n, R, n_groups, flags,
+                                      clip_max, gate_lo, gate_hi, _ptr(mk), n_resp_total, _ptr(w), _ptr(kappa),
+                                      _ptr(loss)), "loss_from_lp_ex")
+    return float(loss[0]), w, kappa
+
+
+STAT_NAMES = ("k1", "k2", "k3", "w_min", "w_max", "dev_max", "dev_median", "dev_peak_over_median", "count")
+
+
+def ratio_stats(lp, lp_rollout, seg_offsets, mask=None):
+    """Ratio diagnostics (dict keyed by STAT_NAMES) and the per-response mean ratio."""
+    lib = _load()
+    lp = np.ascontiguousarray(lp, dtype=np.float64)
+    lr = np.ascontiguousarray(lp_rollout, dtype=np.float64)
+    off = np.ascontiguousarray(seg_offsets, dtype=np.int64)
+    mk = None if mask is None else np.ascontiguousarray(mask, dtype=np.uint8)
+    n, R = lp.shape[0], off.shape[0] - 1
+    stats = np.empty(9, np.float64)
+    rm = np.empty(R, np.float64)
+    _check(lib.oracle_ratio_stats(_ptr(lp), _ptr(lr), _ptr(off), n, R, _ptr(mk), _ptr(stats), _ptr(rm)),
+           "ratio_stats")
+    return dict(zip(STAT_NAMES, stats.tolist())), rm

@@ -291,3 +291,130 @@ int oracle_num_threads(void) {
   return 1;
 #endif
 }
+
+/* ------------------------------------------------------------------------------------
+ * Variants of the loss stage (the baselines the pages contrast REINFORCE Zero with) and
+ * diagnostics of the ratio.  Readings, as the pages give no formulas:
+ *   - truncated IS ("clipping the importance weights can introduce bias", [A] section
+ *     "REINFORCE Zero removes the mismatch first"): w -> min(w, clip_max) in the
+ *     coefficient of each token's gradient, held constant;
+ *   - sequence gate (the standard-kernel baseline on OSWorld, [A] section "Zero mismatch
+ *     expands to newer models"): response i is kept iff gate_lo <= exp(mean_t (lp - lp_rollout))
+ *     <= gate_hi over its counted tokens; a rejected response contributes nothing but its
+ *     reward still enters its group's mean, and N still counts it;
+ *   - token mask: only tokens with mask 1 count; L_i is the number of counted tokens of
+ *     response i (a response with none contributes nothing);
+ *   - n_resp_total > 0 replaces N (responses of the whole data-parallel batch).
+ * kappa_t = -A_i * s_i * m_t * g(w_t) / (N * L_i) and loss = sum_t kappa_t.
+ * ------------------------------------------------------------------------------------ */
+#define ORACLE_CLIP 1
+#define ORACLE_GATE 2
+#define ORACLE_MASK 4
+
+int oracle_loss_from_lp_ex(const double *lp, const double *lp_rollout, const double *rewards,
+                           const int64_t *off, const int32_t *gid, int64_t n, int32_t R, int32_t G,
+                           int32_t flags, double clip_max, double gate_lo, double gate_hi,
+                           const uint8_t *mask, int32_t n_resp_total, double *w_out, double *kappa_out,
+                           double *loss_out) {
+  if (n <= 0 || R <= 0) return 1;
+  if (check_offsets(off, R, n)) return 1;
+  double *A = (double *)malloc(sizeof(double) * (size_t)R);
+  if (!A) return 2;
+  int err = oracle_advantages(rewards, gid, R, G, A);
+  if (err) {
+    free(A);
+    return err;
+  }
+  const double N = n_resp_total > 0 ? (double)n_resp_total : (double)R;
+  double loss = 0.0;
+  for (int32_t i = 0; i < R; ++i) {
+    double L = 0.0, logsum = 0.0;
+    for (int64_t t = off[i]; t < off[i + 1]; ++t) {
+      const int counted = (flags & ORACLE_MASK) ? (mask[t] != 0) : 1;
+      if (counted) {
+        L += 1.0;
+        logsum += lp[t] - lp_rollout[t];
+      }
+    }
+    int keep = L > 0.0;
+    if (keep && (flags & ORACLE_GATE)) {
+      const double g = exp(logsum / L); /* geometric-mean ratio of the response */
+      keep = (g >= gate_lo && g <= gate_hi);
+    }
+    double wsum = 0.0;
+    for (int64_t t = off[i]; t < off[i + 1]; ++t) {
+      const int counted = (flags & ORACLE_MASK) ? (mask[t] != 0) : 1;
+      double w = exp(lp[t] - lp_rollout[t]);
+      if (w_out) w_out[t] = w;
+      if ((flags & ORACLE_CLIP) && w > clip_max) w = clip_max;
+      const double k = (keep && counted) ? -A[i] * w / (N * L) : 0.0;
+      if (kappa_out) kappa_out[t] = k;
+      if (keep && counted) wsum += w;
+    }
+    if (keep) loss += A[i] * (wsum / L);
+  }
+  *loss_out = -loss / N;
+  free(A);
+  return 0;
+}
+
+static int cmp_double(const void *a, const void *b) {
+  const double x = *(const double *)a, y = *(const double *)b;
+  return (x > y) - (x < y);
+}
+
+/*
+ * Diagnostics of the ratio over the counted tokens (mask may be NULL), [A] sections
+ * "Asynchronous training has two different gaps" (importance-weight deviation, peak vs
+ * median) and "Reported results include 2.40 times higher throughput" (rollout-to-learner
+ * KL).  stats: [0] k1 = mean(lp_rollout - lp); [1] k2 = mean((lp - lp_rollout)^2 / 2);
+ * [2] k3 = mean(w - 1 - (lp - lp_rollout)); [3] min w; [4] max w; [5] max |w - 1|;
+ * [6] lower median of |w - 1| (element of rank floor((m - 1) / 2) of the m counted tokens
+ * in ascending order); [7] [5] / [6]; [8] m.  resp_mean_w (may be NULL): per response,
+ * the mean of w over its counted tokens (0 when it has none).
+ */
+int oracle_ratio_stats(const double *lp, const double *lp_rollout, const int64_t *off, int64_t n, int32_t R,
+                       const uint8_t *mask, double *stats, double *resp_mean_w) {
+  if (n <= 0 || R <= 0 || check_offsets(off, R, n)) return 1;
+  double *dev = (double *)malloc(sizeof(double) * (size_t)n);
+  if (!dev) return 2;
+  int64_t m = 0;
+  double k1 = 0, k2 = 0, k3 = 0, wmin = INFINITY, wmax = -INFINITY, dmax = 0;
+  for (int32_t i = 0; i < R; ++i) {
+    double ws = 0.0;
+    int64_t c = 0;
+    for (int64_t t = off[i]; t < off[i + 1]; ++t) {
+      if (mask && !mask[t]) continue;
+      const double x = lp[t] - lp_rollout[t];
+      const double w = exp(x);
+      k1 += -x;
+      k2 += 0.5 * x * x;
+      k3 += w - 1.0 - x;
+      if (w < wmin) wmin = w;
+      if (w > wmax) wmax = w;
+      const double d = fabs(w - 1.0);
+      if (d > dmax) dmax = d;
+      dev[m++] = d;
+      ws += w;
+      ++c;
+    }
+    if (resp_mean_w) resp_mean_w[i] = c ? ws / (double)c : 0.0;
+  }
+  if (m == 0) {
+    free(dev);
+    return 1;
+  }
+  qsort(dev, (size_t)m, sizeof(double), cmp_double);
+  const double med = dev[(m - 1) / 2];
+  stats[0] = k1 / (double)m;
+  stats[1] = k2 / (double)m;
+  stats[2] = k3 / (double)m;
+  stats[3] = wmin;
+  stats[4] = wmax;
+  stats[5] = dmax;
+  stats[6] = med;
+  stats[7] = med > 0 ? dmax / med : INFINITY;
+  stats[8] = (double)m;
+  free(dev);
+  return 0;
+}
