@@ -137,6 +137,85 @@ rz_status rz_segment_loss(const float* lp, const float* lp_rollout, const float*
                           int32_t n_groups, float* loss, float* kappa_out, float* w_out, void* workspace,
                           size_t ws_bytes, void* stream);
 
+/*
+ * Variants of the loss stage: the baselines the pages contrast REINFORCE Zero with
+ * ("vLLM says aligned kernels…", sections "REINFORCE Zero removes the mismatch first" and
+ * "Zero mismatch expands to newer models"), plus a global response count for
+ * data-parallel shards.  A NULL options pointer, or flags == 0 with n_resp_total == 0,
+ * gives exactly (bit for bit) rz_loss_fwd_bwd / rz_segment_loss.
+ *
+ *   kappa_t = -A_i * s_i * m_t * g(w_t) / (N * L_i),   loss = sum_t kappa_t
+ *
+ *   RZ_LOSS_CLIP_IS    g(w) = min(w, clip_max) (clip_max > 0): truncated importance
+ *                      weights, used as a constant coefficient of the token's gradient
+ *                      (the reported loss is the same sum with the capped weights).
+ *   RZ_LOSS_SEQ_GATE   s_i = 1 iff gate_lo <= exp(mean over the counted tokens of response i
+ *                      of (lp - lp_rollout)) <= gate_hi, else 0; a rejected response keeps
+ *                      its reward in its group's mean and stays counted in N.
+ *                      rz_loss_fwd_bwd_ex then runs the forward twice (the gate needs every
+ *                      logprob before any kappa).
+ *   RZ_LOSS_TOKEN_MASK m_t = token_mask[t] != 0 (device [n_tok] bytes, 4-byte aligned);
+ *                      L_i counts only the tokens with m_t = 1 (a response with none
+ *                      contributes nothing).
+ *   n_resp_total > 0   N = n_resp_total instead of n_resp.
+ * Invalid options (unknown flag bits, clip_max <= 0, gate_lo > gate_hi, a missing mask,
+ * n_resp_total < 0) return RZ_ERR_INVALID_ARG.
+ */
+#define RZ_LOSS_CLIP_IS 1
+#define RZ_LOSS_SEQ_GATE 2
+#define RZ_LOSS_TOKEN_MASK 4
+
+typedef struct {
+  int32_t flags;
+  float clip_max;
+  double gate_lo, gate_hi;
+  const uint8_t* token_mask;
+  int32_t n_resp_total;
+} rz_loss_options;
+
+/* rz_loss_fwd_bwd with loss-stage options (same workspace size). */
+rz_status rz_loss_fwd_bwd_ex(const rz_bf16* H, const rz_bf16* W_head, const int32_t* token_ids,
+                             const float* lp_rollout, const float* rewards, const int64_t* seg_offsets,
+                             const int32_t* group_ids, int64_t n_tok, int32_t n_resp, int32_t n_groups, int32_t d,
+                             int32_t V, const rz_loss_options* options, float* loss, rz_bf16* dH, float* dW,
+                             float* lp_out, float* kappa_out, void* workspace, size_t ws_bytes, void* stream);
+
+/* rz_segment_loss with loss-stage options (same workspace size). */
+rz_status rz_segment_loss_ex(const float* lp, const float* lp_rollout, const float* rewards,
+                             const int64_t* seg_offsets, const int32_t* group_ids, int64_t n_tok, int32_t n_resp,
+                             int32_t n_groups, const rz_loss_options* options, float* loss, float* kappa_out,
+                             float* w_out, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Diagnostics of the ratio w_t = exp(lp_t - lp_rollout_t) over the counted tokens
+ * (token_mask nullable) — the pages' observables: the importance-weight deviation peak
+ * against its median ("vLLM says aligned kernels…", section "Asynchronous training has two
+ * different gaps") and the rollout-to-learner KL (section "Reported results include 2.40
+ * times higher throughput").
+ *
+ *   stats_out [9] fp64, device: k1 = mean(lp_rollout - lp), k2 = mean((lp - lp_rollout)^2/2),
+ *             k3 = mean(w - 1 - (lp - lp_rollout)), min w, max w, max |w - 1|, the exact
+ *             lower median of |w - 1| (rank floor((m-1)/2) of the m counted tokens), their
+ *             ratio (peak / median), m
+ *   resp_mean_ratio_out [n_resp] fp32, device, nullable: mean w over each response's counted
+ *             tokens (0 if none)
+ * Deterministic; w is computed exactly as the loss stage computes it.
+ */
+size_t rz_workspace_bytes_ratio_stats(int64_t n_tok, int32_t n_resp);
+rz_status rz_ratio_stats(const float* lp, const float* lp_rollout, const int64_t* seg_offsets, int64_t n_tok,
+                         int32_t n_resp, const uint8_t* token_mask, double* stats_out, float* resp_mean_ratio_out,
+                         void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Frobenius norms of the gradients: norms_out[0] = ||dH|| (bf16 [n_tok, d]),
+ * norms_out[1] = ||dW|| (fp32 [V, d]), fp64, device; fixed-order reductions (deterministic).
+ * The pages report the largest gradient norm before clipping ("vLLM says aligned
+ * kernels…", section "Reported results include 2.40 times higher throughput").
+ */
+size_t rz_workspace_bytes_grad_norms(void);
+rz_status rz_grad_norms(const rz_bf16* dH, const float* dW, int64_t n_tok, int32_t d, int32_t V, double* norms_out,
+                        void* workspace, size_t ws_bytes, void* stream);
+
 /* Kernel kinds reported per launch by rz_loss_fwd_bwd_timed. */
 #define RZ_KERNEL_LMHEAD_LSE 0    /* fused LM head + online log-sum-exp + gather (tensor cores) */
 #define RZ_KERNEL_MERGE_LSE 1     /* fixed-order merge of the vocabulary-segment partials       */

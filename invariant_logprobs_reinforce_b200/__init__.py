@@ -26,8 +26,34 @@ STATUS_NAMES = {
 EXPORTED_SYMBOLS = (
     "rz_status_string", "rz_workspace_bytes_logprobs", "rz_workspace_bytes_loss", "rz_workspace_bytes_segment_loss",
     "rz_token_logprobs", "rz_loss_fwd_bwd", "rz_segment_loss", "rz_read_device_status", "rz_num_launches_loss",
-    "rz_loss_fwd_bwd_timed", "rz_token_logprobs_noalloc",
+    "rz_loss_fwd_bwd_timed", "rz_token_logprobs_noalloc", "rz_loss_fwd_bwd_ex", "rz_segment_loss_ex",
+    "rz_workspace_bytes_ratio_stats", "rz_ratio_stats", "rz_workspace_bytes_grad_norms", "rz_grad_norms",
 )
+RZ_LOSS_CLIP_IS, RZ_LOSS_SEQ_GATE, RZ_LOSS_TOKEN_MASK = 1, 2, 4
+STAT_NAMES = ("k1", "k2", "k3", "w_min", "w_max", "dev_max", "dev_median", "dev_peak_over_median", "count")
+
+
+class rz_loss_options(ctypes.Structure):
+    """Mirror of the C struct rz_loss_options (include/rz.h)."""
+    _fields_ = [("flags", ctypes.c_int32), ("clip_max", ctypes.c_float), ("gate_lo", ctypes.c_double),
+                ("gate_hi", ctypes.c_double), ("token_mask", ctypes.c_void_p), ("n_resp_total", ctypes.c_int32)]
+
+
+def loss_options(clip_max=None, gate=None, token_mask=None, n_resp_total=0):
+    """Build rz_loss_options: clip_max (float), gate ((lo, hi)), token_mask (uint8 CUDA tensor)."""
+    o = rz_loss_options()
+    o.flags, o.clip_max, o.gate_lo, o.gate_hi, o.token_mask = 0, 0.0, 0.0, 0.0, None
+    if clip_max is not None:
+        o.flags |= RZ_LOSS_CLIP_IS
+        o.clip_max = float(clip_max)
+    if gate is not None:
+        o.flags |= RZ_LOSS_SEQ_GATE
+        o.gate_lo, o.gate_hi = float(gate[0]), float(gate[1])
+    if token_mask is not None:
+        o.flags |= RZ_LOSS_TOKEN_MASK
+        o.token_mask = token_mask.data_ptr()
+    o.n_resp_total = int(n_resp_total)
+    return o
 KERNEL_KINDS = ("lmhead_lse", "merge_lse", "response_coef", "token_kappa", "loss_final", "dz", "dh", "dw",
                 "block_first")
 
@@ -69,6 +95,20 @@ def lib() -> ctypes.CDLL:
         L.rz_num_launches_loss.restype = i32
         L.rz_token_logprobs_noalloc.argtypes = [P, P, P, i64, i32, i32, P, P, P]
         L.rz_token_logprobs_noalloc.restype = ctypes.c_int
+        L.rz_loss_fwd_bwd_ex.argtypes = [P, P, P, P, P, P, P, i64, i32, i32, i32, i32, ctypes.POINTER(rz_loss_options),
+                                          P, P, P, P, P, P, sz, P]
+        L.rz_loss_fwd_bwd_ex.restype = ctypes.c_int
+        L.rz_segment_loss_ex.argtypes = [P, P, P, P, P, i64, i32, i32, ctypes.POINTER(rz_loss_options), P, P, P, P,
+                                          sz, P]
+        L.rz_segment_loss_ex.restype = ctypes.c_int
+        L.rz_workspace_bytes_ratio_stats.argtypes = [i64, i32]
+        L.rz_workspace_bytes_ratio_stats.restype = sz
+        L.rz_ratio_stats.argtypes = [P, P, P, i64, i32, P, P, P, P, sz, P]
+        L.rz_ratio_stats.restype = ctypes.c_int
+        L.rz_workspace_bytes_grad_norms.argtypes = []
+        L.rz_workspace_bytes_grad_norms.restype = sz
+        L.rz_grad_norms.argtypes = [P, P, i64, i32, i32, P, P, sz, P]
+        L.rz_grad_norms.restype = ctypes.c_int
         L.rz_read_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
         L.rz_read_device_status.restype = ctypes.c_int
         _lib = L
@@ -256,3 +296,74 @@ def rz_read_device_status(workspace, stream=None):
     bits = ctypes.c_int32(0)
     code = lib().rz_read_device_status(_ptr(workspace), _stream_handle(stream), ctypes.byref(bits))
     return int(code), int(bits.value)
+
+
+def rz_loss_fwd_bwd_ex(H, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids, n_groups, options,
+                       workspace=None, stream=None):
+    """rz_loss_fwd_bwd with rz_loss_options (see loss_options).  Returns the same dict."""
+    torch = _torch()
+    _need(H, torch.bfloat16, "H")
+    dev = H.device
+    n, d = H.shape
+    V = W_head.shape[0]
+    R = rewards.shape[0]
+    out = dict(loss=torch.empty(1, dtype=torch.float32, device=dev),
+               dH=torch.empty((n, d), dtype=torch.bfloat16, device=dev),
+               dW=torch.empty((V, d), dtype=torch.float32, device=dev),
+               lp=torch.empty(n, dtype=torch.float32, device=dev),
+               kappa=torch.empty(n, dtype=torch.float32, device=dev))
+    ws = _workspace(rz_workspace_bytes_loss(n, R, n_groups, d, V), workspace, dev)
+    code = lib().rz_loss_fwd_bwd_ex(_ptr(H), _ptr(W_head), _ptr(token_ids), _ptr(lp_rollout), _ptr(rewards),
+                                    _ptr(seg_offsets), _ptr(group_ids), n, R, n_groups, d, V,
+                                    ctypes.byref(options) if options is not None else None, _ptr(out["loss"]),
+                                    _ptr(out["dH"]), _ptr(out["dW"]), _ptr(out["lp"]), _ptr(out["kappa"]), _ptr(ws),
+                                    ws.numel(), _stream_handle(stream))
+    _check(code, "rz_loss_fwd_bwd_ex")
+    out["workspace"] = ws
+    return out
+
+
+def rz_segment_loss_ex(lp, lp_rollout, rewards, seg_offsets, group_ids, n_groups, options, want_w=False,
+                       workspace=None, stream=None):
+    """rz_segment_loss with rz_loss_options.  Returns dict(loss, kappa, w, workspace)."""
+    torch = _torch()
+    dev = lp.device
+    n = lp.shape[0]
+    R = rewards.shape[0]
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    kappa = torch.empty(n, dtype=torch.float32, device=dev)
+    w = torch.empty(n, dtype=torch.float32, device=dev) if want_w else None
+    ws = _workspace(rz_workspace_bytes_segment_loss(n, R, n_groups), workspace, dev)
+    code = lib().rz_segment_loss_ex(_ptr(lp), _ptr(lp_rollout), _ptr(rewards), _ptr(seg_offsets), _ptr(group_ids), n,
+                                    R, n_groups, ctypes.byref(options) if options is not None else None, _ptr(loss),
+                                    _ptr(kappa), _ptr(w), _ptr(ws), ws.numel(), _stream_handle(stream))
+    _check(code, "rz_segment_loss_ex")
+    return dict(loss=loss, kappa=kappa, w=w, workspace=ws)
+
+
+def rz_ratio_stats(lp, lp_rollout, seg_offsets, token_mask=None, want_resp_mean=True, workspace=None, stream=None):
+    """Ratio diagnostics.  Returns (stats tensor [9] fp64 on device, per-response mean ratio or None)."""
+    torch = _torch()
+    dev = lp.device
+    n = lp.shape[0]
+    R = seg_offsets.shape[0] - 1
+    stats = torch.empty(9, dtype=torch.float64, device=dev)
+    rm = torch.empty(R, dtype=torch.float32, device=dev) if want_resp_mean else None
+    ws = _workspace(int(lib().rz_workspace_bytes_ratio_stats(n, R)), workspace, dev)
+    code = lib().rz_ratio_stats(_ptr(lp), _ptr(lp_rollout), _ptr(seg_offsets), n, R, _ptr(token_mask), _ptr(stats),
+                                _ptr(rm), _ptr(ws), ws.numel(), _stream_handle(stream))
+    _check(code, "rz_ratio_stats")
+    return stats, rm
+
+
+def rz_grad_norms(dH, dW, workspace=None, stream=None):
+    """(||dH||, ||dW||) as an fp64 device tensor [2]."""
+    torch = _torch()
+    dev = dW.device
+    n, d = dH.shape
+    V = dW.shape[0]
+    out = torch.empty(2, dtype=torch.float64, device=dev)
+    ws = _workspace(int(lib().rz_workspace_bytes_grad_norms()), workspace, dev)
+    code = lib().rz_grad_norms(_ptr(dH), _ptr(dW), n, d, V, _ptr(out), _ptr(ws), ws.numel(), _stream_handle(stream))
+    _check(code, "rz_grad_norms")
+    return out

@@ -53,7 +53,7 @@ struct Layout {
   size_t part_m = 0, part_s = 0, zy = 0;
   int64_t part_ld = 0;
   size_t lp = 0, lse = 0, kappa = 0;
-  size_t coef = 0, gsum = 0, gcnt = 0, bsum = 0, bfirst = 0;
+  size_t coef = 0, gsum = 0, gcnt = 0, bsum = 0, bfirst = 0, counted = 0;
   size_t tile_max = 0, dz = 0;
   size_t total = 0;
 };
@@ -85,6 +85,7 @@ Layout make_layout(int64_t n, int32_t R, int32_t G, int32_t V, Path path) {
     L.gcnt = take(sizeof(int) * G);
     L.bsum = take(sizeof(double) * kappa_blocks(n));
     L.bfirst = take(sizeof(int) * kappa_blocks(n));
+    L.counted = take(sizeof(int) * R);
   }
   if (path == Path::Loss) {
     const int64_t C = chunk_capacity(n);
@@ -265,9 +266,46 @@ rz_status run_forward(const rz_bf16* H, const rz_bf16* W, const int32_t* ids, in
   return RZ_OK;
 }
 
-// Loss stage, part 1: checks, group sums, coef_i = -A_i/(N L_i), first response per block.
+// Loss-stage options after defaults: no cap (+inf), no gate, no mask, N = n_resp.
+struct LossOpts {
+  float clip_max = INFINITY;
+  bool gate = false;
+  double gate_lo = 0.0, gate_hi = INFINITY;
+  const uint8_t* mask = nullptr;
+  double N = 0.0;
+};
+
+bool resolve_options(const rz_loss_options* o, int32_t n_resp, LossOpts* out) {
+  LossOpts r;
+  r.N = static_cast<double>(n_resp);
+  if (o != nullptr) {
+    if (o->flags & ~(RZ_LOSS_CLIP_IS | RZ_LOSS_SEQ_GATE | RZ_LOSS_TOKEN_MASK)) return false;
+    if (o->flags & RZ_LOSS_CLIP_IS) {
+      if (!(o->clip_max > 0.0f)) return false;
+      r.clip_max = o->clip_max;
+    }
+    if (o->flags & RZ_LOSS_SEQ_GATE) {
+      if (!(o->gate_lo <= o->gate_hi)) return false;
+      r.gate = true;
+      r.gate_lo = o->gate_lo;
+      r.gate_hi = o->gate_hi;
+    }
+    if (o->flags & RZ_LOSS_TOKEN_MASK) {
+      if (o->token_mask == nullptr || !aligned(o->token_mask, 4)) return false;
+      r.mask = o->token_mask;
+    }
+    if (o->n_resp_total < 0) return false;
+    if (o->n_resp_total > 0) r.N = static_cast<double>(o->n_resp_total);
+  }
+  *out = r;
+  return true;
+}
+
+// Loss stage, part 1: checks, group sums, coef_i = -A_i/(N L_i) (L_i = counted tokens
+// under a mask), first response per block.
 rz_status run_loss_setup(const float* rewards, const int64_t* off, const int32_t* gid, int64_t n, int32_t R,
-                         int32_t G, void* ws, const Layout& L, cudaStream_t stream, Recorder* rec) {
+                         int32_t G, const LossOpts& opt, void* ws, const Layout& L, cudaStream_t stream,
+                         Recorder* rec) {
   int* status = at<int>(ws, L.status);
   int* flags = status + 1;  // cleared together with the status word
   double* gsum = at<double>(ws, L.gsum);
@@ -279,7 +317,14 @@ rz_status run_loss_setup(const float* rewards, const int64_t* off, const int32_t
   coef_groups_kernel<<<static_cast<unsigned>(ceil_div(G, kCoefThreads)), kCoefThreads, 0, stream>>>(
       rewards, gid, R, G, gsum, gcnt, flags);
   if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
-  coef_kernel<<<rb, kCoefThreads, 0, stream>>>(rewards, off, gid, R, G, gsum, gcnt, at<float>(ws, L.coef));
+  int* counted = nullptr;
+  if (opt.mask != nullptr) {
+    counted = at<int>(ws, L.counted);
+    masked_count_kernel<<<static_cast<unsigned>(ceil_div(R, 8)), 256, 0, stream>>>(opt.mask, off, R, counted);
+    if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
+  }
+  coef_kernel<<<rb, kCoefThreads, 0, stream>>>(rewards, off, gid, R, G, opt.N, counted, gsum, gcnt,
+                                               at<float>(ws, L.coef));
   if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
   rec_end(rec, stream);
   const int nb = kappa_blocks(n);
@@ -291,16 +336,25 @@ rz_status run_loss_setup(const float* rewards, const int64_t* off, const int32_t
   return RZ_OK;
 }
 
+// Sequence gate: zero the coefficient of every response whose geometric-mean ratio lies
+// outside [gate_lo, gate_hi] (needs lp of all tokens).
+rz_status run_gate(const float* lp, const float* lp_roll, const int64_t* off, int32_t R, const LossOpts& opt,
+                   void* ws, const Layout& L, cudaStream_t stream) {
+  gate_kernel<<<static_cast<unsigned>(ceil_div(R, 8)), 256, 0, stream>>>(lp, lp_roll, opt.mask, off, R, opt.gate_lo,
+                                                                      opt.gate_hi, at<float>(ws, L.coef));
+  return cudaGetLastError() == cudaSuccess ? RZ_OK : RZ_ERR_CUDA;
+}
+
 // Loss stage, part 2: kappa and ratio for the 4096-token blocks [blk0, blk0 + nblk).
 rz_status run_kappa(const float* lp, const float* lp_roll, const int64_t* off, int64_t n, int32_t R, int blk0,
-                    int nblk, float* kappa, float* w_out, void* ws, const Layout& L, cudaStream_t stream,
-                    Recorder* rec) {
+                    int nblk, const LossOpts& opt, float* kappa, float* w_out, void* ws, const Layout& L,
+                    cudaStream_t stream, Recorder* rec) {
   const int vec_ok = aligned(lp, 16) && aligned(lp_roll, 16) && aligned(kappa, 16) &&
-                     (w_out == nullptr || aligned(w_out, 16));
+                     (w_out == nullptr || aligned(w_out, 16)) && (opt.mask == nullptr || aligned(opt.mask, 4));
   rec_begin(rec, RZ_KERNEL_TOKEN_KAPPA, stream);
   token_kappa_kernel<<<nblk, kKappaThreads, 0, stream>>>(lp, lp_roll, off, R, at<float>(ws, L.coef),
-                                                         at<int>(ws, L.bfirst), n, blk0, vec_ok, kappa, w_out,
-                                                         at<double>(ws, L.bsum));
+                                                         at<int>(ws, L.bfirst), n, blk0, vec_ok, opt.mask,
+                                                         opt.clip_max, kappa, w_out, at<double>(ws, L.bsum));
   if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
   rec_end(rec, stream);
   return RZ_OK;
@@ -316,11 +370,16 @@ rz_status run_loss_final(int64_t n, float* loss, void* ws, const Layout& L, cuda
 }
 
 rz_status run_segment_loss(const float* lp, const float* lp_roll, const float* rewards, const int64_t* off,
-                           const int32_t* gid, int64_t n, int32_t R, int32_t G, float* loss, float* kappa,
-                           float* w_out, void* ws, const Layout& L, cudaStream_t stream, Recorder* rec) {
-  rz_status r = run_loss_setup(rewards, off, gid, n, R, G, ws, L, stream, rec);
+                           const int32_t* gid, int64_t n, int32_t R, int32_t G, const LossOpts& opt, float* loss,
+                           float* kappa, float* w_out, void* ws, const Layout& L, cudaStream_t stream,
+                           Recorder* rec) {
+  rz_status r = run_loss_setup(rewards, off, gid, n, R, G, opt, ws, L, stream, rec);
   if (r != RZ_OK) return r;
-  r = run_kappa(lp, lp_roll, off, n, R, 0, kappa_blocks(n), kappa, w_out, ws, L, stream, rec);
+  if (opt.gate) {
+    r = run_gate(lp, lp_roll, off, R, opt, ws, L, stream);
+    if (r != RZ_OK) return r;
+  }
+  r = run_kappa(lp, lp_roll, off, n, R, 0, kappa_blocks(n), opt, kappa, w_out, ws, L, stream, rec);
   if (r != RZ_OK) return r;
   return run_loss_final(n, loss, ws, L, stream, rec);
 }
@@ -434,10 +493,11 @@ RZ_API rz_status rz_token_logprobs(const rz_bf16* H, const rz_bf16* W_head, cons
   return run_forward(H, W_head, token_ids, 0, n_tok, d, V, lp_out, lse_out, workspace, L, false, st, nullptr);
 }
 
-RZ_API rz_status rz_segment_loss(const float* lp, const float* lp_rollout, const float* rewards,
-                          const int64_t* seg_offsets, const int32_t* group_ids, int64_t n_tok, int32_t n_resp,
-                          int32_t n_groups, float* loss, float* kappa_out, float* w_out, void* workspace,
-                          size_t ws_bytes, void* stream) {
+namespace {
+rz_status segment_loss_impl(const float* lp, const float* lp_rollout, const float* rewards,
+                            const int64_t* seg_offsets, const int32_t* group_ids, int64_t n_tok, int32_t n_resp,
+                            int32_t n_groups, const rz_loss_options* options, float* loss, float* kappa_out,
+                            float* w_out, void* workspace, size_t ws_bytes, void* stream) {
   if (n_tok < 1 || n_tok >= (int64_t{1} << 31) || n_resp < 1 || n_groups < 1) return RZ_ERR_INVALID_ARG;
   if (!lp || !lp_rollout || !rewards || !seg_offsets || !group_ids || !loss || !kappa_out || !workspace)
     return RZ_ERR_INVALID_ARG;
@@ -445,12 +505,31 @@ RZ_API rz_status rz_segment_loss(const float* lp, const float* lp_rollout, const
       !aligned(group_ids, 4) || !aligned(loss, 4) || !aligned(kappa_out, 4) || (w_out && !aligned(w_out, 4)) ||
       !aligned(workspace, kAlign))
     return RZ_ERR_INVALID_ARG;
+  LossOpts opt;
+  if (!resolve_options(options, n_resp, &opt)) return RZ_ERR_INVALID_ARG;
   const Layout L = make_layout(n_tok, n_resp, n_groups, 1, Path::LossStage);
   if (ws_bytes < L.total) return RZ_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(at<int>(workspace, L.status), 0, 16, st) != cudaSuccess) return RZ_ERR_CUDA;
-  return run_segment_loss(lp, lp_rollout, rewards, seg_offsets, group_ids, n_tok, n_resp, n_groups, loss, kappa_out,
-                          w_out, workspace, L, st, nullptr);
+  return run_segment_loss(lp, lp_rollout, rewards, seg_offsets, group_ids, n_tok, n_resp, n_groups, opt, loss,
+                          kappa_out, w_out, workspace, L, st, nullptr);
+}
+}  // namespace
+
+RZ_API rz_status rz_segment_loss(const float* lp, const float* lp_rollout, const float* rewards,
+                                 const int64_t* seg_offsets, const int32_t* group_ids, int64_t n_tok, int32_t n_resp,
+                                 int32_t n_groups, float* loss, float* kappa_out, float* w_out, void* workspace,
+                                 size_t ws_bytes, void* stream) {
+  return segment_loss_impl(lp, lp_rollout, rewards, seg_offsets, group_ids, n_tok, n_resp, n_groups, nullptr, loss,
+                           kappa_out, w_out, workspace, ws_bytes, stream);
+}
+
+RZ_API rz_status rz_segment_loss_ex(const float* lp, const float* lp_rollout, const float* rewards,
+                                    const int64_t* seg_offsets, const int32_t* group_ids, int64_t n_tok,
+                                    int32_t n_resp, int32_t n_groups, const rz_loss_options* options, float* loss,
+                                    float* kappa_out, float* w_out, void* workspace, size_t ws_bytes, void* stream) {
+  return segment_loss_impl(lp, lp_rollout, rewards, seg_offsets, group_ids, n_tok, n_resp, n_groups, options, loss,
+                           kappa_out, w_out, workspace, ws_bytes, stream);
 }
 
 }  // extern "C"
@@ -459,9 +538,12 @@ namespace {
 rz_status loss_fwd_bwd_impl(const rz_bf16* H, const rz_bf16* W_head, const int32_t* token_ids,
                           const float* lp_rollout, const float* rewards, const int64_t* seg_offsets,
                           const int32_t* group_ids, int64_t n_tok, int32_t n_resp, int32_t n_groups, int32_t d,
-                          int32_t V, float* loss, rz_bf16* dH, float* dW, float* lp_out, float* kappa_out,
-                          void* workspace, size_t ws_bytes, void* stream, Recorder* rec) {
+                          int32_t V, const rz_loss_options* options, float* loss, rz_bf16* dH, float* dW,
+                          float* lp_out, float* kappa_out, void* workspace, size_t ws_bytes, void* stream,
+                          Recorder* rec) {
   if (n_tok < 1 || n_tok >= (int64_t{1} << 31) || n_resp < 1 || n_groups < 1) return RZ_ERR_INVALID_ARG;
+  LossOpts opt;
+  if (!resolve_options(options, n_resp, &opt)) return RZ_ERR_INVALID_ARG;
   if (!shape_ok(d, V)) return RZ_ERR_UNSUPPORTED_SHAPE;
   if (!H || !W_head || !token_ids || !lp_rollout || !rewards || !seg_offsets || !group_ids || !loss || !dH ||
       !dW || !workspace)
@@ -478,8 +560,19 @@ rz_status loss_fwd_bwd_impl(const rz_bf16* H, const rz_bf16* W_head, const int32
   float* lp = lp_out ? lp_out : at<float>(workspace, L.lp);
   float* lse = at<float>(workspace, L.lse);
   float* kappa = kappa_out ? kappa_out : at<float>(workspace, L.kappa);
-  rz_status r = run_loss_setup(rewards, seg_offsets, group_ids, n_tok, n_resp, n_groups, workspace, L, st, rec);
+  rz_status r = run_loss_setup(rewards, seg_offsets, group_ids, n_tok, n_resp, n_groups, opt, workspace, L, st, rec);
   if (r != RZ_OK) return r;
+  if (opt.gate) {
+    // the gate needs every token's logprob before any kappa: one forward pass first
+    // (same kernels, so the same lp bits as the pass that follows)
+    for (int64_t c0 = 0; c0 < n_tok; c0 += kChunkTokens) {
+      const int64_t rows = std::min<int64_t>(kChunkTokens, n_tok - c0);
+      r = run_forward(H, W_head, token_ids, c0, rows, d, V, lp, lse, workspace, L, false, st, rec);
+      if (r != RZ_OK) return r;
+    }
+    r = run_gate(lp, lp_rollout, seg_offsets, n_resp, opt, workspace, L, st);
+    if (r != RZ_OK) return r;
+  }
   // chunk by chunk: forward (with the exponentials kept), kappa, backward; the loss
   // partials are per 4096-token block, so the loss does not depend on the chunking
   for (int64_t c0 = 0; c0 < n_tok; c0 += kChunkTokens) {
@@ -488,7 +581,8 @@ rz_status loss_fwd_bwd_impl(const rz_bf16* H, const rz_bf16* W_head, const int32
     if (r != RZ_OK) return r;
     const int blk0 = static_cast<int>(c0 / kKappaBlockTokens);
     const int nblk = static_cast<int>(ceil_div(rows, kKappaBlockTokens));
-    r = run_kappa(lp, lp_rollout, seg_offsets, n_tok, n_resp, blk0, nblk, kappa, nullptr, workspace, L, st, rec);
+    r = run_kappa(lp, lp_rollout, seg_offsets, n_tok, n_resp, blk0, nblk, opt, kappa, nullptr, workspace, L, st,
+                  rec);
     if (r != RZ_OK) return r;
     r = run_backward_chunk(H, W_head, token_ids, c0, rows, d, V, lp, lse, kappa, dH, dW, workspace, L, st, rec);
     if (r != RZ_OK) return r;
@@ -506,7 +600,19 @@ RZ_API rz_status rz_loss_fwd_bwd(const rz_bf16* H, const rz_bf16* W_head, const 
                                  int32_t d, int32_t V, float* loss, rz_bf16* dH, float* dW, float* lp_out,
                                  float* kappa_out, void* workspace, size_t ws_bytes, void* stream) {
   return loss_fwd_bwd_impl(H, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids, n_tok, n_resp,
-                           n_groups, d, V, loss, dH, dW, lp_out, kappa_out, workspace, ws_bytes, stream, nullptr);
+                           n_groups, d, V, nullptr, loss, dH, dW, lp_out, kappa_out, workspace, ws_bytes, stream,
+                           nullptr);
+}
+
+RZ_API rz_status rz_loss_fwd_bwd_ex(const rz_bf16* H, const rz_bf16* W_head, const int32_t* token_ids,
+                                    const float* lp_rollout, const float* rewards, const int64_t* seg_offsets,
+                                    const int32_t* group_ids, int64_t n_tok, int32_t n_resp, int32_t n_groups,
+                                    int32_t d, int32_t V, const rz_loss_options* options, float* loss, rz_bf16* dH,
+                                    float* dW, float* lp_out, float* kappa_out, void* workspace, size_t ws_bytes,
+                                    void* stream) {
+  return loss_fwd_bwd_impl(H, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids, n_tok, n_resp,
+                           n_groups, d, V, options, loss, dH, dW, lp_out, kappa_out, workspace, ws_bytes, stream,
+                           nullptr);
 }
 
 RZ_API int32_t rz_num_launches_loss(int64_t n_tok) {
@@ -524,8 +630,8 @@ RZ_API rz_status rz_loss_fwd_bwd_timed(const rz_bf16* H, const rz_bf16* W_head, 
   if (!launch_events || !launch_kinds || !n_launches || capacity < 0) return RZ_ERR_INVALID_ARG;
   Recorder rec{reinterpret_cast<cudaEvent_t*>(const_cast<void**>(launch_events)), launch_kinds, capacity, 0, false};
   const rz_status r = loss_fwd_bwd_impl(H, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids, n_tok,
-                                        n_resp, n_groups, d, V, loss, dH, dW, lp_out, kappa_out, workspace, ws_bytes,
-                                        stream, &rec);
+                                        n_resp, n_groups, d, V, nullptr, loss, dH, dW, lp_out, kappa_out, workspace,
+                                        ws_bytes, stream, &rec);
   *n_launches = rec.count;
   return r;
 }
@@ -585,6 +691,66 @@ RZ_API rz_status rz_token_logprobs_noalloc(const rz_bf16* H, const rz_bf16* W_he
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(at<int>(scratch, L.status), 0, 16, st) != cudaSuccess) return RZ_ERR_CUDA;
   return run_forward(H, W_head, token_ids, 0, n_tok, d, V, lp_out, lse_out, scratch, L, false, st, nullptr);
+}
+
+namespace {
+int stat_blocks(int64_t n) { return static_cast<int>(ceil_div(n, kStatTokens)); }
+// status | StatPartial [blocks] | histogram [2048] | selection state [4]
+size_t stats_parts_off() { return kAlign; }
+size_t stats_hist_off(int64_t n) { return align_up(stats_parts_off() + sizeof(StatPartial) * stat_blocks(n), kAlign); }
+size_t stats_sel_off(int64_t n) { return align_up(stats_hist_off(n) + sizeof(unsigned) * kStatBins, kAlign); }
+constexpr int kNormBlocks = 1184;  // 8 per SM on 148 SMs; fixed, so the partial order is fixed
+}  // namespace
+
+RZ_API size_t rz_workspace_bytes_ratio_stats(int64_t n_tok, int32_t n_resp) {
+  if (n_tok < 1 || n_tok >= (int64_t{1} << 31) || n_resp < 1) return 0;
+  return align_up(stats_sel_off(n_tok) + 16, kAlign);
+}
+
+RZ_API rz_status rz_ratio_stats(const float* lp, const float* lp_rollout, const int64_t* seg_offsets, int64_t n_tok,
+                                int32_t n_resp, const uint8_t* token_mask, double* stats_out,
+                                float* resp_mean_ratio_out, void* workspace, size_t ws_bytes, void* stream) {
+  if (n_tok < 1 || n_tok >= (int64_t{1} << 31) || n_resp < 1) return RZ_ERR_INVALID_ARG;
+  if (!lp || !lp_rollout || !seg_offsets || !stats_out || !workspace) return RZ_ERR_INVALID_ARG;
+  if (!aligned(lp, 4) || !aligned(lp_rollout, 4) || !aligned(seg_offsets, 8) || !aligned(stats_out, 8) ||
+      (resp_mean_ratio_out && !aligned(resp_mean_ratio_out, 4)) || !aligned(workspace, kAlign))
+    return RZ_ERR_INVALID_ARG;
+  if (ws_bytes < rz_workspace_bytes_ratio_stats(n_tok, n_resp)) return RZ_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  StatPartial* parts = at<StatPartial>(workspace, stats_parts_off());
+  unsigned* hist = at<unsigned>(workspace, stats_hist_off(n_tok));
+  unsigned* sel = at<unsigned>(workspace, stats_sel_off(n_tok));
+  if (cudaMemsetAsync(workspace, 0, 16, st) != cudaSuccess) return RZ_ERR_CUDA;
+  if (cudaMemsetAsync(hist, 0, sizeof(unsigned) * kStatBins, st) != cudaSuccess) return RZ_ERR_CUDA;
+  if (cudaMemsetAsync(sel, 0, 16, st) != cudaSuccess) return RZ_ERR_CUDA;
+  const int nb = stat_blocks(n_tok);
+  ratio_stats_pass0<<<nb, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, parts, hist);
+  ratio_stats_select<<<1, 32, 0, st>>>(hist, kStatBins, 11, sel, parts, nb, 0, stats_out);
+  ratio_stats_pass<<<nb, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, sel, 21, 10, 0x7ffu, hist);
+  ratio_stats_select<<<1, 32, 0, st>>>(hist, kStatBins, 11, sel, parts, nb, 0, stats_out);
+  ratio_stats_pass<<<nb, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, sel, 10, 0, 0x3ffu, hist);
+  ratio_stats_select<<<1, 32, 0, st>>>(hist, 1024, 10, sel, parts, nb, 1, stats_out);
+  if (resp_mean_ratio_out != nullptr)
+    response_mean_ratio_kernel<<<static_cast<unsigned>(ceil_div(n_resp, 8)), 256, 0, st>>>(
+        lp, lp_rollout, token_mask, seg_offsets, n_resp, resp_mean_ratio_out);
+  return cudaGetLastError() == cudaSuccess ? RZ_OK : RZ_ERR_CUDA;
+}
+
+RZ_API size_t rz_workspace_bytes_grad_norms(void) { return align_up(sizeof(double) * 2 * kNormBlocks, kAlign); }
+
+RZ_API rz_status rz_grad_norms(const rz_bf16* dH, const float* dW, int64_t n_tok, int32_t d, int32_t V,
+                               double* norms_out, void* workspace, size_t ws_bytes, void* stream) {
+  if (n_tok < 0 || d < 1 || V < 0 || !norms_out || !workspace) return RZ_ERR_INVALID_ARG;
+  if ((n_tok > 0 && !dH) || (V > 0 && !dW) || !aligned(norms_out, 8) || !aligned(workspace, kAlign))
+    return RZ_ERR_INVALID_ARG;
+  if (ws_bytes < rz_workspace_bytes_grad_norms()) return RZ_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  double* partials = static_cast<double*>(workspace);
+  sumsq_kernel<<<kNormBlocks, 256, 0, st>>>(dH, n_tok * d, 1, partials);
+  sumsq_kernel<<<kNormBlocks, 256, 0, st>>>(dW, static_cast<int64_t>(V) * d, 0, partials + kNormBlocks);
+  sqrt_sum_kernel<<<1, 32, 0, st>>>(partials, kNormBlocks, norms_out);
+  sqrt_sum_kernel<<<1, 32, 0, st>>>(partials + kNormBlocks, kNormBlocks, norms_out + 1);
+  return cudaGetLastError() == cudaSuccess ? RZ_OK : RZ_ERR_CUDA;
 }
 
 RZ_API rz_status rz_read_device_status(const void* workspace, void* stream, int32_t* bits_out) {

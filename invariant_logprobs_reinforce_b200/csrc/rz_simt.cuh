@@ -98,18 +98,63 @@ __global__ void __launch_bounds__(kCoefThreads)
 
 __global__ void __launch_bounds__(kCoefThreads)
     coef_kernel(const float* __restrict__ rewards, const int64_t* __restrict__ off, const int32_t* __restrict__ gid,
-                int R, int G, const double* __restrict__ gsum, const int* __restrict__ gcnt,
-                float* __restrict__ coef) {
+                int R, int G, double N, const int* __restrict__ counted, const double* __restrict__ gsum,
+                const int* __restrict__ gcnt, float* __restrict__ coef) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= R) return;
   const int g = gid[i];
-  const int64_t L = off[i + 1] - off[i];
-  if (g < 0 || g >= G || L <= 0 || gcnt[g] <= 0) {
+  const int64_t L = counted != nullptr ? counted[i] : off[i + 1] - off[i];
+  if (g < 0 || g >= G || off[i + 1] <= off[i] || gcnt[g] <= 0) {
     coef[i] = __int_as_float(0x7fc00000);
     return;
   }
+  if (L <= 0) {  // every token of the response is masked out: it contributes nothing
+    coef[i] = 0.0f;
+    return;
+  }
   const double A = static_cast<double>(rewards[i]) - gsum[g] / static_cast<double>(gcnt[g]);
-  coef[i] = static_cast<float>(-A / (static_cast<double>(R) * static_cast<double>(L)));
+  coef[i] = static_cast<float>(-A / (N * static_cast<double>(L)));
+}
+
+// Per response (one warp each): the number of tokens whose mask byte is non-zero.
+__global__ void __launch_bounds__(256)
+    masked_count_kernel(const uint8_t* __restrict__ mask, const int64_t* __restrict__ off, int R,
+                        int* __restrict__ counted) {
+  const int i = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (i >= R) return;
+  int c = 0;
+  for (int64_t t = off[i] + lane; t < off[i + 1]; t += 32) c += mask[t] != 0;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  if (lane == 0) counted[i] = c;
+}
+
+// Sequence gate (one warp per response): the response's geometric-mean ratio
+// exp(mean over its counted tokens of (lp - lp_rollout)); outside [lo, hi] the response's
+// coefficient becomes 0.  Lane-strided fp64 partials and a fixed butterfly: deterministic.
+__global__ void __launch_bounds__(256)
+    gate_kernel(const float* __restrict__ lp, const float* __restrict__ lp_roll, const uint8_t* __restrict__ mask,
+                const int64_t* __restrict__ off, int R, double lo, double hi, float* __restrict__ coef) {
+  const int i = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (i >= R) return;
+  double sum = 0.0;
+  int c = 0;
+  for (int64_t t = off[i] + lane; t < off[i + 1]; t += 32) {
+    if (mask != nullptr && mask[t] == 0) continue;
+    sum += static_cast<double>(lp[t]) - static_cast<double>(lp_roll[t]);
+    ++c;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    c += __shfl_xor_sync(0xffffffffu, c, o);
+  }
+  if (lane == 0 && c > 0) {
+    const double g = exp(sum / c);
+    if (!(g >= lo && g <= hi)) coef[i] = 0.0f;
+  }
 }
 
 constexpr int kKappaThreads = 256;
@@ -150,7 +195,8 @@ __global__ void __launch_bounds__(kKappaThreads)
     token_kappa_kernel(const float* __restrict__ lp, const float* __restrict__ lp_roll,
                        const int64_t* __restrict__ off, int R, const float* __restrict__ coef,
                        const int* __restrict__ block_first, int64_t n, int block0, int vec_ok,
-                       float* __restrict__ kappa, float* __restrict__ w_out, double* __restrict__ block_sums) {
+                       const uint8_t* __restrict__ mask, float clip_max, float* __restrict__ kappa,
+                       float* __restrict__ w_out, double* __restrict__ block_sums) {
   constexpr int kFar = 1 << 30;  // a relative start beyond the block
   __shared__ int s_rel[kKappaStagedOffsets + 1];  // start of staged response k, relative to the block
   __shared__ float s_coef[kKappaStagedOffsets];
@@ -192,13 +238,15 @@ __global__ void __launch_bounds__(kKappaThreads)
       while (s_rel[k + 1] <= tr) ++k;
       const float a4[4] = {la[it].x, la[it].y, la[it].z, la[it].w};
       const float b4[4] = {lb[it].x, lb[it].y, lb[it].z, lb[it].w};
+      uint32_t m4 = 0x01010101u;
+      if (mask != nullptr) m4 = *reinterpret_cast<const uint32_t*>(mask + b0 + tr);
       float w[4], kv[4];
       float part = 0.0f;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         if (j > 0 && s_rel[k + 1] <= tr + j) ++k;
         w[j] = ex2_approx((a4[j] - b4[j]) * kLog2e);
-        kv[j] = s_coef[k] * w[j];
+        kv[j] = ((m4 >> (8 * j)) & 0xffu) ? s_coef[k] * fminf(w[j], clip_max) : 0.0f;
         part += kv[j];
       }
       const int64_t t0 = b0 + tr;
@@ -217,7 +265,7 @@ __global__ void __launch_bounds__(kKappaThreads)
           const int64_t t = t0 + j;
           while (i + 1 < R && __ldg(off + i + 1) <= t) ++i;
           const float w = ex2_approx((lp[t] - lp_roll[t]) * kLog2e);
-          const float kv = __ldg(coef + i) * w;
+          const float kv = (mask == nullptr || mask[t] != 0) ? __ldg(coef + i) * fminf(w, clip_max) : 0.0f;
           kappa[t] = kv;
           if (w_out != nullptr) w_out[t] = w;
           part += kv;
@@ -253,6 +301,206 @@ __global__ void loss_final_kernel(const double* __restrict__ block_sums, int nb,
 }
 
 // ------------------------------------------------------------------------ backward
+
+// ------------------------------------------------------------------------ diagnostics
+//
+// Ratio statistics over the counted tokens: sums for the KL estimators k1 = lp_rollout - lp,
+// k2 = (lp - lp_rollout)^2 / 2 and k3 = w - 1 - (lp - lp_rollout) (fp64 from the fp32
+// inputs, fixed-order per-block partials), min / max of w, max of the deviation |w - 1|
+// (w as the loss stage computes it, fp32), and the deviation's exact lower
+// median by a three-pass radix select on the deviation's float bits (non-negative floats
+// order like their bit patterns; counts are integers, so the result does not depend on
+// the order of the atomic adds).
+constexpr int kStatThreads = 256;
+constexpr int kStatTokens = 4096;  // tokens per block
+constexpr int kStatBins = 2048;    // 11 bits per radix pass
+
+struct StatPartial {
+  double k1, k2, k3;
+  float w_min, w_max, dev_max;
+  int count;
+};
+
+__device__ __forceinline__ float ratio_of(float a, float b) { return ex2_approx((a - b) * kLog2e); }
+
+__global__ void __launch_bounds__(kStatThreads)
+    ratio_stats_pass0(const float* __restrict__ lp, const float* __restrict__ lp_roll, const uint8_t* __restrict__ mask,
+                      int64_t n, StatPartial* __restrict__ parts, unsigned* __restrict__ hist) {
+  __shared__ unsigned s_hist[kStatBins];
+  __shared__ StatPartial s_part[kStatThreads / 32];
+  for (int b = threadIdx.x; b < kStatBins; b += kStatThreads) s_hist[b] = 0u;
+  __syncthreads();
+  const int64_t b0 = static_cast<int64_t>(blockIdx.x) * kStatTokens;
+  double k1 = 0.0, k2 = 0.0, k3 = 0.0;
+  float wmin = INFINITY, wmax = -INFINITY, dmax = 0.0f;
+  int cnt = 0;
+  for (int j = threadIdx.x; j < kStatTokens; j += kStatThreads) {
+    const int64_t t = b0 + j;
+    if (t >= n) break;
+    if (mask != nullptr && mask[t] == 0) continue;
+    // the KL estimators in fp64 (k3 cancels to second order); min / max / deviation on
+    // the ratio exactly as the loss stage computes it
+    const double x = static_cast<double>(lp[t]) - static_cast<double>(lp_roll[t]);
+    const float w = ratio_of(lp[t], lp_roll[t]);
+    const float dev = fabsf(w - 1.0f);
+    k1 -= x;
+    k2 += 0.5 * x * x;
+    k3 += expm1(x) - x;
+    wmin = fminf(wmin, w);
+    wmax = fmaxf(wmax, w);
+    dmax = fmaxf(dmax, dev);
+    ++cnt;
+    atomicAdd(&s_hist[__float_as_uint(dev) >> 21], 1u);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    k1 += __shfl_xor_sync(0xffffffffu, k1, o);
+    k2 += __shfl_xor_sync(0xffffffffu, k2, o);
+    k3 += __shfl_xor_sync(0xffffffffu, k3, o);
+    wmin = fminf(wmin, __shfl_xor_sync(0xffffffffu, wmin, o));
+    wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, o));
+    dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, o));
+    cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  }
+  if ((threadIdx.x & 31) == 0) s_part[threadIdx.x >> 5] = StatPartial{k1, k2, k3, wmin, wmax, dmax, cnt};
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    StatPartial acc = s_part[0];
+    for (int w = 1; w < kStatThreads / 32; ++w) {
+      acc.k1 += s_part[w].k1;
+      acc.k2 += s_part[w].k2;
+      acc.k3 += s_part[w].k3;
+      acc.w_min = fminf(acc.w_min, s_part[w].w_min);
+      acc.w_max = fmaxf(acc.w_max, s_part[w].w_max);
+      acc.dev_max = fmaxf(acc.dev_max, s_part[w].dev_max);
+      acc.count += s_part[w].count;
+    }
+    parts[blockIdx.x] = acc;
+  }
+  for (int b = threadIdx.x; b < kStatBins; b += kStatThreads)
+    if (s_hist[b]) atomicAdd(&hist[b], s_hist[b]);
+}
+
+// Histogram of the next radix digit among the deviations whose higher bits equal `prefix`.
+__global__ void __launch_bounds__(kStatThreads)
+    ratio_stats_pass(const float* __restrict__ lp, const float* __restrict__ lp_roll, const uint8_t* __restrict__ mask,
+                     int64_t n, const unsigned* __restrict__ sel, int shift_hi, int shift, unsigned digit_mask,
+                     unsigned* __restrict__ hist) {
+  __shared__ unsigned s_hist[kStatBins];
+  for (int b = threadIdx.x; b < kStatBins; b += kStatThreads) s_hist[b] = 0u;
+  __syncthreads();
+  const unsigned prefix = sel[0];
+  const int64_t b0 = static_cast<int64_t>(blockIdx.x) * kStatTokens;
+  for (int j = threadIdx.x; j < kStatTokens; j += kStatThreads) {
+    const int64_t t = b0 + j;
+    if (t >= n) break;
+    if (mask != nullptr && mask[t] == 0) continue;
+    const unsigned key = __float_as_uint(fabsf(ratio_of(lp[t], lp_roll[t]) - 1.0f));
+    if ((key >> shift_hi) == prefix) atomicAdd(&s_hist[(key >> shift) & digit_mask], 1u);
+  }
+  __syncthreads();
+  for (int b = threadIdx.x; b < kStatBins; b += kStatThreads)
+    if (s_hist[b]) atomicAdd(&hist[b], s_hist[b]);
+}
+
+// One thread: find the digit holding rank sel[1] in hist, extend the prefix, keep the rank
+// within that digit, clear hist for the next pass.  On the last pass, write the statistics.
+__global__ void ratio_stats_select(unsigned* __restrict__ hist, int nbins, int digit_bits, unsigned* __restrict__ sel,
+                                   const StatPartial* __restrict__ parts, int nparts, int last,
+                                   double* __restrict__ stats) {
+  if (threadIdx.x != 0) return;
+  if (sel[2] == 0u) {  // first pass: total count and the target rank from the partials
+    long long m = 0;
+    for (int b = 0; b < nparts; ++b) m += parts[b].count;
+    sel[1] = m > 0 ? static_cast<unsigned>((m - 1) / 2) : 0u;
+    sel[2] = 1u;
+    sel[0] = 0u;
+  }
+  unsigned rank = sel[1];
+  int digit = 0;
+  for (; digit < nbins - 1; ++digit) {
+    if (rank < hist[digit]) break;
+    rank -= hist[digit];
+  }
+  for (int b = 0; b < nbins; ++b) hist[b] = 0u;
+  sel[0] = (sel[0] << digit_bits) | static_cast<unsigned>(digit);
+  sel[1] = rank;
+  if (!last) return;
+  StatPartial acc = parts[0];
+  for (int b = 1; b < nparts; ++b) {
+    acc.k1 += parts[b].k1;
+    acc.k2 += parts[b].k2;
+    acc.k3 += parts[b].k3;
+    acc.w_min = fminf(acc.w_min, parts[b].w_min);
+    acc.w_max = fmaxf(acc.w_max, parts[b].w_max);
+    acc.dev_max = fmaxf(acc.dev_max, parts[b].dev_max);
+    acc.count += parts[b].count;
+  }
+  const double m = acc.count > 0 ? static_cast<double>(acc.count) : 1.0;
+  const double med = static_cast<double>(__uint_as_float(sel[0]));
+  stats[0] = acc.k1 / m;
+  stats[1] = acc.k2 / m;
+  stats[2] = acc.k3 / m;
+  stats[3] = acc.w_min;
+  stats[4] = acc.w_max;
+  stats[5] = acc.dev_max;
+  stats[6] = med;
+  stats[7] = med > 0.0 ? acc.dev_max / med : INFINITY;
+  stats[8] = acc.count;
+}
+
+// Per response (one warp each): the mean ratio over its counted tokens (0 if none).
+__global__ void __launch_bounds__(256)
+    response_mean_ratio_kernel(const float* __restrict__ lp, const float* __restrict__ lp_roll,
+                               const uint8_t* __restrict__ mask, const int64_t* __restrict__ off, int R,
+                               float* __restrict__ out) {
+  const int i = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (i >= R) return;
+  double sum = 0.0;
+  int c = 0;
+  for (int64_t t = off[i] + lane; t < off[i + 1]; t += 32) {
+    if (mask != nullptr && mask[t] == 0) continue;
+    sum += ratio_of(lp[t], lp_roll[t]);
+    ++c;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    c += __shfl_xor_sync(0xffffffffu, c, o);
+  }
+  if (lane == 0) out[i] = c > 0 ? static_cast<float>(sum / c) : 0.0f;
+}
+
+// Sum of squares of a bf16 (is_bf16) or fp32 array, per-block fp64 partials in a fixed
+// order (grid-stride, 8 elements per thread per step), then one block sums the partials.
+__global__ void __launch_bounds__(256)
+    sumsq_kernel(const void* __restrict__ x, int64_t count, int is_bf16, double* __restrict__ partials) {
+  __shared__ double s_w[8];
+  double acc = 0.0;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < count; i += stride) {
+    const float v = is_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(x)[i])
+                            : reinterpret_cast<const float*>(x)[i];
+    acc += static_cast<double>(v) * v;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) s_w[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double s = 0.0;
+    for (int w = 0; w < 8; ++w) s += s_w[w];
+    partials[blockIdx.x] = s;
+  }
+}
+
+__global__ void sqrt_sum_kernel(const double* __restrict__ partials, int np, double* __restrict__ out) {
+  if (threadIdx.x != 0) return;
+  double s = 0.0;
+  for (int b = 0; b < np; ++b) s += partials[b];
+  *out = sqrt(s);
+}
 
 // dZ[t, v] = kappa_t ([v == y_t] - p_tv) in bf16, in place over the stored fp16
 // e_tv = exp(z_tv - tile_max_t,tile) of the forward: p_tv = e_tv exp(tile_max - lse_t).
