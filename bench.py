@@ -43,6 +43,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-loss-stage", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="tokens-per-call sweep 2^12..2^20 of the workload (forward and forward+backward)")
     ap.add_argument("--n-tok-cap", type=int, default=None,
                     help="keep only the leading whole groups that fit (small profiling cases)")
     return ap.parse_args()
@@ -281,6 +283,20 @@ def run_rz(args, rank, world, local_rank):
     torch.cuda.synchronize()
     fwd_ms = f0.elapsed_time(f1) / fsteps
 
+    # forward from e4m3 operands (quantised once, outside the timed region)
+    H8, hs8 = rz.rz_quantize_rows_e4m3(H)
+    W8, ws8 = rz.rz_quantize_rows_e4m3(W)
+    lp8 = torch.empty(n, dtype=torch.float32, device=dev)
+    for _ in range(2):
+        rz.rz_token_logprobs_fp8(H8, hs8, W8, ws8, ids, lp_out=lp8, workspace=wsf, stream=stream, want_lse=False)
+    f0.record(stream)
+    for _ in range(fsteps):
+        rz.rz_token_logprobs_fp8(H8, hs8, W8, ws8, ids, lp_out=lp8, workspace=wsf, stream=stream, want_lse=False)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    fwd8_ms = f0.elapsed_time(f1) / fsteps
+    del H8, W8
+
     loss_stage = None
     if not args.no_loss_stage:
         loss_stage = run_loss_stage(rz, torch, dev, stream)
@@ -312,7 +328,7 @@ def run_rz(args, rank, world, local_rank):
         dominant=dom, achieved=ach, peak=peak_tflops, peak_src=peak_src,
         traffic=traffic_for(dom, tens[dom]["rows"] / tens[dom]["launches"]),
         fwd_ms=fwd_ms, fwd_tok_s=world * n / (fwd_ms * 1e-3), launches=launches_total, e2e=e2e, cfg=cfg,
-        loss_stage=loss_stage,
+        loss_stage=loss_stage, fwd8_ms=fwd8_ms,
     )
 
 
@@ -361,10 +377,38 @@ def run_loss_stage(rz, torch, dev, stream, n_tok=1 << 26, reps=20):
     nbytes = 12 * n_tok + 16 * R
     peaks, src = load_peaks()
     gbs = nbytes / (ms * 1e-3) / 1e9
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    # the truncated-IS + token-mask variant (adds a 1-byte mask read per token)
+    mask = (torch.rand(n_tok, generator=g, device=dev) < 0.9).to(torch.uint8)
+    opts = rz.loss_options(clip_max=1.05, token_mask=mask)
+    ms_var = timed(lambda: rz.rz_segment_loss_ex(lp, lr, t_r, t_off, t_gid, G, opts, workspace=ws, stream=stream))
+    var_bytes = 13 * n_tok + 16 * R
+    # ratio diagnostics: three passes over lp and lp_rollout (radix select), 8 B/token each
+    ws_st = torch.empty(int(rz.lib().rz_workspace_bytes_ratio_stats(n_tok, R)), dtype=torch.uint8, device=dev)
+    ms_st = timed(lambda: rz.rz_ratio_stats(lp, lr, t_off, want_resp_mean=False, workspace=ws_st, stream=stream))
+    st_bytes = 3 * 8 * n_tok
+    hbm = peaks["hbm_gbs"]
     return {"n_tok": n_tok, "n_resp": R, "n_groups": G, "ms_per_call": ms, "algorithmic_bytes": nbytes,
-            "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+            "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
             "bound": "hbm", "peak_source": f"hbm_gbs of {src}",
-            "note": "whole rz_segment_loss call (3 launches); inputs 768 MB > L2"}
+            "note": "whole rz_segment_loss call (coefficients, block starts, kappa, loss); inputs 768 MB > L2",
+            "variant_clip_mask": {"ms_per_call": ms_var, "achieved": var_bytes / (ms_var * 1e-3) / 1e9,
+                                  "frac": var_bytes / (ms_var * 1e-3) / 1e9 / hbm},
+            "ratio_stats": {"ms_per_call": ms_st, "achieved": st_bytes / (ms_st * 1e-3) / 1e9,
+                            "frac": st_bytes / (ms_st * 1e-3) / 1e9 / hbm,
+                            "note": "3 radix-select passes, 8 B/token each"}}
 
 
 def run_e2e(rz, torch, dev, stream, H, W, ids, lp_roll, rewards, off, gid, G, n, d, V, args):
@@ -407,6 +451,78 @@ def run_e2e(rz, torch, dev, stream, H, W, ids, lp_roll, rewards, off, gid, G, n,
     d2h = loss_h.numel() * 4 + lp_h.numel() * 4
     return {"value": n / (ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "ms_per_step": ms}
+
+
+# --------------------------------------------------------------------------- sweep
+
+def run_sweep(args, local_rank):
+    """Tokens per call 2^12 .. 2^20 over one generated batch of the workload: forward alone
+    and forward + loss + backward, tokens/s and fraction of the sustained bf16 peak."""
+    import torch
+    import workloads as wl
+    import invariant_logprobs_reinforce_b200 as rz
+    from invariant_logprobs_reinforce_b200 import build as rzbuild
+    rzbuild.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream()
+    prob = wl.full_config(args.workload, device=str(dev), n_tok_cap=args.n_tok_cap or (1 << 20))
+    seg = prob.seg
+    d, V = prob.d, prob.V
+    peaks, src = load_peaks()
+    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    lp_all, _ = rz.rz_token_logprobs(prob.H, prob.W, prob.ids)
+    torch.cuda.synchronize()
+    lr_all = torch.from_numpy(wl.rollout_logprobs_with_lag(lp_all.cpu().numpy(), prob.noise, prob.seed)).to(dev)
+    points = []
+    for e in range(12, 21):
+        n = 1 << e
+        if n > prob.n_tok:
+            break
+        # whole responses up to n tokens (the last one truncated), one group per 16 responses
+        R = int(np.searchsorted(seg.seg_offsets, n, side="left"))
+        off = seg.seg_offsets[:R + 1].copy()
+        off[-1] = n
+        if off[-2] == n:
+            off = off[:-1]
+            R -= 1
+        gid = (np.arange(R) // 16).astype(np.int32)
+        G = int(gid[-1]) + 1
+        H, ids = prob.H[:n], prob.ids[:n]
+        t_off = torch.from_numpy(off).to(dev)
+        t_gid = torch.from_numpy(gid).to(dev)
+        t_r = torch.from_numpy(seg.rewards[:R].copy()).to(dev)
+        ws = torch.empty(rz.rz_workspace_bytes_loss(n, R, G, d, V), dtype=torch.uint8, device=dev)
+        wsf = torch.empty(rz.rz_workspace_bytes_logprobs(n, d, V), dtype=torch.uint8, device=dev)
+        lp = torch.empty(n, dtype=torch.float32, device=dev)
+        out = dict(loss=torch.empty(1, device=dev), dH=torch.empty((n, d), dtype=torch.bfloat16, device=dev),
+                   dW=torch.empty((V, d), dtype=torch.float32, device=dev))
+
+        def fwd():
+            rz.rz_token_logprobs(H, prob.W, ids, lp_out=lp, workspace=wsf, stream=stream, want_lse=False)
+
+        def step():
+            rz.rz_loss_fwd_bwd(H, prob.W, ids, lr_all[:n], t_r, t_off, t_gid, G, loss=out["loss"], dH=out["dH"],
+                               dW=out["dW"], want_lp=False, want_kappa=False, workspace=ws, stream=stream)
+
+        res = {"n_tok": n, "n_resp": R}
+        for name, fn, flops in (("fwd", fwd, 2.0), ("fwd_bwd", step, 6.0)):
+            reps = max(2, min(20, int(2e15 / (flops * n * d * V)) + 1))
+            for _ in range(2):
+                fn()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(reps):
+                fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ms = a.elapsed_time(b) / reps
+            res[name] = {"ms": ms, "tokens_per_s": n / (ms * 1e-3),
+                         "tensor_frac": n * flops * d * V / (ms * 1e-3) / (peak * 1e12)}
+        points.append(res)
+        del ws, wsf, out
+    return {"workload": args.workload, "d": d, "V": V, "peak_tflops": peak, "peak_source": src, "points": points}
 
 
 # --------------------------------------------------------------------------- CPU oracle
@@ -480,6 +596,11 @@ def main():
             print(json.dumps(line), flush=True)
         return 0
 
+    if args.sweep:
+        if rank == 0:
+            print(json.dumps({"sweep": run_sweep(args, local_rank)}), flush=True)
+        return 0
+
     if world > 1:
         import datetime
         import torch
@@ -513,6 +634,11 @@ def main():
             "tensor_frac_6dV": res["value"] / world * 6 * res["d"] * res["V"] / (res["peak"] * 1e12),
             "fwd_only": {"tokens_per_s": res["fwd_tok_s"], "ms_per_step": res["fwd_ms"],
                          "tensor_frac_2dV": res["fwd_tok_s"] / world * 2 * res["d"] * res["V"] / (res["peak"] * 1e12)},
+            "fwd_only_fp8": {"tokens_per_s": res["n_tok"] * world / (res["fwd8_ms"] * 1e-3),
+                             "ms_per_step": res["fwd8_ms"],
+                             "tensor_frac_2dV": res["n_tok"] * 2 * res["d"] * res["V"] / (res["fwd8_ms"] * 1e-3)
+                             / (2 * res["peak"] * 1e12),
+                             "peak_note": "e4m3 peak = 2 x the measured sustained bf16 peak (nominal ratio)"},
             "kernels": res["kernels"],
             "loss_stage": res["loss_stage"],
             "gpu_launches": res["launches"],

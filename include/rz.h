@@ -216,6 +216,26 @@ size_t rz_workspace_bytes_grad_norms(void);
 rz_status rz_grad_norms(const rz_bf16* dH, const float* dW, int64_t n_tok, int32_t d, int32_t V, double* norms_out,
                         void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * Low-precision forward: token logprobs from e4m3 (fp8) operands with per-row scales, the
+ * pages' "low-precision compute" of the rollout side ("vLLM Train-Inference Consistency
+ * Release Notes", section "The Technical Challenge"; "vLLM says aligned kernels…", section
+ * "Zero mismatch expands to newer models": FP8 weights), under the same batch-invariance
+ * contract as rz_token_logprobs.
+ *
+ *   rz_quantize_rows_e4m3: X [rows, d] bf16 -> X8 [rows, d] e4m3 bytes and scale [rows] fp32,
+ *     scale = max|x| / 448 (1 for an all-zero row), X8 = e4m3(x / scale), round to nearest
+ *     even, saturating (both divisions IEEE fp32).
+ *   rz_token_logprobs_fp8: z[t,v] = (sum_k H8[t,k] W8[v,k]) * h_scale[t] * w_scale[v]
+ *     (e4m3 x e4m3 products accumulated in fp32 on the tensor cores, then the two scales
+ *     applied in that order); lp, lse as rz_token_logprobs.  d must be a multiple of 128;
+ *     workspace size = rz_workspace_bytes_logprobs(n_tok, d, V).
+ */
+rz_status rz_quantize_rows_e4m3(const rz_bf16* X, int64_t rows, int32_t d, uint8_t* X8, float* scale, void* stream);
+rz_status rz_token_logprobs_fp8(const uint8_t* H8, const float* h_scale, const uint8_t* W8, const float* w_scale,
+                                const int32_t* token_ids, int64_t n_tok, int32_t d, int32_t V, float* lp_out,
+                                float* lse_out, void* workspace, size_t ws_bytes, void* stream);
+
 /* Kernel kinds reported per launch by rz_loss_fwd_bwd_timed. */
 #define RZ_KERNEL_LMHEAD_LSE 0    /* fused LM head + online log-sum-exp + gather (tensor cores) */
 #define RZ_KERNEL_MERGE_LSE 1     /* fixed-order merge of the vocabulary-segment partials       */

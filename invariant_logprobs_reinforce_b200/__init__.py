@@ -28,6 +28,7 @@ EXPORTED_SYMBOLS = (
     "rz_token_logprobs", "rz_loss_fwd_bwd", "rz_segment_loss", "rz_read_device_status", "rz_num_launches_loss",
     "rz_loss_fwd_bwd_timed", "rz_token_logprobs_noalloc", "rz_loss_fwd_bwd_ex", "rz_segment_loss_ex",
     "rz_workspace_bytes_ratio_stats", "rz_ratio_stats", "rz_workspace_bytes_grad_norms", "rz_grad_norms",
+    "rz_quantize_rows_e4m3", "rz_token_logprobs_fp8",
 )
 RZ_LOSS_CLIP_IS, RZ_LOSS_SEQ_GATE, RZ_LOSS_TOKEN_MASK = 1, 2, 4
 STAT_NAMES = ("k1", "k2", "k3", "w_min", "w_max", "dev_max", "dev_median", "dev_peak_over_median", "count")
@@ -109,6 +110,10 @@ def lib() -> ctypes.CDLL:
         L.rz_workspace_bytes_grad_norms.restype = sz
         L.rz_grad_norms.argtypes = [P, P, i64, i32, i32, P, P, sz, P]
         L.rz_grad_norms.restype = ctypes.c_int
+        L.rz_quantize_rows_e4m3.argtypes = [P, i64, i32, P, P, P]
+        L.rz_quantize_rows_e4m3.restype = ctypes.c_int
+        L.rz_token_logprobs_fp8.argtypes = [P, P, P, P, P, i64, i32, i32, P, P, P, sz, P]
+        L.rz_token_logprobs_fp8.restype = ctypes.c_int
         L.rz_read_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
         L.rz_read_device_status.restype = ctypes.c_int
         _lib = L
@@ -367,3 +372,32 @@ def rz_grad_norms(dH, dW, workspace=None, stream=None):
     code = lib().rz_grad_norms(_ptr(dH), _ptr(dW), n, d, V, _ptr(out), _ptr(ws), ws.numel(), _stream_handle(stream))
     _check(code, "rz_grad_norms")
     return out
+
+
+def rz_quantize_rows_e4m3(X, stream=None):
+    """bf16 [rows, d] -> (e4m3 codes as uint8 [rows, d], fp32 per-row scales [rows])."""
+    torch = _torch()
+    _need(X, torch.bfloat16, "X")
+    rows, d = X.shape
+    q = torch.empty((rows, d), dtype=torch.uint8, device=X.device)
+    sc = torch.empty(rows, dtype=torch.float32, device=X.device)
+    _check(lib().rz_quantize_rows_e4m3(_ptr(X), rows, d, _ptr(q), _ptr(sc), _stream_handle(stream)),
+           "rz_quantize_rows_e4m3")
+    return q, sc
+
+
+def rz_token_logprobs_fp8(H8, h_scale, W8, w_scale, token_ids, lp_out=None, lse_out=None, workspace=None,
+                          stream=None, want_lse=True):
+    """Token logprobs from e4m3 operands with per-row scales.  Returns (lp, lse)."""
+    torch = _torch()
+    _need(H8, torch.uint8, "H8")
+    dev = H8.device
+    n, d = H8.shape
+    V = W8.shape[0]
+    lp = lp_out if lp_out is not None else torch.empty(n, dtype=torch.float32, device=dev)
+    lse = lse_out if lse_out is not None else (torch.empty(n, dtype=torch.float32, device=dev) if want_lse else None)
+    ws = _workspace(rz_workspace_bytes_logprobs(n, d, V), workspace, dev)
+    code = lib().rz_token_logprobs_fp8(_ptr(H8), _ptr(h_scale), _ptr(W8), _ptr(w_scale), _ptr(token_ids), n, d, V,
+                                       _ptr(lp), _ptr(lse), _ptr(ws), ws.numel(), _stream_handle(stream))
+    _check(code, "rz_token_logprobs_fp8")
+    return lp, lse

@@ -241,6 +241,8 @@ rz_status run_forward(const rz_bf16* H, const rz_bf16* W, const int32_t* ids, in
     e.part_ld = L.part_ld;
     e.zy = zy;
     e.tile_max = at<float>(ws, L.tile_max);
+    e.row_scale = nullptr;
+    e.col_scale = nullptr;
     if (launch_gemm<false, false>(mH, mW, s, pos, e, status, stream) != cudaSuccess) return RZ_ERR_CUDA;
   } else {
     EpiLse<false> e;
@@ -254,6 +256,8 @@ rz_status run_forward(const rz_bf16* H, const rz_bf16* W, const int32_t* ids, in
     e.part_ld = L.part_ld;
     e.zy = zy;
     e.tile_max = nullptr;
+    e.row_scale = nullptr;
+    e.col_scale = nullptr;
     if (launch_gemm<false, false>(mH, mW, s, pos, e, status, stream) != cudaSuccess) return RZ_ERR_CUDA;
   }
   rec_end(rec, stream);
@@ -264,6 +268,48 @@ rz_status run_forward(const rz_bf16* H, const rz_bf16* W, const int32_t* ids, in
   if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
   rec_end(rec, stream);
   return RZ_OK;
+}
+
+// Forward with scaled e4m3 operands (kind::f8f6f4, 128-element K blocks): the same
+// epilogue and merge as run_forward, with the logits rescaled per row and column.
+rz_status run_forward_fp8(const uint8_t* H8, const float* hs, const uint8_t* W8, const float* wsc,
+                          const int32_t* ids, int64_t n, int32_t d, int32_t V, float* lp, float* lse, void* ws,
+                          const Layout& L, cudaStream_t stream) {
+  int* status = at<int>(ws, L.status);
+  CUtensorMap mH, mW;
+  if (!make_map(&mH, CU_TENSOR_MAP_DATA_TYPE_UINT8, H8, d, n, static_cast<uint64_t>(d), BK_FP8, BM,
+                CU_TENSOR_MAP_SWIZZLE_128B))
+    return RZ_ERR_CUDA;
+  if (!make_map(&mW, CU_TENSOR_MAP_DATA_TYPE_UINT8, W8, d, V, static_cast<uint64_t>(d), BK_FP8, BN,
+                CU_TENSOR_MAP_SWIZZLE_128B))
+    return RZ_ERR_CUDA;
+  GemmSched s = make_sched(n, V, kSegTiles, 32, d);
+  s.num_kb = static_cast<int>(ceil_div(d, BK_FP8));
+  const OperandPos pos{0, 0, 0, 0};
+  EpiLse<false> e;
+  std::memset(&e.p_map, 0, sizeof(e.p_map));
+  e.ids = ids;
+  e.rows = n;
+  e.V = V;
+  e.n_tiles = num_vocab_tiles(V);
+  e.part_m = at<float>(ws, L.part_m);
+  e.part_s = at<float>(ws, L.part_s);
+  e.part_ld = L.part_ld;
+  e.zy = at<float>(ws, L.zy);
+  e.tile_max = nullptr;
+  e.row_scale = hs;
+  e.col_scale = wsc;
+  auto kernel = gemm_tc_kernel<false, false, EpiLse<false>, true>;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) != cudaSuccess)
+    return RZ_ERR_CUDA;
+  const int sms = sm_count();
+  if (sms <= 0) return RZ_ERR_CUDA;
+  kernel<<<std::max(1, std::min(s.num_units, sms)), kGemmThreads, kGemmSmemBytes, stream>>>(mH, mW, s, pos, e,
+                                                                                          status);
+  if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
+  merge_lse_kernel<<<static_cast<unsigned>(ceil_div(n, 256)), 256, 0, stream>>>(
+      e.part_m, e.part_s, L.part_ld, e.zy, ids, n, V, num_segments(V), lp, lse, status);
+  return cudaGetLastError() == cudaSuccess ? RZ_OK : RZ_ERR_CUDA;
 }
 
 // Loss-stage options after defaults: no cap (+inf), no gate, no mask, N = n_resp.
@@ -695,16 +741,17 @@ RZ_API rz_status rz_token_logprobs_noalloc(const rz_bf16* H, const rz_bf16* W_he
 
 namespace {
 int stat_blocks(int64_t n) { return static_cast<int>(ceil_div(n, kStatTokens)); }
-// status | StatPartial [blocks] | histogram [2048] | selection state [4]
+// status | StatPartial [blocks] | histogram [2048] | selection state [4] | reduced partial
 size_t stats_parts_off() { return kAlign; }
 size_t stats_hist_off(int64_t n) { return align_up(stats_parts_off() + sizeof(StatPartial) * stat_blocks(n), kAlign); }
 size_t stats_sel_off(int64_t n) { return align_up(stats_hist_off(n) + sizeof(unsigned) * kStatBins, kAlign); }
+size_t stats_acc_off(int64_t n) { return align_up(stats_sel_off(n) + 16, kAlign); }
 constexpr int kNormBlocks = 1184;  // 8 per SM on 148 SMs; fixed, so the partial order is fixed
 }  // namespace
 
 RZ_API size_t rz_workspace_bytes_ratio_stats(int64_t n_tok, int32_t n_resp) {
   if (n_tok < 1 || n_tok >= (int64_t{1} << 31) || n_resp < 1) return 0;
-  return align_up(stats_sel_off(n_tok) + 16, kAlign);
+  return align_up(stats_acc_off(n_tok) + sizeof(StatPartial), kAlign);
 }
 
 RZ_API rz_status rz_ratio_stats(const float* lp, const float* lp_rollout, const int64_t* seg_offsets, int64_t n_tok,
@@ -724,12 +771,14 @@ RZ_API rz_status rz_ratio_stats(const float* lp, const float* lp_rollout, const 
   if (cudaMemsetAsync(hist, 0, sizeof(unsigned) * kStatBins, st) != cudaSuccess) return RZ_ERR_CUDA;
   if (cudaMemsetAsync(sel, 0, 16, st) != cudaSuccess) return RZ_ERR_CUDA;
   const int nb = stat_blocks(n_tok);
+  StatPartial* acc = at<StatPartial>(workspace, stats_acc_off(n_tok));
   ratio_stats_pass0<<<nb, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, parts, hist);
-  ratio_stats_select<<<1, 32, 0, st>>>(hist, kStatBins, 11, sel, parts, nb, 0, stats_out);
+  ratio_stats_reduce<<<1, 1024, 0, st>>>(parts, nb, acc, sel);
+  ratio_stats_select<<<1, 1024, 0, st>>>(hist, kStatBins, 11, sel, acc, 0, stats_out);
   ratio_stats_pass<<<nb, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, sel, 21, 10, 0x7ffu, hist);
-  ratio_stats_select<<<1, 32, 0, st>>>(hist, kStatBins, 11, sel, parts, nb, 0, stats_out);
+  ratio_stats_select<<<1, 1024, 0, st>>>(hist, kStatBins, 11, sel, acc, 0, stats_out);
   ratio_stats_pass<<<nb, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, sel, 10, 0, 0x3ffu, hist);
-  ratio_stats_select<<<1, 32, 0, st>>>(hist, 1024, 10, sel, parts, nb, 1, stats_out);
+  ratio_stats_select<<<1, 1024, 0, st>>>(hist, 1024, 10, sel, acc, 1, stats_out);
   if (resp_mean_ratio_out != nullptr)
     response_mean_ratio_kernel<<<static_cast<unsigned>(ceil_div(n_resp, 8)), 256, 0, st>>>(
         lp, lp_rollout, token_mask, seg_offsets, n_resp, resp_mean_ratio_out);
@@ -751,6 +800,35 @@ RZ_API rz_status rz_grad_norms(const rz_bf16* dH, const float* dW, int64_t n_tok
   sqrt_sum_kernel<<<1, 32, 0, st>>>(partials, kNormBlocks, norms_out);
   sqrt_sum_kernel<<<1, 32, 0, st>>>(partials + kNormBlocks, kNormBlocks, norms_out + 1);
   return cudaGetLastError() == cudaSuccess ? RZ_OK : RZ_ERR_CUDA;
+}
+
+RZ_API rz_status rz_quantize_rows_e4m3(const rz_bf16* X, int64_t rows, int32_t d, uint8_t* X8, float* scale,
+                                       void* stream) {
+  if (rows < 0 || rows >= (int64_t{1} << 31) || d < 1) return RZ_ERR_INVALID_ARG;
+  if (rows == 0) return RZ_OK;
+  if (!X || !X8 || !scale || !aligned(X, 2) || !aligned(scale, 4)) return RZ_ERR_INVALID_ARG;
+  quantize_rows_e4m3_kernel<<<static_cast<unsigned>(rows), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const __nv_bfloat16*>(X), d, X8, scale);
+  return cudaGetLastError() == cudaSuccess ? RZ_OK : RZ_ERR_CUDA;
+}
+
+RZ_API rz_status rz_token_logprobs_fp8(const uint8_t* H8, const float* h_scale, const uint8_t* W8,
+                                       const float* w_scale, const int32_t* token_ids, int64_t n_tok, int32_t d,
+                                       int32_t V, float* lp_out, float* lse_out, void* workspace, size_t ws_bytes,
+                                       void* stream) {
+  if (n_tok < 0 || n_tok >= (int64_t{1} << 31)) return RZ_ERR_INVALID_ARG;
+  if (!shape_ok(d, V) || d % BK_FP8 != 0) return RZ_ERR_UNSUPPORTED_SHAPE;
+  if (n_tok == 0) return RZ_OK;
+  if (!H8 || !h_scale || !W8 || !w_scale || !token_ids || !lp_out || !workspace) return RZ_ERR_INVALID_ARG;
+  if (!aligned(H8, 16) || !aligned(W8, 16) || !aligned(h_scale, 4) || !aligned(w_scale, 4) ||
+      !aligned(token_ids, 4) || !aligned(lp_out, 4) || (lse_out && !aligned(lse_out, 4)) ||
+      !aligned(workspace, kAlign))
+    return RZ_ERR_INVALID_ARG;
+  const Layout L = make_layout(n_tok, 0, 0, V, Path::Forward);
+  if (ws_bytes < L.total) return RZ_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(at<int>(workspace, L.status), 0, 16, st) != cudaSuccess) return RZ_ERR_CUDA;
+  return run_forward_fp8(H8, h_scale, W8, w_scale, token_ids, n_tok, d, V, lp_out, lse_out, workspace, L, st);
 }
 
 RZ_API rz_status rz_read_device_status(const void* workspace, void* stream, int32_t* bits_out) {

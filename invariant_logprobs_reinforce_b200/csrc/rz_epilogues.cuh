@@ -61,9 +61,11 @@ struct EpiLse {
   int64_t part_ld;
   float* zy;          // [rows] logit of the sampled token
   float* tile_max;    // STORE_P: [rows][n_tiles]
+  const float* row_scale;  // nullable: logit = acc * row_scale[row] * col_scale[col] (scaled fp8 operands)
+  const float* col_scale;
 
   struct State {
-    float m, s;
+    float m, s, rs;
     int y;
     int64_t row;
   };
@@ -73,6 +75,17 @@ struct EpiLse {
     st.y = st.row < rows ? __ldg(ids + st.row) : -1;
     st.m = -INFINITY;
     st.s = 0.0f;
+    st.rs = (row_scale != nullptr && st.row < rows) ? __ldg(row_scale + st.row) : 1.0f;
+  }
+
+  // scaled operands: z = acc * row_scale * col_scale (one rounding per factor, fixed order)
+  __device__ __forceinline__ void scale_logits(const State& st, int col0, float (&v)[32]) const {
+    if (col_scale == nullptr) return;  // uniform
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float cs = col0 + j < V ? __ldg(col_scale + col0 + j) : 0.0f;
+      v[j] = (v[j] * st.rs) * cs;
+    }
   }
 
   __device__ __forceinline__ void tile(State& st, uint32_t taddr, int mb, int nt, int r, int lane,
@@ -86,6 +99,7 @@ struct EpiLse {
       float v[32];
       __syncwarp();  // the TMEM load is warp-collective: reconverge first
       tmem_ld_32cols(taddr + c * 32, v);
+      scale_logits(st, col0, v);
 #pragma unroll
       for (int j = 0; j < 32; ++j)
         if (col0 + j < V) tmax = fmaxf(tmax, v[j]);
@@ -99,6 +113,7 @@ struct EpiLse {
       float v[32];
       __syncwarp();
       tmem_ld_32cols(taddr + c * 32, v);
+      scale_logits(st, col0, v);
       const unsigned off = static_cast<unsigned>(st.y - col0);
       if (off < 32u) {
         float z = v[0];

@@ -27,7 +27,8 @@ namespace rz {
 
 constexpr int BM = 128;
 constexpr int BN = 256;
-constexpr int BK = 64;
+constexpr int BK = 64;      // bf16 elements per K block (128 bytes)
+constexpr int BK_FP8 = 128; // e4m3 elements per K block (128 bytes)
 constexpr int kStages = 4;
 constexpr int kStageBytesA = BM * BK * 2;  // 16 KB
 constexpr int kStageBytesB = BN * BK * 2;  // 32 KB
@@ -72,11 +73,11 @@ struct OperandPos {
   int b_row_base, b_k_base;
 };
 
-template <bool MN_MAJOR, int ROWS>
+template <bool MN_MAJOR, int ROWS, int KB_ELEMS = BK>
 __device__ __forceinline__ void load_operand(const CUtensorMap* map, uint64_t* bar, uint8_t* dst, int mn0,
                                              int kb, int row_base, int k_base) {
   if constexpr (!MN_MAJOR) {
-    tma_load_2d(map, bar, dst, kb * BK, row_base + mn0);
+    tma_load_2d(map, bar, dst, kb * KB_ELEMS, row_base + mn0);
   } else {
 #pragma unroll
     for (int j = 0; j < ROWS / 64; ++j) tma_load_2d(map, bar, dst + j * 8192, mn0 + j * 64, k_base + kb * BK);
@@ -129,7 +130,9 @@ struct WarpStage {
   }
 };
 
-template <bool A_MN, bool B_MN, class Epi>
+// FP8: e4m3 operands (both K-major), kind::f8f6f4, 128-element K blocks; the stage layout
+// (128-byte rows, 128-byte swizzle) and the per-instruction 32-byte K step are unchanged.
+template <bool A_MN, bool B_MN, class Epi, bool FP8 = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmSched sched, const OperandPos pos, const __grid_constant__ Epi epi,
@@ -198,10 +201,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               break;
             }
             mbar_arrive_expect_tx(&full[stage], kStageBytes);
-            load_operand<A_MN, BM>(&tmA, &full[stage], stage_a + stage * kStageBytesA, m0, kb, pos.a_row_base,
-                                   pos.a_k_base);
-            load_operand<B_MN, BN>(&tmB, &full[stage], stage_b + stage * kStageBytesB, n0, kb, pos.b_row_base,
-                                   pos.b_k_base);
+            constexpr int kKb = FP8 ? BK_FP8 : BK;
+            load_operand<A_MN, BM, kKb>(&tmA, &full[stage], stage_a + stage * kStageBytesA, m0, kb,
+                                        pos.a_row_base, pos.a_k_base);
+            load_operand<B_MN, BN, kKb>(&tmB, &full[stage], stage_b + stage * kStageBytesB, n0, kb,
+                                        pos.b_row_base, pos.b_k_base);
             issued_phase[stage] = static_cast<int>(phase);
             if (++stage == kStages) {
               stage = 0;
@@ -222,7 +226,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ UMMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, A_MN, B_MN);
+      static_assert(!FP8 || (!A_MN && !B_MN), "e4m3 operands are K-major");
+      constexpr uint32_t idesc = FP8 ? idesc_e4m3_f32(BM, BN) : idesc_bf16_f32(BM, BN, A_MN, B_MN);
       int stage = 0;
       uint32_t phase = 0;
       uint32_t it = 0;  // tile counter -> accumulator buffer
@@ -246,9 +251,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint64_t a_desc = operand_desc<A_MN>(smem_u32(stage_a + stage * kStageBytesA));
             const uint64_t b_desc = operand_desc<B_MN>(smem_u32(stage_b + stage * kStageBytesB));
 #pragma unroll
-            for (int k = 0; k < BK / 16; ++k) {
-              umma_bf16(d_tmem, a_desc + k * operand_k_step<A_MN>(), b_desc + k * operand_k_step<B_MN>(), idesc,
-                        (kb | k) != 0 ? 1u : 0u);
+            for (int k = 0; k < 4; ++k) {  // 4 instructions of 32 bytes of K each
+              if constexpr (FP8)
+                umma_e4m3(d_tmem, a_desc + k * operand_k_step<A_MN>(), b_desc + k * operand_k_step<B_MN>(), idesc,
+                          (kb | k) != 0 ? 1u : 0u);
+              else
+                umma_bf16(d_tmem, a_desc + k * operand_k_step<A_MN>(), b_desc + k * operand_k_step<B_MN>(), idesc,
+                          (kb | k) != 0 ? 1u : 0u);
             }
             umma_commit(&empty[stage]);  // stage reusable once these MMAs have read it
             if (++stage == kStages) {

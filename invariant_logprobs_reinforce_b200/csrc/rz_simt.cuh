@@ -13,6 +13,8 @@
 // section "Achieving Bitwise Consistency" (kernel determinism, batch independence).
 #pragma once
 
+#include <cuda_fp8.h>
+
 #include "rz_epilogues.cuh"
 
 namespace rz {
@@ -216,12 +218,14 @@ __global__ void __launch_bounds__(kKappaThreads)
   const bool full = vec_ok && nb == kKappaBlockTokens;
   const int wrel = warp * (kKappaBlockTokens / 8);
   float4 la[kKappaIters], lb[kKappaIters];
+  uint32_t mk[kKappaIters];
   if (full) {
 #pragma unroll
     for (int it = 0; it < kKappaIters; ++it) {
       const int64_t t0 = b0 + wrel + it * 128 + lane * 4;
       la[it] = __ldcs(reinterpret_cast<const float4*>(lp + t0));
       lb[it] = __ldcs(reinterpret_cast<const float4*>(lp_roll + t0));
+      mk[it] = mask != nullptr ? __ldcs(reinterpret_cast<const unsigned int*>(mask + t0)) : 0x01010101u;
     }
   }
   __syncthreads();
@@ -238,8 +242,7 @@ __global__ void __launch_bounds__(kKappaThreads)
       while (s_rel[k + 1] <= tr) ++k;
       const float a4[4] = {la[it].x, la[it].y, la[it].z, la[it].w};
       const float b4[4] = {lb[it].x, lb[it].y, lb[it].z, lb[it].w};
-      uint32_t m4 = 0x01010101u;
-      if (mask != nullptr) m4 = *reinterpret_cast<const uint32_t*>(mask + b0 + tr);
+      const uint32_t m4 = mk[it];
       float w[4], kv[4];
       float part = 0.0f;
 #pragma unroll
@@ -302,6 +305,34 @@ __global__ void loss_final_kernel(const double* __restrict__ block_sums, int nb,
 
 // ------------------------------------------------------------------------ backward
 
+// ------------------------------------------------------------------------ fp8 operands
+//
+// Per-row e4m3 quantisation of a bf16 matrix (one block per row): scale = max|x| / 448
+// (1 for an all-zero row), q = e4m3(x / scale) rounded to nearest even with saturation.
+// x / scale and max|x| / 448 are IEEE fp32 divisions, so the codes are reproducible bit
+// for bit by any fp32 implementation of the same two steps.
+constexpr float kE4m3Max = 448.0f;
+
+__global__ void __launch_bounds__(256)
+    quantize_rows_e4m3_kernel(const __nv_bfloat16* __restrict__ X, int d, uint8_t* __restrict__ Q,
+                              float* __restrict__ scale) {
+  __shared__ float s_max[8];
+  const int64_t row = blockIdx.x;
+  const __nv_bfloat16* x = X + row * d;
+  float m = 0.0f;
+  for (int k = threadIdx.x; k < d; k += blockDim.x) m = fmaxf(m, fabsf(__bfloat162float(x[k])));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) s_max[threadIdx.x >> 5] = m;
+  __syncthreads();
+  m = s_max[0];
+  for (int w = 1; w < 8; ++w) m = fmaxf(m, s_max[w]);
+  const float sc = m > 0.0f ? __fdiv_rn(m, kE4m3Max) : 1.0f;
+  if (threadIdx.x == 0) scale[row] = sc;
+  for (int k = threadIdx.x; k < d; k += blockDim.x)
+    Q[row * d + k] = __nv_cvt_float_to_fp8(__fdiv_rn(__bfloat162float(x[k]), sc), __NV_SATFINITE, __NV_E4M3);
+}
+
 // ------------------------------------------------------------------------ diagnostics
 //
 // Ratio statistics over the counted tokens: sums for the KL estimators k1 = lp_rollout - lp,
@@ -323,6 +354,16 @@ struct StatPartial {
 
 __device__ __forceinline__ float ratio_of(float a, float b) { return ex2_approx((a - b) * kLog2e); }
 
+// Add 1 to s_hist[bin] for every active lane, one shared-memory atomic per distinct bin in
+// the warp (lanes holding equal bins are grouped first; with deviations clustered in a few
+// bins, per-lane atomics would serialise).
+__device__ __forceinline__ void warp_hist_add(unsigned* s_hist, unsigned bin, bool active) {
+  const unsigned live = __ballot_sync(0xffffffffu, active);
+  if (!active) return;
+  const unsigned peers = __match_any_sync(live, bin);
+  if ((threadIdx.x & 31) == static_cast<unsigned>(__ffs(peers) - 1)) atomicAdd(&s_hist[bin], __popc(peers));
+}
+
 __global__ void __launch_bounds__(kStatThreads)
     ratio_stats_pass0(const float* __restrict__ lp, const float* __restrict__ lp_roll, const uint8_t* __restrict__ mask,
                       int64_t n, StatPartial* __restrict__ parts, unsigned* __restrict__ hist) {
@@ -334,23 +375,25 @@ __global__ void __launch_bounds__(kStatThreads)
   double k1 = 0.0, k2 = 0.0, k3 = 0.0;
   float wmin = INFINITY, wmax = -INFINITY, dmax = 0.0f;
   int cnt = 0;
-  for (int j = threadIdx.x; j < kStatTokens; j += kStatThreads) {
+  for (int j = threadIdx.x; j < kStatTokens; j += kStatThreads) {  // uniform trip count per warp
     const int64_t t = b0 + j;
-    if (t >= n) break;
-    if (mask != nullptr && mask[t] == 0) continue;
-    // the KL estimators in fp64 (k3 cancels to second order); min / max / deviation on
-    // the ratio exactly as the loss stage computes it
-    const double x = static_cast<double>(lp[t]) - static_cast<double>(lp_roll[t]);
-    const float w = ratio_of(lp[t], lp_roll[t]);
-    const float dev = fabsf(w - 1.0f);
-    k1 -= x;
-    k2 += 0.5 * x * x;
-    k3 += expm1(x) - x;
-    wmin = fminf(wmin, w);
-    wmax = fmaxf(wmax, w);
-    dmax = fmaxf(dmax, dev);
-    ++cnt;
-    atomicAdd(&s_hist[__float_as_uint(dev) >> 21], 1u);
+    const bool on = t < n && (mask == nullptr || mask[t] != 0);
+    float dev = 0.0f;
+    if (on) {
+      // the KL estimators in fp64 (k3 cancels to second order); min / max / deviation on
+      // the ratio exactly as the loss stage computes it
+      const double x = static_cast<double>(lp[t]) - static_cast<double>(lp_roll[t]);
+      const float w = ratio_of(lp[t], lp_roll[t]);
+      dev = fabsf(w - 1.0f);
+      k1 -= x;
+      k2 += 0.5 * x * x;
+      k3 += expm1(x) - x;
+      wmin = fminf(wmin, w);
+      wmax = fmaxf(wmax, w);
+      dmax = fmaxf(dmax, dev);
+      ++cnt;
+    }
+    warp_hist_add(s_hist, __float_as_uint(dev) >> 21, on);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -391,51 +434,84 @@ __global__ void __launch_bounds__(kStatThreads)
   __syncthreads();
   const unsigned prefix = sel[0];
   const int64_t b0 = static_cast<int64_t>(blockIdx.x) * kStatTokens;
-  for (int j = threadIdx.x; j < kStatTokens; j += kStatThreads) {
+  for (int j = threadIdx.x; j < kStatTokens; j += kStatThreads) {  // uniform trip count per warp
     const int64_t t = b0 + j;
-    if (t >= n) break;
-    if (mask != nullptr && mask[t] == 0) continue;
-    const unsigned key = __float_as_uint(fabsf(ratio_of(lp[t], lp_roll[t]) - 1.0f));
-    if ((key >> shift_hi) == prefix) atomicAdd(&s_hist[(key >> shift) & digit_mask], 1u);
+    bool on = t < n && (mask == nullptr || mask[t] != 0);
+    unsigned key = 0u;
+    if (on) {
+      key = __float_as_uint(fabsf(ratio_of(lp[t], lp_roll[t]) - 1.0f));
+      on = (key >> shift_hi) == prefix;
+    }
+    warp_hist_add(s_hist, (key >> shift) & digit_mask, on);
   }
   __syncthreads();
   for (int b = threadIdx.x; b < kStatBins; b += kStatThreads)
     if (s_hist[b]) atomicAdd(&hist[b], s_hist[b]);
 }
 
-// One thread: find the digit holding rank sel[1] in hist, extend the prefix, keep the rank
-// within that digit, clear hist for the next pass.  On the last pass, write the statistics.
-__global__ void ratio_stats_select(unsigned* __restrict__ hist, int nbins, int digit_bits, unsigned* __restrict__ sel,
-                                   const StatPartial* __restrict__ parts, int nparts, int last,
-                                   double* __restrict__ stats) {
-  if (threadIdx.x != 0) return;
-  if (sel[2] == 0u) {  // first pass: total count and the target rank from the partials
-    long long m = 0;
-    for (int b = 0; b < nparts; ++b) m += parts[b].count;
-    sel[1] = m > 0 ? static_cast<unsigned>((m - 1) / 2) : 0u;
-    sel[2] = 1u;
-    sel[0] = 0u;
+// One block: reduce the per-block partials in a fixed order (strided, then a tree) into
+// acc, and set the target rank floor((m - 1) / 2) of the lower median.
+__global__ void __launch_bounds__(1024)
+    ratio_stats_reduce(const StatPartial* __restrict__ parts, int nparts, StatPartial* __restrict__ acc_out,
+                       unsigned* __restrict__ sel) {
+  __shared__ StatPartial sh[1024];
+  StatPartial a{0.0, 0.0, 0.0, INFINITY, -INFINITY, 0.0f, 0};
+  for (int b = threadIdx.x; b < nparts; b += blockDim.x) {
+    const StatPartial p = parts[b];
+    a.k1 += p.k1;
+    a.k2 += p.k2;
+    a.k3 += p.k3;
+    a.w_min = fminf(a.w_min, p.w_min);
+    a.w_max = fmaxf(a.w_max, p.w_max);
+    a.dev_max = fmaxf(a.dev_max, p.dev_max);
+    a.count += p.count;
   }
+  sh[threadIdx.x] = a;
+  __syncthreads();
+  for (int w = blockDim.x >> 1; w > 0; w >>= 1) {
+    if (threadIdx.x < w) {
+      StatPartial& x = sh[threadIdx.x];
+      const StatPartial& y = sh[threadIdx.x + w];
+      x.k1 += y.k1;
+      x.k2 += y.k2;
+      x.k3 += y.k3;
+      x.w_min = fminf(x.w_min, y.w_min);
+      x.w_max = fmaxf(x.w_max, y.w_max);
+      x.dev_max = fmaxf(x.dev_max, y.dev_max);
+      x.count += y.count;
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    *acc_out = sh[0];
+    sel[0] = 0u;
+    sel[1] = sh[0].count > 0 ? static_cast<unsigned>((sh[0].count - 1) / 2) : 0u;
+  }
+}
+
+// One block: find the digit holding rank sel[1] in hist (bins staged in shared memory),
+// extend the prefix, keep the rank within that digit, clear hist for the next pass.  On
+// the last pass, write the statistics.
+__global__ void __launch_bounds__(1024)
+    ratio_stats_select(unsigned* __restrict__ hist, int nbins, int digit_bits, unsigned* __restrict__ sel,
+                       const StatPartial* __restrict__ acc_in, int last, double* __restrict__ stats) {
+  __shared__ unsigned s_hist[kStatBins];
+  for (int b = threadIdx.x; b < nbins; b += blockDim.x) {
+    s_hist[b] = hist[b];
+    hist[b] = 0u;
+  }
+  __syncthreads();
+  if (threadIdx.x != 0) return;
   unsigned rank = sel[1];
   int digit = 0;
   for (; digit < nbins - 1; ++digit) {
-    if (rank < hist[digit]) break;
-    rank -= hist[digit];
+    if (rank < s_hist[digit]) break;
+    rank -= s_hist[digit];
   }
-  for (int b = 0; b < nbins; ++b) hist[b] = 0u;
   sel[0] = (sel[0] << digit_bits) | static_cast<unsigned>(digit);
   sel[1] = rank;
   if (!last) return;
-  StatPartial acc = parts[0];
-  for (int b = 1; b < nparts; ++b) {
-    acc.k1 += parts[b].k1;
-    acc.k2 += parts[b].k2;
-    acc.k3 += parts[b].k3;
-    acc.w_min = fminf(acc.w_min, parts[b].w_min);
-    acc.w_max = fmaxf(acc.w_max, parts[b].w_max);
-    acc.dev_max = fmaxf(acc.dev_max, parts[b].dev_max);
-    acc.count += parts[b].count;
-  }
+  const StatPartial acc = *acc_in;
   const double m = acc.count > 0 ? static_cast<double>(acc.count) : 1.0;
   const double med = static_cast<double>(__uint_as_float(sel[0]));
   stats[0] = acc.k1 / m;

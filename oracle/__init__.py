@@ -245,3 +245,25 @@ def ratio_stats(lp, lp_rollout, seg_offsets, mask=None):
     _check(lib.oracle_ratio_stats(_ptr(lp), _ptr(lr), _ptr(off), n, R, _ptr(mk), _ptr(stats), _ptr(rm)),
            "ratio_stats")
     return dict(zip(STAT_NAMES, stats.tolist())), rm
+
+
+E4M3_MAX = 448.0
+
+
+def quantize_rows_e4m3(X_bits):
+    """Per-row e4m3 codes of a bf16 matrix (uint16 bit patterns): scale = max|x| / 448 in fp32
+    (1 for an all-zero row), code = e4m3(x / scale) with fp32 division, round to nearest
+    even (torch's CPU conversion).  Returns (codes uint8 [rows, d], scale fp32 [rows])."""
+    import torch
+    x = torch.from_numpy(np.ascontiguousarray(X_bits).view(np.int16)).view(torch.bfloat16).float()
+    m = x.abs().amax(dim=1)
+    sc = torch.where(m > 0, m / torch.tensor(E4M3_MAX, dtype=torch.float32), torch.ones_like(m))
+    y = (x / sc[:, None]).clamp(-E4M3_MAX, E4M3_MAX)
+    q = y.to(torch.float8_e4m3fn)
+    return q.view(torch.uint8).numpy().copy(), sc.numpy().copy()
+
+
+def decode_e4m3(codes):
+    """fp64 values of e4m3 codes (uint8)."""
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(codes)).view(torch.float8_e4m3fn).double().numpy()

@@ -336,3 +336,25 @@ def test_invalid_inputs_are_rejected(oracle, bad):
         p["seg_offsets"] = np.array([0, 3, 3, 6, 10], np.int64)
     with pytest.raises(oracle.OracleError):
         _loss(oracle, p)
+
+
+# ---------------------------------------------------------------- e4m3 operands
+
+def test_e4m3_quantisation_reference(oracle):
+    """Codes decode to x / scale rounded to e4m3 (3 mantissa bits): exact for values that
+    are e4m3 numbers times the scale, within half an e4m3 ulp otherwise; the row maximum
+    maps to +-448; zero rows get scale 1 and zero codes."""
+    rng = np.random.default_rng(0)
+    X = rng.standard_normal((5, 64)).astype(np.float32)
+    X[3] = 0.0
+    X[4] = np.array([2.0 ** k for k in range(-6, 2)] * 8, np.float32)  # x / scale = 224 x: 3.5 .. 448, all e4m3
+    bits = wl.bf16_bits(X)
+    q, sc = oracle.quantize_rows_e4m3(bits)
+    xf = wl.bits_to_f32(bits).astype(np.float64)
+    dec = oracle.decode_e4m3(q) * sc[:, None].astype(np.float64)
+    assert sc[3] == 1.0 and np.all(q[3] == 0)
+    for r in (0, 1, 2):
+        assert np.max(np.abs(oracle.decode_e4m3(q[r]))) == 448.0
+        rel = np.abs(dec[r] - xf[r]) / np.maximum(np.abs(xf[r]), 2.0 ** -6 * sc[r])
+        assert rel.max() <= 2.0 ** -4 + 1e-12
+    np.testing.assert_array_equal(oracle.decode_e4m3(q[4]), xf[4] * 224.0)
