@@ -236,6 +236,30 @@ rz_status rz_token_logprobs_fp8(const uint8_t* H8, const float* h_scale, const u
                                 const int32_t* token_ids, int64_t n_tok, int32_t d, int32_t V, float* lp_out,
                                 float* lse_out, void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * Cross-GPU consistency ("vLLM Train-Inference Consistency Release Notes", section
+ * "Achieving Bitwise Consistency": communication reductions that do not vary with timing
+ * or scheduling).  The reduction step of a data-parallel all-reduce of dW:
+ *   out[i] = sum_{r = 0 .. nshards-1} stacked[r * count + i]
+ * in rank order, accumulated in fp64 and rounded once, so the result is the same bits on
+ * every rank whatever collective moved the shards.  stacked [nshards, count] fp32 and out
+ * [count] fp32 are device arrays; used after an all-to-all that gives each rank its slice
+ * from every rank, before an all-gather (invariant_logprobs_reinforce_b200.dp).
+ */
+rz_status rz_sum_shards_f32(const float* stacked, int32_t nshards, int64_t count, float* out, void* stream);
+
+/*
+ * Self-test of the bounded waits: every mbarrier wait in this library gives up after a time
+ * limit (4 s in the kernels) instead of spinning forever, sets RZ_DEV_WAIT_TIMEOUT in the
+ * status word and lets the kernel exit normally.  This launches one thread that waits, with
+ * limit_ns (at most 10 s), on a barrier nothing arrives on.  Afterwards
+ * rz_read_device_status(workspace) reports RZ_ERR_DEVICE_TIMEOUT; waited_ns_out (host,
+ * nullable; when given the call synchronises the stream) receives the time waited.
+ * workspace: at least 256 bytes, 256-byte aligned.
+ */
+rz_status rz_selftest_wait_timeout(uint64_t limit_ns, void* workspace, size_t ws_bytes, uint64_t* waited_ns_out,
+                                   void* stream);
+
 /* Kernel kinds reported per launch by rz_loss_fwd_bwd_timed. */
 #define RZ_KERNEL_LMHEAD_LSE 0    /* fused LM head + online log-sum-exp + gather (tensor cores) */
 #define RZ_KERNEL_MERGE_LSE 1     /* fixed-order merge of the vocabulary-segment partials       */

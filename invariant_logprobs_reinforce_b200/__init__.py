@@ -28,7 +28,7 @@ EXPORTED_SYMBOLS = (
     "rz_token_logprobs", "rz_loss_fwd_bwd", "rz_segment_loss", "rz_read_device_status", "rz_num_launches_loss",
     "rz_loss_fwd_bwd_timed", "rz_token_logprobs_noalloc", "rz_loss_fwd_bwd_ex", "rz_segment_loss_ex",
     "rz_workspace_bytes_ratio_stats", "rz_ratio_stats", "rz_workspace_bytes_grad_norms", "rz_grad_norms",
-    "rz_quantize_rows_e4m3", "rz_token_logprobs_fp8",
+    "rz_quantize_rows_e4m3", "rz_token_logprobs_fp8", "rz_sum_shards_f32", "rz_selftest_wait_timeout",
 )
 RZ_LOSS_CLIP_IS, RZ_LOSS_SEQ_GATE, RZ_LOSS_TOKEN_MASK = 1, 2, 4
 STAT_NAMES = ("k1", "k2", "k3", "w_min", "w_max", "dev_max", "dev_median", "dev_peak_over_median", "count")
@@ -114,6 +114,10 @@ def lib() -> ctypes.CDLL:
         L.rz_quantize_rows_e4m3.restype = ctypes.c_int
         L.rz_token_logprobs_fp8.argtypes = [P, P, P, P, P, i64, i32, i32, P, P, P, sz, P]
         L.rz_token_logprobs_fp8.restype = ctypes.c_int
+        L.rz_sum_shards_f32.argtypes = [P, i32, i64, P, P]
+        L.rz_sum_shards_f32.restype = ctypes.c_int
+        L.rz_selftest_wait_timeout.argtypes = [ctypes.c_uint64, P, sz, ctypes.POINTER(ctypes.c_uint64), P]
+        L.rz_selftest_wait_timeout.restype = ctypes.c_int
         L.rz_read_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
         L.rz_read_device_status.restype = ctypes.c_int
         _lib = L
@@ -401,3 +405,25 @@ def rz_token_logprobs_fp8(H8, h_scale, W8, w_scale, token_ids, lp_out=None, lse_
                                        _ptr(lp), _ptr(lse), _ptr(ws), ws.numel(), _stream_handle(stream))
     _check(code, "rz_token_logprobs_fp8")
     return lp, lse
+
+
+def rz_sum_shards_f32(stacked, out=None, stream=None):
+    """Rank-order sum of the rows of a [nshards, count] fp32 CUDA tensor (fp64 accumulation)."""
+    torch = _torch()
+    _need(stacked, torch.float32, "stacked")
+    nshards, count = stacked.shape
+    out = out if out is not None else torch.empty(count, dtype=torch.float32, device=stacked.device)
+    _check(lib().rz_sum_shards_f32(_ptr(stacked), nshards, count, _ptr(out), _stream_handle(stream)),
+           "rz_sum_shards_f32")
+    return out
+
+
+def rz_selftest_wait_timeout(limit_ns: int, stream=None):
+    """Run the bounded-wait self-test; returns (status code, status bits, waited ns)."""
+    torch = _torch()
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    waited = ctypes.c_uint64(0)
+    _check(lib().rz_selftest_wait_timeout(limit_ns, _ptr(ws), ws.numel(), ctypes.byref(waited),
+                                          _stream_handle(stream)), "rz_selftest_wait_timeout")
+    code, bits = rz_read_device_status(ws, stream)
+    return code, bits, int(waited.value)

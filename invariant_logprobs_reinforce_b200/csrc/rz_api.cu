@@ -831,6 +831,35 @@ RZ_API rz_status rz_token_logprobs_fp8(const uint8_t* H8, const float* h_scale, 
   return run_forward_fp8(H8, h_scale, W8, w_scale, token_ids, n_tok, d, V, lp_out, lse_out, workspace, L, st);
 }
 
+RZ_API rz_status rz_sum_shards_f32(const float* stacked, int32_t nshards, int64_t count, float* out, void* stream) {
+  if (nshards < 1 || count < 0 || count > (int64_t{1} << 40)) return RZ_ERR_INVALID_ARG;
+  if (count == 0) return RZ_OK;
+  if (!stacked || !out || !aligned(stacked, 4) || !aligned(out, 4)) return RZ_ERR_INVALID_ARG;
+  const int sms = sm_count();
+  if (sms <= 0) return RZ_ERR_CUDA;
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(ceil_div(count, 256), int64_t{8} * sms));
+  sum_shards_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(stacked, nshards, count, out);
+  return cudaGetLastError() == cudaSuccess ? RZ_OK : RZ_ERR_CUDA;
+}
+
+RZ_API rz_status rz_selftest_wait_timeout(uint64_t limit_ns, void* workspace, size_t ws_bytes,
+                                          uint64_t* waited_ns_out, void* stream) {
+  if (!workspace || ws_bytes < 256 || !aligned(workspace, kAlign) || limit_ns > 10000000000ull)
+    return RZ_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(workspace, 0, 16, st) != cudaSuccess) return RZ_ERR_CUDA;
+  unsigned long long* waited = at<unsigned long long>(workspace, 16);
+  wait_timeout_selftest_kernel<<<1, 32, 0, st>>>(limit_ns, static_cast<int*>(workspace), waited);
+  if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
+  if (waited_ns_out != nullptr) {
+    unsigned long long w = 0;
+    if (cudaMemcpyAsync(&w, waited, sizeof(w), cudaMemcpyDeviceToHost, st) != cudaSuccess) return RZ_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return RZ_ERR_CUDA;
+    *waited_ns_out = w;
+  }
+  return RZ_OK;
+}
+
 RZ_API rz_status rz_read_device_status(const void* workspace, void* stream, int32_t* bits_out) {
   if (!workspace) return RZ_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -333,6 +333,37 @@ __global__ void __launch_bounds__(256)
     Q[row * d + k] = __nv_cvt_float_to_fp8(__fdiv_rn(__bfloat162float(x[k]), sc), __NV_SATFINITE, __NV_E4M3);
 }
 
+// ------------------------------------------------------------------------ self-test
+//
+// The bounded-wait path of every kernel here, exercised on its own: one thread waits on an
+// mbarrier that nothing arrives on, with the given limit; the wait gives up, the kernel
+// sets the timeout status bit and records how long it waited, and returns normally.
+__global__ void wait_timeout_selftest_kernel(uint64_t limit_ns, int* status, unsigned long long* waited_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_mbarrier_init();
+  const uint64_t t0 = global_timer_ns();
+  const bool ok = mbar_wait(&bar, 0, nullptr, limit_ns);  // phase 0 never completes
+  *waited_ns = global_timer_ns() - t0;
+  if (!ok) atomicOr(status, kDevWaitTimeout);
+}
+
+// ------------------------------------------------------------------------ cross-GPU sum
+//
+// out[i] = sum over r = 0 .. nshards-1, in that order, of stacked[r * count + i]
+// (fp64 accumulation, one rounding to fp32): the reduction step of a data-parallel
+// all-reduce whose result does not depend on timing, topology or the collective library.
+__global__ void __launch_bounds__(256)
+    sum_shards_kernel(const float* __restrict__ stacked, int nshards, int64_t count, float* __restrict__ out) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < count; i += stride) {
+    double acc = 0.0;
+    for (int r = 0; r < nshards; ++r) acc += static_cast<double>(__ldcs(stacked + r * count + i));
+    out[i] = static_cast<float>(acc);
+  }
+}
+
 // ------------------------------------------------------------------------ diagnostics
 //
 // Ratio statistics over the counted tokens: sums for the KL estimators k1 = lp_rollout - lp,

@@ -42,6 +42,46 @@ def test_max_over_ranks_and_throughput():
     assert bench.job_throughput(1000, 2, 500.0) == pytest.approx(4000.0)
 
 
+def _dar_worker(rank, world, port, out):
+    sys.path.insert(0, ROOT)
+    import torch
+    from invariant_logprobs_reinforce_b200 import dp
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        g = torch.Generator().manual_seed(100 + rank)
+        x = (torch.randn(1001, generator=g) * 10 ** torch.randn(1001, generator=g)).float()  # 1001: uneven slices
+
+        def rank_order_sum(stacked):  # the librz kernel's arithmetic (fp64, rank order), for CPU ranks
+            acc = torch.zeros(stacked.shape[1], dtype=torch.float64)
+            for r in range(stacked.shape[0]):
+                acc += stacked[r].double()
+            return acc.float()
+
+        y = dp.deterministic_all_reduce(x, sum_shards=rank_order_sum)
+        out[rank] = (x.numpy().tobytes(), y.numpy().tobytes())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_deterministic_all_reduce_orchestration():
+    """all-to-all of slices, rank-order sum, all-gather: the same bits on every rank,
+    equal to the rank-order fp64 sum of the inputs."""
+    import numpy as np
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        mp.start_processes(_dar_worker, args=(2, _free_port(), out), nprocs=2, join=True, start_method="spawn")
+        res = dict(out)
+    x0 = np.frombuffer(res[0][0], np.float32)
+    x1 = np.frombuffer(res[1][0], np.float32)
+    y0 = np.frombuffer(res[0][1], np.float32)
+    y1 = np.frombuffer(res[1][1], np.float32)
+    assert y0.tobytes() == y1.tobytes()
+    ref = (x0.astype(np.float64) + x1.astype(np.float64)).astype(np.float32)
+    assert np.array_equal(y0.view(np.uint32), ref.view(np.uint32))
+
+
 def test_reference_arm_under_torchrun_prints_once():
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
            "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), "bench.py", "--impl", "reference",

@@ -100,3 +100,16 @@ def test_optional_outputs_and_empty_call(rz, prob):
     ids0 = torch.empty((0,), dtype=torch.int32, device="cuda")
     lp0, _ = rz.rz_token_logprobs(H0, dev["W"], ids0)
     assert lp0.numel() == 0
+
+
+def test_bounded_wait_gives_up_and_reports_timeout(rz):
+    """A wait on a barrier nothing arrives on ends after its limit with the timeout status;
+    the context stays usable (a normal call follows)."""
+    code, bits, waited = rz.rz_selftest_wait_timeout(50_000_000)  # 50 ms
+    assert code == 6 and bits & 8  # RZ_ERR_DEVICE_TIMEOUT, RZ_DEV_WAIT_TIMEOUT
+    assert 50_000_000 <= waited < 2_000_000_000
+    H = torch.randn(10, 64, device="cuda").to(torch.bfloat16)
+    W = torch.randn(100, 64, device="cuda").to(torch.bfloat16)
+    ids = torch.randint(0, 100, (10,), device="cuda", dtype=torch.int32)
+    lp, _ = rz.rz_token_logprobs(H, W, ids)
+    assert torch.isfinite(lp).all()
