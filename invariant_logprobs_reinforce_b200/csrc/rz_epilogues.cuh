@@ -90,29 +90,21 @@ struct EpiLse {
 
   __device__ __forceinline__ void tile(State& st, uint32_t taddr, int mb, int nt, int r, int lane,
                                        WarpStage& stage) const {
+    // chunks of 32 columns holding at least one column < V (uniform across the warp)
+    const int nch = min(BN / 32, (V - nt * BN + 31) / 32);
     // pass 1: tile maximum over the valid columns
     float tmax = -INFINITY;
-#pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    tmem_for_chunks(taddr, nch, [&](int c, float (&v)[32]) {
       const int col0 = nt * BN + c * 32;
-      if (col0 >= V) break;  // uniform across the warp
-      float v[32];
-      __syncwarp();  // the TMEM load is warp-collective: reconverge first
-      tmem_ld_32cols(taddr + c * 32, v);
       scale_logits(st, col0, v);
 #pragma unroll
       for (int j = 0; j < 32; ++j)
         if (col0 + j < V) tmax = fmaxf(tmax, v[j]);
-    }
+    });
     // pass 2: exponentials relative to the tile maximum, their sum, the gather
     float tsum = 0.0f;
-#pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    tmem_for_chunks(taddr, nch, [&](int c, float (&v)[32]) {
       const int col0 = nt * BN + c * 32;
-      if (col0 >= V) break;
-      float v[32];
-      __syncwarp();
-      tmem_ld_32cols(taddr + c * 32, v);
       scale_logits(st, col0, v);
       const unsigned off = static_cast<unsigned>(st.y - col0);
       if (off < 32u) {
@@ -135,7 +127,7 @@ struct EpiLse {
                               pack_half2(e[8 * q + 4], e[8 * q + 5]), pack_half2(e[8 * q + 6], e[8 * q + 7]));
         stage.store_rows(&p_map, lane, row, col0, mb * BM + (r - lane), rows);
       }
-    }
+    });
     const float m_new = fmaxf(st.m, tmax);
     st.s = st.s * ex2_approx((st.m - m_new) * kLog2e) + tsum * ex2_approx((tmax - m_new) * kLog2e);
     st.m = m_new;
@@ -162,20 +154,16 @@ struct EpiDh {
 
   __device__ __forceinline__ void tile(State&, uint32_t taddr, int mb, int nt, int r, int lane,
                                        WarpStage& stage) const {
-#pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    const int nch = min(BN / 32, (out_cols - nt * BN) / 32);
+    tmem_for_chunks(taddr, nch, [&](int c, float (&v)[32]) {
       const int col0 = nt * BN + c * 32;
-      if (col0 >= out_cols) break;
-      float v[32];
-      __syncwarp();
-      tmem_ld_32cols(taddr + c * 32, v);
       uint4 row[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q)
         row[q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
                             pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
       stage.store_rows(&out_map, lane, row, col0, mb * BM + (r - lane), out_rows);
-    }
+    });
   }
 
   __device__ __forceinline__ void end_unit(const State&, int, int, int) const {}
@@ -199,13 +187,9 @@ struct EpiDw {
 
   __device__ __forceinline__ void tile(State&, uint32_t taddr, int mb, int nt, int r, int lane,
                                        WarpStage& stage) const {
-#pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    const int nch = min(BN / 32, (out_cols - nt * BN) / 32);
+    tmem_for_chunks(taddr, nch, [&](int c, float (&v)[32]) {
       const int col0 = nt * BN + c * 32;
-      if (col0 >= out_cols) break;
-      float v[32];
-      __syncwarp();
-      tmem_ld_32cols(taddr + c * 32, v);
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint4 row[4];
@@ -215,7 +199,7 @@ struct EpiDw {
                               __float_as_uint(v[16 * h + 4 * q + 2]), __float_as_uint(v[16 * h + 4 * q + 3]));
         stage.store_rows(&out_map, lane, row, col0 + 16 * h, mb * BM + (r - lane), out_rows, accumulate != 0);
       }
-    }
+    });
   }
 
   __device__ __forceinline__ void end_unit(const State&, int, int, int) const {}

@@ -196,6 +196,61 @@ __device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, float (&v)[32]) {
   for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
 }
 
+// Split TMEM load: issue 32 columns now, wait later.  The wait names the destination
+// registers as read-write operands so no use of them can be scheduled before it.
+__device__ __forceinline__ void tmem_ld_issue(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+// Wait for every TMEM load this thread issued; r (the last load's registers) is ready after.
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                 "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                 "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
+}
+
+// Visit the 32-column chunks c = 0 .. nchunks-1 of a TMEM accumulator row block, loading
+// chunk c+1 while chunk c is processed (two register sets).  fn(c, float (&v)[32]).
+// Every lane of the warp must call this with the same arguments (warp-collective loads).
+template <class Fn>
+__device__ __forceinline__ void tmem_for_chunks(uint32_t taddr, int nchunks, Fn&& fn) {
+  uint32_t ra[32], rb[32];
+  float v[32];
+  if (nchunks <= 0) return;
+  __syncwarp();
+  tmem_ld_issue(taddr, ra);
+#pragma unroll 1
+  for (int c = 0; c < nchunks; c += 2) {
+    tmem_ld_wait(ra);
+    if (c + 1 < nchunks) tmem_ld_issue(taddr + (c + 1) * 32, rb);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(ra[j]);
+    fn(c, v);
+    if (c + 1 >= nchunks) break;
+    __syncwarp();
+    tmem_ld_wait(rb);
+    if (c + 2 < nchunks) tmem_ld_issue(taddr + (c + 2) * 32, ra);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(rb[j]);
+    fn(c + 1, v);
+    __syncwarp();
+  }
+}
+
 // ---------------------------------------------------------------- UMMA descriptors
 
 // Shared-memory matrix descriptor for a 128-byte-swizzled bf16 tile (sm_100 format):
