@@ -75,12 +75,13 @@ struct OperandPos {
 
 template <bool MN_MAJOR, int ROWS, int KB_ELEMS = BK>
 __device__ __forceinline__ void load_operand(const CUtensorMap* map, uint64_t* bar, uint8_t* dst, int mn0,
-                                             int kb, int row_base, int k_base) {
+                                             int kb, int row_base, int k_base, uint64_t pol) {
   if constexpr (!MN_MAJOR) {
-    tma_load_2d(map, bar, dst, kb * KB_ELEMS, row_base + mn0);
+    tma_load_2d(map, bar, dst, kb * KB_ELEMS, row_base + mn0, pol);
   } else {
 #pragma unroll
-    for (int j = 0; j < ROWS / 64; ++j) tma_load_2d(map, bar, dst + j * 8192, mn0 + j * 64, k_base + kb * BK);
+    for (int j = 0; j < ROWS / 64; ++j)
+      tma_load_2d(map, bar, dst + j * 8192, mn0 + j * 64, k_base + kb * BK, pol);
   }
 }
 
@@ -186,6 +187,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      const uint64_t pol_a = make_l2_policy<Epi::kL2PolicyA>();
+      const uint64_t pol_b = make_l2_policy<Epi::kL2PolicyB>();
       int issued_phase[kStages];
 #pragma unroll
       for (int s = 0; s < kStages; ++s) issued_phase[s] = -1;
@@ -203,9 +206,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_arrive_expect_tx(&full[stage], kStageBytes);
             constexpr int kKb = FP8 ? BK_FP8 : BK;
             load_operand<A_MN, BM, kKb>(&tmA, &full[stage], stage_a + stage * kStageBytesA, m0, kb,
-                                        pos.a_row_base, pos.a_k_base);
+                                        pos.a_row_base, pos.a_k_base, pol_a);
             load_operand<B_MN, BN, kKb>(&tmB, &full[stage], stage_b + stage * kStageBytesB, n0, kb,
-                                        pos.b_row_base, pos.b_k_base);
+                                        pos.b_row_base, pos.b_k_base, pol_b);
             issued_phase[stage] = static_cast<int>(phase);
             if (++stage == kStages) {
               stage = 0;

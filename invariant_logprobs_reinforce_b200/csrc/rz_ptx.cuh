@@ -83,13 +83,30 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
-// 2D tiled load of one box into shared memory, completing on `bar` (transaction bytes).
+// L2 eviction priority of an operand's lines: a stream read once goes first, a block
+// that every tile of the launch re-reads stays.
+enum L2Policy : int { kL2Normal = 0, kL2EvictFirst = 1, kL2EvictLast = 2 };
+
+template <int POL>
+__device__ __forceinline__ uint64_t make_l2_policy() {
+  uint64_t p;
+  if constexpr (POL == kL2EvictFirst)
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  else if constexpr (POL == kL2EvictLast)
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  else
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// 2D tiled load of one box into shared memory, completing on `bar` (transaction bytes),
+// with the L2 policy `pol` (from make_l2_policy) on the lines it reads.
 __device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* bar, void* dst, int32_t x,
-                                            int32_t y) {
+                                            int32_t y, uint64_t pol) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(pol)
       : "memory");
 }
 
