@@ -385,6 +385,27 @@ struct StatPartial {
 
 __device__ __forceinline__ float ratio_of(float a, float b) { return ex2_approx((a - b) * kLog2e); }
 
+// e^x - 1 - x in fp64.  For |x| < 1/2 the Taylor series x^2 (1/2! + x/3! + ... + x^11/13!)
+// by Horner's rule (truncation below 1e-14 relative); outside that range expm1(x) - x.
+__device__ __forceinline__ double expm1_minus_x(double x) {
+  if (fabs(x) < 0.5) {
+    double p = 1.0 / 6227020800.0;  // 1/13!
+    p = fma(p, x, 1.0 / 479001600.0);
+    p = fma(p, x, 1.0 / 39916800.0);
+    p = fma(p, x, 1.0 / 3628800.0);
+    p = fma(p, x, 1.0 / 362880.0);
+    p = fma(p, x, 1.0 / 40320.0);
+    p = fma(p, x, 1.0 / 5040.0);
+    p = fma(p, x, 1.0 / 720.0);
+    p = fma(p, x, 1.0 / 120.0);
+    p = fma(p, x, 1.0 / 24.0);
+    p = fma(p, x, 1.0 / 6.0);
+    p = fma(p, x, 0.5);
+    return p * x * x;
+  }
+  return expm1(x) - x;
+}
+
 // Add 1 to s_hist[bin] for every active lane, one shared-memory atomic per distinct bin in
 // the warp (lanes holding equal bins are grouped first; with deviations clustered in a few
 // bins, per-lane atomics would serialise).
@@ -395,36 +416,74 @@ __device__ __forceinline__ void warp_hist_add(unsigned* s_hist, unsigned bin, bo
   if ((threadIdx.x & 31) == static_cast<unsigned>(__ffs(peers) - 1)) atomicAdd(&s_hist[bin], __popc(peers));
 }
 
+// A block covers kStatTokens tokens as quads of 4 consecutive tokens, kStatQuads per
+// thread, all loaded before any is used (16-byte loads when `vec`: both arrays 16-byte
+// aligned; scalar loads at the tail of the array).
+constexpr int kStatQuads = kStatTokens / 4 / kStatThreads;
+
+struct StatQuads {
+  float a[kStatQuads][4], b[kStatQuads][4];
+  bool on[kStatQuads][4];
+};
+
+__device__ __forceinline__ void load_stat_quads(const float* __restrict__ lp, const float* __restrict__ lp_roll,
+                                                const uint8_t* __restrict__ mask, int64_t n, bool vec,
+                                                StatQuads& q) {
+  const int64_t b0 = static_cast<int64_t>(blockIdx.x) * kStatTokens;
+#pragma unroll
+  for (int k = 0; k < kStatQuads; ++k) {
+    const int64_t t = b0 + 4 * (threadIdx.x + k * kStatThreads);
+    if (vec && t + 3 < n) {
+      const float4 x = __ldcs(reinterpret_cast<const float4*>(lp + t));
+      const float4 y = __ldcs(reinterpret_cast<const float4*>(lp_roll + t));
+      q.a[k][0] = x.x, q.a[k][1] = x.y, q.a[k][2] = x.z, q.a[k][3] = x.w;
+      q.b[k][0] = y.x, q.b[k][1] = y.y, q.b[k][2] = y.z, q.b[k][3] = y.w;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        q.a[k][i] = t + i < n ? __ldcs(lp + t + i) : 0.0f;
+        q.b[k][i] = t + i < n ? __ldcs(lp_roll + t + i) : 0.0f;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) q.on[k][i] = t + i < n && (mask == nullptr || mask[t + i] != 0);
+  }
+}
+
 __global__ void __launch_bounds__(kStatThreads)
     ratio_stats_pass0(const float* __restrict__ lp, const float* __restrict__ lp_roll, const uint8_t* __restrict__ mask,
-                      int64_t n, StatPartial* __restrict__ parts, unsigned* __restrict__ hist) {
+                      int64_t n, bool vec, StatPartial* __restrict__ parts, unsigned* __restrict__ hist) {
   __shared__ unsigned s_hist[kStatBins];
   __shared__ StatPartial s_part[kStatThreads / 32];
   for (int b = threadIdx.x; b < kStatBins; b += kStatThreads) s_hist[b] = 0u;
+  StatQuads q;
+  load_stat_quads(lp, lp_roll, mask, n, vec, q);
   __syncthreads();
-  const int64_t b0 = static_cast<int64_t>(blockIdx.x) * kStatTokens;
   double k1 = 0.0, k2 = 0.0, k3 = 0.0;
   float wmin = INFINITY, wmax = -INFINITY, dmax = 0.0f;
   int cnt = 0;
-  for (int j = threadIdx.x; j < kStatTokens; j += kStatThreads) {  // uniform trip count per warp
-    const int64_t t = b0 + j;
-    const bool on = t < n && (mask == nullptr || mask[t] != 0);
-    float dev = 0.0f;
-    if (on) {
-      // the KL estimators in fp64 (k3 cancels to second order); min / max / deviation on
-      // the ratio exactly as the loss stage computes it
-      const double x = static_cast<double>(lp[t]) - static_cast<double>(lp_roll[t]);
-      const float w = ratio_of(lp[t], lp_roll[t]);
-      dev = fabsf(w - 1.0f);
-      k1 -= x;
-      k2 += 0.5 * x * x;
-      k3 += expm1(x) - x;
-      wmin = fminf(wmin, w);
-      wmax = fmaxf(wmax, w);
-      dmax = fmaxf(dmax, dev);
-      ++cnt;
+#pragma unroll
+  for (int k = 0; k < kStatQuads; ++k) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const bool on = q.on[k][i];
+      float dev = 0.0f;
+      if (on) {
+        // the KL estimators in fp64 (k3 cancels to second order); min / max / deviation
+        // on the ratio exactly as the loss stage computes it
+        const double x = static_cast<double>(q.a[k][i]) - static_cast<double>(q.b[k][i]);
+        const float w = ratio_of(q.a[k][i], q.b[k][i]);
+        dev = fabsf(w - 1.0f);
+        k1 -= x;
+        k2 += 0.5 * x * x;
+        k3 += expm1_minus_x(x);
+        wmin = fminf(wmin, w);
+        wmax = fmaxf(wmax, w);
+        dmax = fmaxf(dmax, dev);
+        ++cnt;
+      }
+      warp_hist_add(s_hist, __float_as_uint(dev) >> 21, on);
     }
-    warp_hist_add(s_hist, __float_as_uint(dev) >> 21, on);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -458,22 +517,26 @@ __global__ void __launch_bounds__(kStatThreads)
 // Histogram of the next radix digit among the deviations whose higher bits equal `prefix`.
 __global__ void __launch_bounds__(kStatThreads)
     ratio_stats_pass(const float* __restrict__ lp, const float* __restrict__ lp_roll, const uint8_t* __restrict__ mask,
-                     int64_t n, const unsigned* __restrict__ sel, int shift_hi, int shift, unsigned digit_mask,
-                     unsigned* __restrict__ hist) {
+                     int64_t n, bool vec, const unsigned* __restrict__ sel, int shift_hi, int shift,
+                     unsigned digit_mask, unsigned* __restrict__ hist) {
   __shared__ unsigned s_hist[kStatBins];
   for (int b = threadIdx.x; b < kStatBins; b += kStatThreads) s_hist[b] = 0u;
-  __syncthreads();
+  StatQuads q;
+  load_stat_quads(lp, lp_roll, mask, n, vec, q);
   const unsigned prefix = sel[0];
-  const int64_t b0 = static_cast<int64_t>(blockIdx.x) * kStatTokens;
-  for (int j = threadIdx.x; j < kStatTokens; j += kStatThreads) {  // uniform trip count per warp
-    const int64_t t = b0 + j;
-    bool on = t < n && (mask == nullptr || mask[t] != 0);
-    unsigned key = 0u;
-    if (on) {
-      key = __float_as_uint(fabsf(ratio_of(lp[t], lp_roll[t]) - 1.0f));
-      on = (key >> shift_hi) == prefix;
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < kStatQuads; ++k) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      bool on = q.on[k][i];
+      unsigned key = 0u;
+      if (on) {
+        key = __float_as_uint(fabsf(ratio_of(q.a[k][i], q.b[k][i]) - 1.0f));
+        on = (key >> shift_hi) == prefix;
+      }
+      warp_hist_add(s_hist, (key >> shift) & digit_mask, on);
     }
-    warp_hist_add(s_hist, (key >> shift) & digit_mask, on);
   }
   __syncthreads();
   for (int b = threadIdx.x; b < kStatBins; b += kStatThreads)

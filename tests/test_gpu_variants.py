@@ -145,6 +145,47 @@ def test_ratio_stats_against_oracle(rz, oracle, masked):
     np.testing.assert_allclose(rm.cpu().numpy(), rm_o, rtol=2e-6)
 
 
+def test_ratio_stats_same_bits_at_any_alignment(rz, oracle):
+    """16-byte aligned inputs take vector loads, others scalar ones; the token -> thread
+    assignment is the same, so the statistics must not change by a bit.  A ragged n
+    (not a multiple of 4) exercises the scalar tail of both."""
+    seg, lp, lr, mask = _stage_inputs(seed=41)
+    n = int(seg.seg_offsets[-1]) - 3
+    off = seg.seg_offsets.copy()
+    off[-1] = n
+    off_t = _t(off)
+    a_lp, a_lr, a_m = _t(lp[:n]), _t(lr[:n]), _t(mask[:n])
+    # the same values one element into a fresh buffer: 4-byte but not 16-byte aligned
+    b_lp = torch.zeros(n + 1, device="cuda")
+    b_lr = torch.zeros(n + 1, device="cuda")
+    b_lp[1:] = a_lp
+    b_lr[1:] = a_lr
+    assert a_lp.data_ptr() % 16 == 0 and b_lp[1:].data_ptr() % 16 == 4
+    for m in (None, a_m):
+        sa, ra = rz.rz_ratio_stats(a_lp, a_lr, off_t, token_mask=m)
+        sb, rb = rz.rz_ratio_stats(b_lp[1:], b_lr[1:], off_t, token_mask=m)
+        assert torch.equal(sa.view(torch.int64), sb.view(torch.int64))
+        assert torch.equal(ra.view(torch.int32), rb.view(torch.int32))
+    st_o, _ = oracle.ratio_stats(lp[:n].astype(np.float64), lr[:n].astype(np.float64), off, mask=None)
+    st = dict(zip(rz.STAT_NAMES, rz.rz_ratio_stats(b_lp[1:], b_lr[1:], off_t)[0].cpu().numpy().tolist()))
+    assert st["count"] == st_o["count"] == n
+    for k in ("k1", "k2", "k3"):
+        assert abs(st[k] - st_o[k]) <= 1e-9 * abs(st_o[k]) + 1e-15, k
+
+
+def test_ratio_stats_k3_far_from_zero(rz, oracle):
+    """|lp - lp_rollout| beyond 1/2 leaves the series for expm1; both ranges against fp64."""
+    rng = np.random.default_rng(9)
+    n = 50_000
+    lp = (-rng.exponential(2.0, n)).astype(np.float32)
+    lr = (lp + rng.choice([-1.5, -0.6, -0.49, 0.3, 0.51, 2.0], n) * rng.uniform(0.5, 1.0, n)).astype(np.float32)
+    off = np.array([0, n // 3, n], np.int64)
+    st_o, _ = oracle.ratio_stats(lp.astype(np.float64), lr.astype(np.float64), off)
+    st = dict(zip(rz.STAT_NAMES, rz.rz_ratio_stats(_t(lp), _t(lr), _t(off))[0].cpu().numpy().tolist()))
+    for k in ("k1", "k2", "k3"):
+        assert abs(st[k] - st_o[k]) <= 1e-9 * abs(st_o[k]) + 1e-15, k
+
+
 def test_grad_norms_match_fp64_norms(rz):
     g = torch.Generator(device="cuda")
     g.manual_seed(3)
