@@ -413,7 +413,9 @@ def run_loss_stage(rz, torch, dev, stream, n_tok=1 << 26, reps=20):
 
 def run_e2e(rz, torch, dev, stream, H, W, ids, lp_roll, rewards, off, gid, G, n, d, V, args):
     """The same step through the public call with inputs in pinned host memory: H2D of every
-    input and D2H of the loss and logprobs inside the timed region."""
+    input and D2H of the loss and logprobs inside the timed region.  W and the small inputs
+    are copied first; H goes through rz_loss_fwd_bwd_streamed, which copies it chunk by chunk
+    on its own stream while the previous chunk computes."""
     host = {k: t.cpu().pin_memory() for k, t in
             dict(H=H, W=W, ids=ids, lp_roll=lp_roll, rewards=rewards, off=off, gid=gid).items()}
     dbuf = {k: torch.empty_like(t, device=dev) for k, t in host.items()}
@@ -428,10 +430,10 @@ def run_e2e(rz, torch, dev, stream, H, W, ids, lp_roll, rewards, off, gid, G, n,
 
     def step():
         for k in host:
-            dbuf[k].copy_(host[k], non_blocking=True)
-        rz.rz_loss_fwd_bwd(dbuf["H"], dbuf["W"], dbuf["ids"], dbuf["lp_roll"], dbuf["rewards"], dbuf["off"],
-                           dbuf["gid"], G, loss=out["loss"], dH=out["dH"], dW=out["dW"], lp_out=out["lp"],
-                           kappa_out=None, want_kappa=False, workspace=ws, stream=stream)
+            if k != "H":
+                dbuf[k].copy_(host[k], non_blocking=True)
+        rz.rz_loss_fwd_bwd_streamed(host["H"], dbuf["H"], dbuf["W"], dbuf["ids"], dbuf["lp_roll"], dbuf["rewards"],
+                                    dbuf["off"], dbuf["gid"], G, out=out, workspace=ws, stream=stream)
         loss_h.copy_(out["loss"], non_blocking=True)
         lp_h.copy_(out["lp"], non_blocking=True)
 

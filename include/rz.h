@@ -180,6 +180,32 @@ rz_status rz_loss_fwd_bwd_ex(const rz_bf16* H, const rz_bf16* W_head, const int3
                              int32_t V, const rz_loss_options* options, float* loss, rz_bf16* dH, float* dW,
                              float* lp_out, float* kappa_out, void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * rz_loss_fwd_bwd_ex with the hidden states read from HOST memory, the copy overlapped with
+ * the compute.  The call enqueues on a copy stream of its own (one per device, created on
+ * first use) one cudaMemcpyAsync per 16384-token chunk of H_host into H_dev, and each
+ * chunk's kernels on `stream` wait for that chunk's copy only, so the copy of chunk c + 1
+ * runs while chunk c computes.  The copies begin after all work already enqueued on
+ * `stream` (which may still be reading H_dev).  With RZ_LOSS_SEQ_GATE the first forward
+ * pass waits for every chunk.
+ *
+ *   H_host  host, [n_tok, d] bf16 row-major; pinned (cudaHostAlloc / cudaHostRegister) for
+ *           the copies to overlap (pageable memory works, without overlap).  Must stay
+ *           unchanged until the call's work on `stream` has finished.
+ *   H_dev   device, [n_tok, d] bf16, 16-byte aligned, caller-owned; on return of the work
+ *           it holds a copy of H_host.
+ *   every other argument as rz_loss_fwd_bwd_ex (device pointers, same workspace size).
+ * Errors: as rz_loss_fwd_bwd_ex, plus RZ_ERR_INVALID_ARG for a null H_host and RZ_ERR_CUDA
+ * when the copy stream, its event or a copy cannot be created or enqueued (nothing of the
+ * compute is enqueued past that point).
+ */
+rz_status rz_loss_fwd_bwd_streamed(const rz_bf16* H_host, rz_bf16* H_dev, const rz_bf16* W_head,
+                                   const int32_t* token_ids, const float* lp_rollout, const float* rewards,
+                                   const int64_t* seg_offsets, const int32_t* group_ids, int64_t n_tok,
+                                   int32_t n_resp, int32_t n_groups, int32_t d, int32_t V,
+                                   const rz_loss_options* options, float* loss, rz_bf16* dH, float* dW,
+                                   float* lp_out, float* kappa_out, void* workspace, size_t ws_bytes, void* stream);
+
 /* rz_segment_loss with loss-stage options (same workspace size). */
 rz_status rz_segment_loss_ex(const float* lp, const float* lp_rollout, const float* rewards,
                              const int64_t* seg_offsets, const int32_t* group_ids, int64_t n_tok, int32_t n_resp,

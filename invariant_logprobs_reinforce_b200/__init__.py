@@ -26,7 +26,8 @@ STATUS_NAMES = {
 EXPORTED_SYMBOLS = (
     "rz_status_string", "rz_workspace_bytes_logprobs", "rz_workspace_bytes_loss", "rz_workspace_bytes_segment_loss",
     "rz_token_logprobs", "rz_loss_fwd_bwd", "rz_segment_loss", "rz_read_device_status", "rz_num_launches_loss",
-    "rz_loss_fwd_bwd_timed", "rz_token_logprobs_noalloc", "rz_loss_fwd_bwd_ex", "rz_segment_loss_ex",
+    "rz_loss_fwd_bwd_timed", "rz_token_logprobs_noalloc", "rz_loss_fwd_bwd_ex", "rz_loss_fwd_bwd_streamed",
+    "rz_segment_loss_ex",
     "rz_workspace_bytes_ratio_stats", "rz_ratio_stats", "rz_workspace_bytes_grad_norms", "rz_grad_norms",
     "rz_quantize_rows_e4m3", "rz_token_logprobs_fp8", "rz_sum_shards_f32", "rz_selftest_wait_timeout",
 )
@@ -99,6 +100,9 @@ def lib() -> ctypes.CDLL:
         L.rz_loss_fwd_bwd_ex.argtypes = [P, P, P, P, P, P, P, i64, i32, i32, i32, i32, ctypes.POINTER(rz_loss_options),
                                           P, P, P, P, P, P, sz, P]
         L.rz_loss_fwd_bwd_ex.restype = ctypes.c_int
+        L.rz_loss_fwd_bwd_streamed.argtypes = [P, P, P, P, P, P, P, P, i64, i32, i32, i32, i32,
+                                                ctypes.POINTER(rz_loss_options), P, P, P, P, P, P, sz, P]
+        L.rz_loss_fwd_bwd_streamed.restype = ctypes.c_int
         L.rz_segment_loss_ex.argtypes = [P, P, P, P, P, i64, i32, i32, ctypes.POINTER(rz_loss_options), P, P, P, P,
                                           sz, P]
         L.rz_segment_loss_ex.restype = ctypes.c_int
@@ -328,6 +332,38 @@ def rz_loss_fwd_bwd_ex(H, W_head, token_ids, lp_rollout, rewards, seg_offsets, g
                                     _ptr(out["dH"]), _ptr(out["dW"]), _ptr(out["lp"]), _ptr(out["kappa"]), _ptr(ws),
                                     ws.numel(), _stream_handle(stream))
     _check(code, "rz_loss_fwd_bwd_ex")
+    out["workspace"] = ws
+    return out
+
+
+def rz_loss_fwd_bwd_streamed(H_host, H_dev, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids, n_groups,
+                             options=None, out=None, workspace=None, stream=None):
+    """rz_loss_fwd_bwd_ex with H read from host memory (H_host: CPU bf16 tensor, pinned for the copies to
+    overlap the compute) into the device buffer H_dev, chunk by chunk.  `out` (the dict this returns) may be
+    passed back in to reuse its buffers.  H_host must stay unchanged until the work on the stream is done."""
+    torch = _torch()
+    _need(H_dev, torch.bfloat16, "H_dev")
+    if H_host.dtype != torch.bfloat16 or H_host.device.type != "cpu" or not H_host.is_contiguous():
+        raise ValueError("H_host must be a contiguous CPU bf16 tensor")
+    if tuple(H_host.shape) != tuple(H_dev.shape):
+        raise ValueError("H_host and H_dev must have the same shape")
+    dev = H_dev.device
+    n, d = H_dev.shape
+    V = W_head.shape[0]
+    R = rewards.shape[0]
+    if out is None:
+        out = dict(loss=torch.empty(1, dtype=torch.float32, device=dev),
+                   dH=torch.empty((n, d), dtype=torch.bfloat16, device=dev),
+                   dW=torch.empty((V, d), dtype=torch.float32, device=dev),
+                   lp=torch.empty(n, dtype=torch.float32, device=dev),
+                   kappa=torch.empty(n, dtype=torch.float32, device=dev))
+    ws = _workspace(rz_workspace_bytes_loss(n, R, n_groups, d, V), workspace, dev)
+    code = lib().rz_loss_fwd_bwd_streamed(_ptr(H_host), _ptr(H_dev), _ptr(W_head), _ptr(token_ids), _ptr(lp_rollout),
+                                          _ptr(rewards), _ptr(seg_offsets), _ptr(group_ids), n, R, n_groups, d, V,
+                                          ctypes.byref(options) if options is not None else None, _ptr(out["loss"]),
+                                          _ptr(out["dH"]), _ptr(out["dW"]), _ptr(out.get("lp")), _ptr(out.get("kappa")),
+                                          _ptr(ws), ws.numel(), _stream_handle(stream))
+    _check(code, "rz_loss_fwd_bwd_streamed")
     out["workspace"] = ws
     return out
 

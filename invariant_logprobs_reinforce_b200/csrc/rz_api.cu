@@ -581,12 +581,73 @@ RZ_API rz_status rz_segment_loss_ex(const float* lp, const float* lp_rollout, co
 }  // extern "C"
 
 namespace {
+// A non-blocking stream per device for host-to-device copies, created on first use.
+cudaStream_t copy_stream_for_current_device() {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static cudaStream_t streams[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (streams[dev] == nullptr && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess)
+    streams[dev] = nullptr;
+  return streams[dev];
+}
+
+// Rows of H streamed from host memory: copies of row ranges go out on the copy stream, in
+// order, each followed by a record of one event; the compute stream waits on the event
+// right after each record is enqueued, so every wait sees the copies enqueued before it.
+struct HostRows {
+  const rz_bf16* host;
+  rz_bf16* dev;
+  int64_t d;
+  cudaStream_t copy = nullptr;
+  cudaEvent_t ev = nullptr;
+  int64_t next = 0;  // first row whose copy is not yet enqueued
+
+  HostRows(const rz_bf16* h, rz_bf16* dv, int64_t cols) : host(h), dev(dv), d(cols) {}
+  HostRows(const HostRows&) = delete;
+  HostRows& operator=(const HostRows&) = delete;
+  ~HostRows() {
+    if (ev != nullptr) cudaEventDestroy(ev);  // released once its pending records complete
+  }
+
+  // The copy stream starts after everything already enqueued on `st` (which may still read
+  // the device buffer).
+  rz_status start(cudaStream_t st) {
+    copy = copy_stream_for_current_device();
+    if (copy == nullptr) return RZ_ERR_CUDA;
+    if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) {
+      ev = nullptr;
+      return RZ_ERR_CUDA;
+    }
+    if (cudaEventRecord(ev, st) != cudaSuccess || cudaStreamWaitEvent(copy, ev, 0) != cudaSuccess)
+      return RZ_ERR_CUDA;
+    return RZ_OK;
+  }
+
+  // Enqueue the copy of rows [next, upto) and record the event after it.
+  rz_status enqueue(int64_t upto) {
+    if (upto <= next) return RZ_OK;
+    const size_t off = static_cast<size_t>(next) * static_cast<size_t>(d);
+    const size_t bytes = static_cast<size_t>(upto - next) * static_cast<size_t>(d) * sizeof(rz_bf16);
+    if (cudaMemcpyAsync(dev + off, host + off, bytes, cudaMemcpyHostToDevice, copy) != cudaSuccess ||
+        cudaEventRecord(ev, copy) != cudaSuccess)
+      return RZ_ERR_CUDA;
+    next = upto;
+    return RZ_OK;
+  }
+
+  // Work enqueued on `st` after this waits for every copy enqueued so far.
+  rz_status wait(cudaStream_t st) { return cudaStreamWaitEvent(st, ev, 0) == cudaSuccess ? RZ_OK : RZ_ERR_CUDA; }
+};
+
 rz_status loss_fwd_bwd_impl(const rz_bf16* H, const rz_bf16* W_head, const int32_t* token_ids,
                           const float* lp_rollout, const float* rewards, const int64_t* seg_offsets,
                           const int32_t* group_ids, int64_t n_tok, int32_t n_resp, int32_t n_groups, int32_t d,
                           int32_t V, const rz_loss_options* options, float* loss, rz_bf16* dH, float* dW,
                           float* lp_out, float* kappa_out, void* workspace, size_t ws_bytes, void* stream,
-                          Recorder* rec) {
+                          Recorder* rec, HostRows* host_rows = nullptr) {
   if (n_tok < 1 || n_tok >= (int64_t{1} << 31) || n_resp < 1 || n_groups < 1) return RZ_ERR_INVALID_ARG;
   LossOpts opt;
   if (!resolve_options(options, n_resp, &opt)) return RZ_ERR_INVALID_ARG;
@@ -608,6 +669,12 @@ rz_status loss_fwd_bwd_impl(const rz_bf16* H, const rz_bf16* W_head, const int32
   float* kappa = kappa_out ? kappa_out : at<float>(workspace, L.kappa);
   rz_status r = run_loss_setup(rewards, seg_offsets, group_ids, n_tok, n_resp, n_groups, opt, workspace, L, st, rec);
   if (r != RZ_OK) return r;
+  if (host_rows != nullptr) {  // the first chunk (every chunk for the gate's first pass)
+    r = host_rows->start(st);
+    if (r == RZ_OK) r = host_rows->enqueue(opt.gate ? n_tok : std::min<int64_t>(kChunkTokens, n_tok));
+    if (r == RZ_OK) r = host_rows->wait(st);
+    if (r != RZ_OK) return r;
+  }
   if (opt.gate) {
     // the gate needs every token's logprob before any kappa: one forward pass first
     // (same kernels, so the same lp bits as the pass that follows)
@@ -623,6 +690,10 @@ rz_status loss_fwd_bwd_impl(const rz_bf16* H, const rz_bf16* W_head, const int32
   // partials are per 4096-token block, so the loss does not depend on the chunking
   for (int64_t c0 = 0; c0 < n_tok; c0 += kChunkTokens) {
     const int64_t rows = std::min<int64_t>(kChunkTokens, n_tok - c0);
+    if (host_rows != nullptr) {  // the next chunk's copy overlaps this chunk's compute
+      r = host_rows->enqueue(std::min<int64_t>(c0 + rows + kChunkTokens, n_tok));
+      if (r != RZ_OK) return r;
+    }
     r = run_forward(H, W_head, token_ids, c0, rows, d, V, lp, lse, workspace, L, true, st, rec);
     if (r != RZ_OK) return r;
     const int blk0 = static_cast<int>(c0 / kKappaBlockTokens);
@@ -632,6 +703,10 @@ rz_status loss_fwd_bwd_impl(const rz_bf16* H, const rz_bf16* W_head, const int32
     if (r != RZ_OK) return r;
     r = run_backward_chunk(H, W_head, token_ids, c0, rows, d, V, lp, lse, kappa, dH, dW, workspace, L, st, rec);
     if (r != RZ_OK) return r;
+    if (host_rows != nullptr && c0 + rows < n_tok) {
+      r = host_rows->wait(st);  // before the next chunk's kernels
+      if (r != RZ_OK) return r;
+    }
   }
   return run_loss_final(n_tok, loss, workspace, L, st, rec);
 }
@@ -659,6 +734,20 @@ RZ_API rz_status rz_loss_fwd_bwd_ex(const rz_bf16* H, const rz_bf16* W_head, con
   return loss_fwd_bwd_impl(H, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids, n_tok, n_resp,
                            n_groups, d, V, options, loss, dH, dW, lp_out, kappa_out, workspace, ws_bytes, stream,
                            nullptr);
+}
+
+RZ_API rz_status rz_loss_fwd_bwd_streamed(const rz_bf16* H_host, rz_bf16* H_dev, const rz_bf16* W_head,
+                                          const int32_t* token_ids, const float* lp_rollout, const float* rewards,
+                                          const int64_t* seg_offsets, const int32_t* group_ids, int64_t n_tok,
+                                          int32_t n_resp, int32_t n_groups, int32_t d, int32_t V,
+                                          const rz_loss_options* options, float* loss, rz_bf16* dH, float* dW,
+                                          float* lp_out, float* kappa_out, void* workspace, size_t ws_bytes,
+                                          void* stream) {
+  if (H_host == nullptr) return RZ_ERR_INVALID_ARG;
+  HostRows rows(H_host, H_dev, d);
+  return loss_fwd_bwd_impl(H_dev, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids, n_tok, n_resp,
+                           n_groups, d, V, options, loss, dH, dW, lp_out, kappa_out, workspace, ws_bytes, stream,
+                           nullptr, &rows);
 }
 
 RZ_API int32_t rz_num_launches_loss(int64_t n_tok) {
@@ -775,11 +864,11 @@ RZ_API rz_status rz_ratio_stats(const float* lp, const float* lp_rollout, const 
   const bool vec = aligned(lp, 16) && aligned(lp_rollout, 16);
   ratio_stats_pass0<<<nb, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, vec, parts, hist);
   ratio_stats_reduce<<<1, 1024, 0, st>>>(parts, nb, acc, sel);
-  ratio_stats_select<<<1, 1024, 0, st>>>(hist, kStatBins, 11, sel, acc, 0, stats_out);
+  ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, kStatBins, 11, sel, acc, 0, stats_out);
   ratio_stats_pass<<<nb, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, vec, sel, 21, 10, 0x7ffu, hist);
-  ratio_stats_select<<<1, 1024, 0, st>>>(hist, kStatBins, 11, sel, acc, 0, stats_out);
+  ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, kStatBins, 11, sel, acc, 0, stats_out);
   ratio_stats_pass<<<nb, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, vec, sel, 10, 0, 0x3ffu, hist);
-  ratio_stats_select<<<1, 1024, 0, st>>>(hist, 1024, 10, sel, acc, 1, stats_out);
+  ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, 1024, 10, sel, acc, 1, stats_out);
   if (resp_mean_ratio_out != nullptr)
     response_mean_ratio_kernel<<<static_cast<unsigned>(ceil_div(n_resp, 8)), 256, 0, st>>>(
         lp, lp_rollout, token_mask, seg_offsets, n_resp, resp_mean_ratio_out);
