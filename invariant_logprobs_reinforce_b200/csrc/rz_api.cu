@@ -243,6 +243,7 @@ rz_status run_forward(const rz_bf16* H, const rz_bf16* W, const int32_t* ids, in
     e.tile_max = at<float>(ws, L.tile_max);
     e.row_scale = nullptr;
     e.col_scale = nullptr;
+    e.col_scale_vec = 0;
     if (launch_gemm<false, false>(mH, mW, s, pos, e, status, stream) != cudaSuccess) return RZ_ERR_CUDA;
   } else {
     EpiLse<false> e;
@@ -258,6 +259,7 @@ rz_status run_forward(const rz_bf16* H, const rz_bf16* W, const int32_t* ids, in
     e.tile_max = nullptr;
     e.row_scale = nullptr;
     e.col_scale = nullptr;
+    e.col_scale_vec = 0;
     if (launch_gemm<false, false>(mH, mW, s, pos, e, status, stream) != cudaSuccess) return RZ_ERR_CUDA;
   }
   rec_end(rec, stream);
@@ -299,6 +301,7 @@ rz_status run_forward_fp8(const uint8_t* H8, const float* hs, const uint8_t* W8,
   e.tile_max = nullptr;
   e.row_scale = hs;
   e.col_scale = wsc;
+  e.col_scale_vec = aligned(wsc, 16) ? 1 : 0;
   auto kernel = gemm_tc_kernel<false, false, EpiLse<false>, true>;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) != cudaSuccess)
     return RZ_ERR_CUDA;

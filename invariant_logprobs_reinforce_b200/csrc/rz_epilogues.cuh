@@ -65,13 +65,16 @@ struct EpiLse {
   int64_t part_ld;
   float* zy;          // [rows] logit of the sampled token
   float* tile_max;    // STORE_P: [rows][n_tiles]
-  const float* row_scale;  // nullable: logit = acc * row_scale[row] * col_scale[col] (scaled fp8 operands)
+  const float* row_scale;  // nullable: logit = row_scale[row] * (acc * col_scale[col]) (scaled fp8 operands)
   const float* col_scale;
+  int col_scale_vec;       // col_scale is 16-byte aligned: read it four columns at a time
 
   struct State {
     float m, s, rs;
     int y;
     int64_t row;
+    float4 cs_next[2];  // scaled operands: this lane's 8 column scales of tile cs_next_tile
+    int cs_next_tile;
   };
 
   __device__ __forceinline__ void begin_unit(State& st, int mb, int, int r) const {
@@ -80,15 +83,59 @@ struct EpiLse {
     st.m = -INFINITY;
     st.s = 0.0f;
     st.rs = (row_scale != nullptr && st.row < rows) ? __ldg(row_scale + st.row) : 1.0f;
+    st.cs_next_tile = -1;
   }
 
-  // scaled operands: z = acc * row_scale * col_scale (one rounding per factor, fixed order)
-  __device__ __forceinline__ void scale_logits(const State& st, int col0, float (&v)[32]) const {
-    if (col_scale == nullptr) return;  // uniform
+  // Lane l's share of tile nt's 256 column scales: columns nt*256 + 8l .. 8l+7 (0 past V).
+  __device__ __forceinline__ void fetch_col_scales(int nt, int lane, float4 (&cs)[2]) const {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const float cs = col0 + j < V ? __ldg(col_scale + col0 + j) : 0.0f;
-      v[j] = (v[j] * st.rs) * cs;
+    for (int h = 0; h < 2; ++h) {
+      const int c = nt * BN + 8 * lane + 4 * h;
+      if (col_scale_vec && c + 3 < V) {
+        cs[h] = __ldg(reinterpret_cast<const float4*>(col_scale + c));
+      } else {
+        cs[h].x = c < V ? __ldg(col_scale + c) : 0.0f;
+        cs[h].y = c + 1 < V ? __ldg(col_scale + c + 1) : 0.0f;
+        cs[h].z = c + 2 < V ? __ldg(col_scale + c + 2) : 0.0f;
+        cs[h].w = c + 3 < V ? __ldg(col_scale + c + 3) : 0.0f;
+      }
+    }
+  }
+
+  // Scaled operands: put tile nt's column scales into the warp's shared buffer (from the
+  // registers filled one tile ahead, else straight from memory) and start fetching tile
+  // nt + 1's, so the global-memory latency of the scales is hidden behind a tile of work.
+  __device__ __forceinline__ void stage_col_scales(State& st, int nt, int lane, float* buf) const {
+    float4 cur[2];
+    if (st.cs_next_tile == nt) {
+      cur[0] = st.cs_next[0];
+      cur[1] = st.cs_next[1];
+    } else {
+      fetch_col_scales(nt, lane, cur);
+    }
+    __syncwarp();  // every lane is done with the previous tile's scales
+    reinterpret_cast<float4*>(buf)[2 * lane] = cur[0];
+    reinterpret_cast<float4*>(buf)[2 * lane + 1] = cur[1];
+    __syncwarp();
+    if (nt + 1 < n_tiles) {
+      fetch_col_scales(nt + 1, lane, st.cs_next);
+      st.cs_next_tile = nt + 1;
+    }
+  }
+
+  // Scaled operands: y = acc * col_scale (one rounding), the scales of the chunk's 32
+  // columns read from the warp's shared buffer (broadcast); the positive row scale is kept
+  // out of the per-logit work (see tile).
+  __device__ __forceinline__ void scale_columns(const float* buf, int c, float (&v)[32]) const {
+    if (col_scale == nullptr) return;  // uniform
+    const float4* cs4 = reinterpret_cast<const float4*>(buf + c * 32);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float4 cs = cs4[q];
+      v[4 * q] *= cs.x;
+      v[4 * q + 1] *= cs.y;
+      v[4 * q + 2] *= cs.z;
+      v[4 * q + 3] *= cs.w;
     }
   }
 
@@ -96,31 +143,38 @@ struct EpiLse {
                                        WarpStage& stage) const {
     // chunks of 32 columns holding at least one column < V (uniform across the warp)
     const int nch = min(BN / 32, (V - nt * BN + 31) / 32);
-    // pass 1: tile maximum over the valid columns
-    float tmax = -INFINITY;
+    // The logits are z = rs * y with y = acc (bf16) or acc * col_scale (fp8) and rs the row
+    // scale (1 for bf16).  rs > 0, so max z = rs * max y exactly, and
+    // exp(z - max z) = 2^((y - max y) * (rs log2 e)); with rs = 1 this is the plain form.
+    const float c2 = st.rs * kLog2e;
+    // scaled operands only (never with STORE_P, whose staging slots the buffer shares)
+    float* cs_buf = reinterpret_cast<float*>(stage.base);
+    if (!STORE_P && col_scale != nullptr) stage_col_scales(st, nt, lane, cs_buf);
+    // pass 1: tile maximum of y over the valid columns
+    float ymax = -INFINITY;
     tmem_for_chunks(taddr, nch, [&](int c, float (&v)[32]) {
       const int col0 = nt * BN + c * 32;
-      scale_logits(st, col0, v);
+      scale_columns(cs_buf, c, v);
 #pragma unroll
       for (int j = 0; j < 32; ++j)
-        if (col0 + j < V) tmax = fmaxf(tmax, v[j]);
+        if (col0 + j < V) ymax = fmaxf(ymax, v[j]);
     });
     // pass 2: exponentials relative to the tile maximum, their sum, the gather
     float tsum = 0.0f;
     tmem_for_chunks(taddr, nch, [&](int c, float (&v)[32]) {
       const int col0 = nt * BN + c * 32;
-      scale_logits(st, col0, v);
+      scale_columns(cs_buf, c, v);
       const unsigned off = static_cast<unsigned>(st.y - col0);
       if (off < 32u) {
         float z = v[0];
 #pragma unroll
         for (int j = 1; j < 32; ++j) z = (static_cast<unsigned>(j) == off) ? v[j] : z;
-        zy[st.row] = z;
+        zy[st.row] = st.rs * z;
       }
       float e[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        e[j] = (col0 + j < V) ? ex2_approx((v[j] - tmax) * kLog2e) : 0.0f;
+        e[j] = (col0 + j < V) ? ex2_approx((v[j] - ymax) * c2) : 0.0f;
         tsum += e[j];
       }
       if constexpr (STORE_P) {
@@ -132,6 +186,7 @@ struct EpiLse {
         stage.store_rows(&p_map, lane, row, col0, mb * BM + (r - lane), rows);
       }
     });
+    const float tmax = st.rs * ymax;
     const float m_new = fmaxf(st.m, tmax);
     st.s = st.s * ex2_approx((st.m - m_new) * kLog2e) + tsum * ex2_approx((tmax - m_new) * kLog2e);
     st.m = m_new;
