@@ -21,6 +21,7 @@ import math
 import os
 import subprocess
 import sys
+import threading
 import time
 
 import numpy as np
@@ -60,6 +61,47 @@ def load_peaks():
 
 
 # --------------------------------------------------------------------------- clocks
+
+class NvmlClock:
+    """Median SM clock over a short timed region: NVML reads every 5 ms from a thread (reads
+    only; nothing is set).  None where NVML is unavailable."""
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.samples = []
+        self._stop = False
+        self._thread = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            handle = pynvml.nvmlDeviceGetHandleByIndex(self.idx)
+        except Exception:
+            return self
+
+        def run():
+            while not self._stop:
+                try:
+                    self.samples.append(pynvml.nvmlDeviceGetClockInfo(handle, pynvml.NVML_CLOCK_SM))
+                except Exception:
+                    return
+                time.sleep(0.005)
+
+        self._thread = threading.Thread(target=run, daemon=True)
+        self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop = True
+        if self._thread is not None:
+            self._thread.join()
+        return False
+
+    @property
+    def sm_mhz(self):
+        return float(np.median(self.samples)) if self.samples else None
+
 
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
@@ -332,7 +374,7 @@ def run_rz(args, rank, world, local_rank):
     )
 
 
-def run_loss_stage(rz, torch, dev, stream, n_tok=1 << 26, reps=20):
+def run_loss_stage(rz, torch, dev, stream, n_tok=1 << 26, reps=200):
     """The loss stage alone (rz_segment_loss) at 2^26 tokens with the moe_head response
     shape (lengths U{256..4096}, groups of 16, Bernoulli(0.5) rewards): HBM-bound, 12
     algorithmic bytes per token (read lp and lp_rollout, write kappa) plus 16 per
@@ -368,47 +410,53 @@ def run_loss_stage(rz, torch, dev, stream, n_tok=1 << 26, reps=20):
         rz.rz_segment_loss(lp, lr, t_r, t_off, t_gid, G, loss=loss, kappa_out=kappa, workspace=ws, stream=stream)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(reps):
-        rz.rz_segment_loss(lp, lr, t_r, t_off, t_gid, G, loss=loss, kappa_out=kappa, workspace=ws, stream=stream)
-    e1.record(stream)
-    torch.cuda.synchronize()
+    with NvmlClock(dev.index if dev.index is not None else 0) as clk:
+        e0.record(stream)
+        for _ in range(reps):
+            rz.rz_segment_loss(lp, lr, t_r, t_off, t_gid, G, loss=loss, kappa_out=kappa, workspace=ws,
+                               stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / reps
     nbytes = 12 * n_tok + 16 * R
     peaks, src = load_peaks()
     gbs = nbytes / (ms * 1e-3) / 1e9
 
-    def timed(fn):
+    def timed(fn, n_rep):
         for _ in range(3):
             fn()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(reps):
-            fn()
-        b.record(stream)
-        torch.cuda.synchronize()
-        return a.elapsed_time(b) / reps
+        with NvmlClock(dev.index if dev.index is not None else 0) as c:
+            a.record(stream)
+            for _ in range(n_rep):
+                fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+        return a.elapsed_time(b) / n_rep, c.sm_mhz
 
     # the truncated-IS + token-mask variant (adds a 1-byte mask read per token)
     mask = (torch.rand(n_tok, generator=g, device=dev) < 0.9).to(torch.uint8)
     opts = rz.loss_options(clip_max=1.05, token_mask=mask)
-    ms_var = timed(lambda: rz.rz_segment_loss_ex(lp, lr, t_r, t_off, t_gid, G, opts, workspace=ws, stream=stream))
+    ms_var, _ = timed(lambda: rz.rz_segment_loss_ex(lp, lr, t_r, t_off, t_gid, G, opts, workspace=ws, stream=stream),
+                      reps)
     var_bytes = 13 * n_tok + 16 * R
     # ratio diagnostics: three passes over lp and lp_rollout (radix select), 8 B/token each
     ws_st = torch.empty(int(rz.lib().rz_workspace_bytes_ratio_stats(n_tok, R)), dtype=torch.uint8, device=dev)
-    ms_st = timed(lambda: rz.rz_ratio_stats(lp, lr, t_off, want_resp_mean=False, workspace=ws_st, stream=stream))
+    ms_st, mhz_st = timed(lambda: rz.rz_ratio_stats(lp, lr, t_off, want_resp_mean=False, workspace=ws_st,
+                                                    stream=stream), reps // 2)
     st_bytes = 3 * 8 * n_tok
     hbm = peaks["hbm_gbs"]
     return {"n_tok": n_tok, "n_resp": R, "n_groups": G, "ms_per_call": ms, "algorithmic_bytes": nbytes,
             "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
             "bound": "hbm", "peak_source": f"hbm_gbs of {src}",
             "note": "whole rz_segment_loss call (coefficients, block starts, kappa, loss); inputs 768 MB > L2",
+            "sm_mhz": clk.sm_mhz,
             "variant_clip_mask": {"ms_per_call": ms_var, "achieved": var_bytes / (ms_var * 1e-3) / 1e9,
                                   "frac": var_bytes / (ms_var * 1e-3) / 1e9 / hbm},
             "ratio_stats": {"ms_per_call": ms_st, "achieved": st_bytes / (ms_st * 1e-3) / 1e9,
                             "frac": st_bytes / (ms_st * 1e-3) / 1e9 / hbm,
-                            "note": "3 radix-select passes, 8 B/token each"}}
+                            "sm_mhz": mhz_st, "note": "3 radix-select passes, 8 B/token each"}}
 
 
 def run_e2e(rz, torch, dev, stream, H, W, ids, lp_roll, rewards, off, gid, G, n, d, V, args):

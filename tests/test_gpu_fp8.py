@@ -44,7 +44,7 @@ def _fp8_problem(rz, p):
 
 
 @pytest.mark.parametrize("shape", [(2, 4, (16, 64), 256, 4096, 101), (3, 3, (20, 90), 128, 5000, 201),
-                                   (1, 2, (1, 3), 384, 7, 202)])
+                                   (1, 2, (1, 3), 384, 7, 202), (2, 3, (10, 40), 256, 3003, 207)])
 def test_fp8_logprobs_against_oracle(rz, oracle, shape):
     g_, gs, lengths, d, V, seed = shape
     p = wl.custom(g_, gs, ("uniform",) + tuple(lengths), d, V, seed)
@@ -55,6 +55,21 @@ def test_fp8_logprobs_against_oracle(rz, oracle, shape):
     lp_o, lse_o = oracle.token_logprobs(Hd, Wd, p.ids)
     assert np.abs(lp.cpu().numpy() - lp_o).max() <= h.LP_ATOL
     assert np.abs(lse.cpu().numpy() - lse_o).max() <= h.LP_ATOL
+
+
+def test_fp8_same_bits_with_unaligned_column_scales(rz):
+    """Column scales at a 4-byte (not 16-byte) aligned address take the scalar loads; the
+    logits and so the logprobs must not change by a bit.  V = 3003 leaves a ragged last tile."""
+    p = wl.custom(2, 3, ("uniform", 10, 40), 256, 3003, 208)
+    dev, H8, hs, W8, ws = _fp8_problem(rz, p)
+    buf = torch.zeros(ws.numel() + 1, dtype=torch.float32, device="cuda")
+    buf[1:] = ws
+    ws_off = buf[1:]
+    assert ws.data_ptr() % 16 == 0 and ws_off.data_ptr() % 16 == 4
+    lp_a, lse_a = rz.rz_token_logprobs_fp8(H8, hs, W8, ws, dev["ids"])
+    lp_b, lse_b = rz.rz_token_logprobs_fp8(H8, hs, W8, ws_off, dev["ids"])
+    assert torch.equal(lp_a.view(torch.int32), lp_b.view(torch.int32))
+    assert torch.equal(lse_a.view(torch.int32), lse_b.view(torch.int32))
 
 
 def test_fp8_zero_head(rz):
