@@ -865,12 +865,19 @@ RZ_API rz_status rz_ratio_stats(const float* lp, const float* lp_rollout, const 
   const int nb = stat_blocks(n_tok);
   StatPartial* acc = at<StatPartial>(workspace, stats_acc_off(n_tok));
   const bool vec = aligned(lp, 16) && aligned(lp_rollout, 16);
-  ratio_stats_pass0<<<nb, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, vec, parts, hist);
+  // pass 0 (arithmetic-heavy, few histogram bins) runs one CTA per token block; the radix
+  // passes run persistent CTAs, a few per SM, that flush their histograms once
+  const int sms = sm_count();
+  if (sms <= 0) return RZ_ERR_CUDA;
+  const int grid = std::min(nb, kStatCtasPerSm * sms);
+  ratio_stats_pass0<<<nb, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, vec, nb, parts, hist);
   ratio_stats_reduce<<<1, 1024, 0, st>>>(parts, nb, acc, sel);
   ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, kStatBins, 11, sel, acc, 0, stats_out);
-  ratio_stats_pass<<<nb, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, vec, sel, 21, 10, 0x7ffu, hist);
+  ratio_stats_pass<<<grid, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, vec, nb, sel, 21, 10, 0x7ffu,
+                                                  hist);
   ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, kStatBins, 11, sel, acc, 0, stats_out);
-  ratio_stats_pass<<<nb, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, vec, sel, 10, 0, 0x3ffu, hist);
+  ratio_stats_pass<<<grid, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, vec, nb, sel, 10, 0, 0x3ffu,
+                                                  hist);
   ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, 1024, 10, sel, acc, 1, stats_out);
   if (resp_mean_ratio_out != nullptr)
     response_mean_ratio_kernel<<<static_cast<unsigned>(ceil_div(n_resp, 8)), 256, 0, st>>>(

@@ -193,7 +193,7 @@ __global__ void block_first_kernel(const int64_t* __restrict__ off, int R, int64
 // finds its first token's response by a short walk and then advances with one compare
 // per token (a boundary can only fall between two consecutive tokens).  Otherwise the
 // block walks the global offsets.
-__global__ void __launch_bounds__(kKappaThreads)
+__global__ void __launch_bounds__(kKappaThreads, 5)
     token_kappa_kernel(const float* __restrict__ lp, const float* __restrict__ lp_roll,
                        const int64_t* __restrict__ off, int R, const float* __restrict__ coef,
                        const int* __restrict__ block_first, int64_t n, int block0, int vec_ok,
@@ -235,11 +235,19 @@ __global__ void __launch_bounds__(kKappaThreads)
 
   double local = 0.0;
   if (staged && full) {
-    int k = 0;  // staged response of the current token
+    // staged response k of the current token, the start of response k + 1 and coef_k in
+    // registers: a token that starts no new response reads no shared memory
+    int k = 0;
+    int next = s_rel[1];
+    float ck = s_coef[0];
 #pragma unroll
     for (int it = 0; it < kKappaIters; ++it) {
       const int tr = wrel + it * 128 + lane * 4;
-      while (s_rel[k + 1] <= tr) ++k;
+      if (next <= tr) {
+        do ++k; while (s_rel[k + 1] <= tr);
+        next = s_rel[k + 1];
+        ck = s_coef[k];
+      }
       const float a4[4] = {la[it].x, la[it].y, la[it].z, la[it].w};
       const float b4[4] = {lb[it].x, lb[it].y, lb[it].z, lb[it].w};
       const uint32_t m4 = mk[it];
@@ -247,9 +255,13 @@ __global__ void __launch_bounds__(kKappaThreads)
       float part = 0.0f;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        if (j > 0 && s_rel[k + 1] <= tr + j) ++k;
+        if (j > 0 && next <= tr + j) {  // responses are non-empty: at most one start per token
+          ++k;
+          next = s_rel[k + 1];
+          ck = s_coef[k];
+        }
         w[j] = ex2_approx((a4[j] - b4[j]) * kLog2e);
-        kv[j] = ((m4 >> (8 * j)) & 0xffu) ? s_coef[k] * fminf(w[j], clip_max) : 0.0f;
+        kv[j] = ((m4 >> (8 * j)) & 0xffu) ? ck * fminf(w[j], clip_max) : 0.0f;
         part += kv[j];
       }
       const int64_t t0 = b0 + tr;
@@ -376,6 +388,7 @@ __global__ void __launch_bounds__(256)
 constexpr int kStatThreads = 256;
 constexpr int kStatTokens = 4096;  // tokens per block
 constexpr int kStatBins = 2048;    // 11 bits per radix pass
+constexpr int kStatCtasPerSm = 4;  // resident CTAs per SM of the persistent passes (register-limited)
 
 struct StatPartial {
   double k1, k2, k3;
@@ -424,9 +437,9 @@ struct StatQuads {
 };
 
 __device__ __forceinline__ void load_stat_quads(const float* __restrict__ lp, const float* __restrict__ lp_roll,
-                                                const uint8_t* __restrict__ mask, int64_t n, bool vec,
+                                                const uint8_t* __restrict__ mask, int64_t n, bool vec, int blk,
                                                 StatQuads& q) {
-  const int64_t b0 = static_cast<int64_t>(blockIdx.x) * kStatTokens;
+  const int64_t b0 = static_cast<int64_t>(blk) * kStatTokens;
 #pragma unroll
   for (int k = 0; k < kStatQuads; ++k) {
     const int64_t t = b0 + 4 * (threadIdx.x + k * kStatThreads);
@@ -447,65 +460,71 @@ __device__ __forceinline__ void load_stat_quads(const float* __restrict__ lp, co
   }
 }
 
+// Both passes loop over the 4096-token blocks blk = blockIdx.x, blockIdx.x + gridDim.x, ...
+// (one block per CTA when the grid covers them all): each block's fp64 partial is computed
+// the same way whichever CTA takes it, so the statistics do not depend on the grid, and a
+// CTA adds its shared histogram into the global one once, at the end (integer counts).
 __global__ void __launch_bounds__(kStatThreads)
     ratio_stats_pass0(const float* __restrict__ lp, const float* __restrict__ lp_roll, const uint8_t* __restrict__ mask,
-                      int64_t n, bool vec, StatPartial* __restrict__ parts, unsigned* __restrict__ hist) {
+                      int64_t n, bool vec, int nblk, StatPartial* __restrict__ parts, unsigned* __restrict__ hist) {
   __shared__ unsigned s_hist[kStatBins];
   __shared__ StatPartial s_part[kStatThreads / 32];
   for (int b = threadIdx.x; b < kStatBins; b += kStatThreads) s_hist[b] = 0u;
-  StatQuads q;
-  load_stat_quads(lp, lp_roll, mask, n, vec, q);
   __syncthreads();
-  double k1 = 0.0, k2 = 0.0, k3 = 0.0;
-  float wmin = INFINITY, wmax = -INFINITY, dmax = 0.0f;
-  int cnt = 0;
+  for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x) {
+    StatQuads q;
+    load_stat_quads(lp, lp_roll, mask, n, vec, blk, q);
+    double k1 = 0.0, k2 = 0.0, k3 = 0.0;
+    float wmin = INFINITY, wmax = -INFINITY, dmax = 0.0f;
+    int cnt = 0;
 #pragma unroll
-  for (int k = 0; k < kStatQuads; ++k) {
+    for (int k = 0; k < kStatQuads; ++k) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const bool on = q.on[k][i];
-      float dev = 0.0f;
-      if (on) {
-        // the KL estimators in fp64 (k3 cancels to second order); min / max / deviation
-        // on the ratio exactly as the loss stage computes it
-        const double x = static_cast<double>(q.a[k][i]) - static_cast<double>(q.b[k][i]);
-        const float w = ratio_of(q.a[k][i], q.b[k][i]);
-        dev = fabsf(w - 1.0f);
-        k1 -= x;
-        k2 += 0.5 * x * x;
-        k3 += expm1_minus_x(x);
-        wmin = fminf(wmin, w);
-        wmax = fmaxf(wmax, w);
-        dmax = fmaxf(dmax, dev);
-        ++cnt;
+      for (int i = 0; i < 4; ++i) {
+        const bool on = q.on[k][i];
+        if (on) {
+          // the KL estimators in fp64 (k3 cancels to second order); min / max / deviation
+          // on the ratio exactly as the loss stage computes it
+          const double x = static_cast<double>(q.a[k][i]) - static_cast<double>(q.b[k][i]);
+          const float w = ratio_of(q.a[k][i], q.b[k][i]);
+          const float dev = fabsf(w - 1.0f);
+          k1 -= x;
+          k2 += 0.5 * x * x;
+          k3 += expm1_minus_x(x);
+          wmin = fminf(wmin, w);
+          wmax = fmaxf(wmax, w);
+          dmax = fmaxf(dmax, dev);
+          ++cnt;
+          hist_add(s_hist, __float_as_uint(dev) >> 21, true);
+        }
       }
-      hist_add(s_hist, __float_as_uint(dev) >> 21, on);
     }
-  }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    k1 += __shfl_xor_sync(0xffffffffu, k1, o);
-    k2 += __shfl_xor_sync(0xffffffffu, k2, o);
-    k3 += __shfl_xor_sync(0xffffffffu, k3, o);
-    wmin = fminf(wmin, __shfl_xor_sync(0xffffffffu, wmin, o));
-    wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, o));
-    dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, o));
-    cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-  }
-  if ((threadIdx.x & 31) == 0) s_part[threadIdx.x >> 5] = StatPartial{k1, k2, k3, wmin, wmax, dmax, cnt};
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    StatPartial acc = s_part[0];
-    for (int w = 1; w < kStatThreads / 32; ++w) {
-      acc.k1 += s_part[w].k1;
-      acc.k2 += s_part[w].k2;
-      acc.k3 += s_part[w].k3;
-      acc.w_min = fminf(acc.w_min, s_part[w].w_min);
-      acc.w_max = fmaxf(acc.w_max, s_part[w].w_max);
-      acc.dev_max = fmaxf(acc.dev_max, s_part[w].dev_max);
-      acc.count += s_part[w].count;
+    for (int o = 16; o > 0; o >>= 1) {
+      k1 += __shfl_xor_sync(0xffffffffu, k1, o);
+      k2 += __shfl_xor_sync(0xffffffffu, k2, o);
+      k3 += __shfl_xor_sync(0xffffffffu, k3, o);
+      wmin = fminf(wmin, __shfl_xor_sync(0xffffffffu, wmin, o));
+      wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, o));
+      dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, o));
+      cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
     }
-    parts[blockIdx.x] = acc;
+    if ((threadIdx.x & 31) == 0) s_part[threadIdx.x >> 5] = StatPartial{k1, k2, k3, wmin, wmax, dmax, cnt};
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      StatPartial acc = s_part[0];
+      for (int w = 1; w < kStatThreads / 32; ++w) {
+        acc.k1 += s_part[w].k1;
+        acc.k2 += s_part[w].k2;
+        acc.k3 += s_part[w].k3;
+        acc.w_min = fminf(acc.w_min, s_part[w].w_min);
+        acc.w_max = fmaxf(acc.w_max, s_part[w].w_max);
+        acc.dev_max = fmaxf(acc.dev_max, s_part[w].dev_max);
+        acc.count += s_part[w].count;
+      }
+      parts[blk] = acc;
+    }
+    __syncthreads();  // s_part is rewritten by the next block
   }
   for (int b = threadIdx.x; b < kStatBins; b += kStatThreads)
     if (s_hist[b]) atomicAdd(&hist[b], s_hist[b]);
@@ -514,25 +533,24 @@ __global__ void __launch_bounds__(kStatThreads)
 // Histogram of the next radix digit among the deviations whose higher bits equal `prefix`.
 __global__ void __launch_bounds__(kStatThreads)
     ratio_stats_pass(const float* __restrict__ lp, const float* __restrict__ lp_roll, const uint8_t* __restrict__ mask,
-                     int64_t n, bool vec, const unsigned* __restrict__ sel, int shift_hi, int shift,
+                     int64_t n, bool vec, int nblk, const unsigned* __restrict__ sel, int shift_hi, int shift,
                      unsigned digit_mask, unsigned* __restrict__ hist) {
   __shared__ unsigned s_hist[kStatBins];
   for (int b = threadIdx.x; b < kStatBins; b += kStatThreads) s_hist[b] = 0u;
-  StatQuads q;
-  load_stat_quads(lp, lp_roll, mask, n, vec, q);
   const unsigned prefix = sel[0];
   __syncthreads();
+  for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x) {
+    StatQuads q;
+    load_stat_quads(lp, lp_roll, mask, n, vec, blk, q);
 #pragma unroll
-  for (int k = 0; k < kStatQuads; ++k) {
+    for (int k = 0; k < kStatQuads; ++k) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      bool on = q.on[k][i];
-      unsigned key = 0u;
-      if (on) {
-        key = __float_as_uint(fabsf(ratio_of(q.a[k][i], q.b[k][i]) - 1.0f));
-        on = (key >> shift_hi) == prefix;
+      for (int i = 0; i < 4; ++i) {
+        if (q.on[k][i]) {
+          const unsigned key = __float_as_uint(fabsf(ratio_of(q.a[k][i], q.b[k][i]) - 1.0f));
+          if ((key >> shift_hi) == prefix) hist_add(s_hist, (key >> shift) & digit_mask, true);
+        }
       }
-      hist_add(s_hist, (key >> shift) & digit_mask, on);
     }
   }
   __syncthreads();
