@@ -324,6 +324,8 @@ def run_rz(args, rank, world, local_rank):
     f1.record(stream)
     torch.cuda.synchronize()
     fwd_ms = f0.elapsed_time(f1) / fsteps
+    if dist:
+        fwd_ms = max_over_ranks(fwd_ms, dev)
 
     # forward from e4m3 operands (quantised once, outside the timed region)
     H8, hs8 = rz.rz_quantize_rows_e4m3(H)
@@ -337,6 +339,8 @@ def run_rz(args, rank, world, local_rank):
     f1.record(stream)
     torch.cuda.synchronize()
     fwd8_ms = f0.elapsed_time(f1) / fsteps
+    if dist:
+        fwd8_ms = max_over_ranks(fwd8_ms, dev)
     del H8, W8
 
     loss_stage = None
@@ -345,7 +349,7 @@ def run_rz(args, rank, world, local_rank):
 
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(rz, torch, dev, stream, H, W, ids, lp_roll, rewards, off, gid, G, n, d, V, args)
+        e2e = run_e2e(rz, torch, dev, stream, H, W, ids, lp_roll, rewards, off, gid, G, n, d, V, args, world)
 
     peaks, peak_src = load_peaks()
     peak_tflops = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
@@ -459,7 +463,7 @@ def run_loss_stage(rz, torch, dev, stream, n_tok=1 << 26, reps=200):
                             "sm_mhz": mhz_st, "note": "3 radix-select passes, 8 B/token each"}}
 
 
-def run_e2e(rz, torch, dev, stream, H, W, ids, lp_roll, rewards, off, gid, G, n, d, V, args):
+def run_e2e(rz, torch, dev, stream, H, W, ids, lp_roll, rewards, off, gid, G, n, d, V, args, world=1):
     """The same step through the public call with inputs in pinned host memory: H2D of every
     input and D2H of the loss and logprobs inside the timed region.  W and the small inputs
     are copied first; H goes through rz_loss_fwd_bwd_streamed, which copies it chunk by chunk
@@ -497,10 +501,12 @@ def run_e2e(rz, torch, dev, stream, H, W, ids, lp_roll, rewards, off, gid, G, n,
     e1.record(stream)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = loss_h.numel() * 4 + lp_h.numel() * 4
-    return {"value": n / (ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "ms_per_step": ms}
+    if world > 1:  # every rank copies its own inputs: the job's time is the slowest rank's
+        ms = max_over_ranks(ms, dev)
+    h2d = world * sum(t.numel() * t.element_size() for t in host.values())
+    d2h = world * (loss_h.numel() * 4 + lp_h.numel() * 4)
+    return {"value": world * n / (ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": ms, "bytes_note": "summed over all ranks"}
 
 
 # --------------------------------------------------------------------------- sweep
