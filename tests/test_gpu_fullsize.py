@@ -1,5 +1,8 @@
-"""Parity at the full Qwen3-4B-shaped workload, in the launch configuration bench.py
-times (d=2560, V=151936, 512 responses, ~360k tokens, 23 backward chunks).
+"""Parity at full size, in the launch configuration bench.py times: the Qwen3-4B-shaped
+workload (d=2560, V=151936, 512 responses, ~360k tokens, 23 backward chunks), the lag-64
+agentic workload (the same head, 256 responses of 1K-16K tokens, ~1.4M tokens, heavy-tailed
+Student-t lag) and the MoE-shaped head (d=7168, V=129280) at 2^20 tokens, the largest call
+of its throughput sweep.
 
 The oracle cannot recompute all of it in fp64, so it checks sampled outputs one by one
 (lp, lse, kappa and dH of sampled token rows) and the rest through properties that hold
@@ -27,8 +30,9 @@ def rz():
     return rz
 
 
-def test_qwen3_4b_full_size_sampled_rows(rz, oracle):
-    prob = wl.full_config("qwen3_4b", device="cuda")
+@pytest.mark.parametrize("name,cap", [("qwen3_4b", None), ("lag64", None), ("moe_head", 1 << 20)])
+def test_full_size_sampled_rows(rz, oracle, name, cap):
+    prob = wl.full_config(name, device="cuda", n_tok_cap=cap)
     seg = prob.seg
     n, d, V = prob.n_tok, prob.d, prob.V
     lp0, lse0 = rz.rz_token_logprobs(prob.H, prob.W, prob.ids)
@@ -73,3 +77,5 @@ def test_qwen3_4b_full_size_sampled_rows(rz, oracle):
     colabs = dW.double().abs().sum(dim=0)
     assert torch.all(colsum <= 1e-2 * colabs)
     assert torch.isfinite(dW).all() and torch.isfinite(out["dH"].float()).all()
+    del out, dW, lp0, lse0, prob
+    torch.cuda.empty_cache()
