@@ -252,10 +252,13 @@ rz_status rz_grad_norms(const rz_bf16* dH, const float* dW, int64_t n_tok, int32
  *   rz_quantize_rows_e4m3: X [rows, d] bf16 -> X8 [rows, d] e4m3 bytes and scale [rows] fp32,
  *     scale = max|x| / 448 (1 for an all-zero row), X8 = e4m3(x / scale), round to nearest
  *     even, saturating (both divisions IEEE fp32).
- *   rz_token_logprobs_fp8: z[t,v] = (sum_k H8[t,k] W8[v,k]) * h_scale[t] * w_scale[v]
- *     (e4m3 x e4m3 products accumulated in fp32 on the tensor cores, then the two scales
- *     applied in that order); lp, lse as rz_token_logprobs.  d must be a multiple of 128;
- *     workspace size = rz_workspace_bytes_logprobs(n_tok, d, V).
+ *   rz_token_logprobs_fp8: z[t,v] = h_scale[t] * y[t,v], y[t,v] = (sum_k H8[t,k] W8[v,k]) *
+ *     w_scale[v] (e4m3 x e4m3 products accumulated in fp32 on the tensor cores, then the
+ *     column scale, one fp32 rounding); the row scale (positive) enters the log-sum-exp as
+ *     exp(z - max z) = 2^((y - max y) * h_scale[t] * log2 e), and lp = h_scale[t] * y[t,y_t] - lse;
+ *     lse as rz_token_logprobs.  d must be a multiple of 128; w_scale needs 4-byte
+ *     alignment (16 bytes for the fastest loads); workspace size =
+ *     rz_workspace_bytes_logprobs(n_tok, d, V).
  */
 rz_status rz_quantize_rows_e4m3(const rz_bf16* X, int64_t rows, int32_t d, uint8_t* X8, float* scale, void* stream);
 rz_status rz_token_logprobs_fp8(const uint8_t* H8, const float* h_scale, const uint8_t* W8, const float* w_scale,
