@@ -197,8 +197,34 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmSc
   return cudaGetLastError();
 }
 
+// L2 eviction policies of the operand loads, from the operands' sizes and reuse (L2 126 MB):
+//  - an operand re-read by every wave of tiles stays (evict-last) while it fits in what
+//    the streams leave of L2: the forward's group of H row blocks, dW's chunk of H;
+//  - a streamed operand read by the output tiles of its row block side by side goes first
+//    (evict-first) while those tiles are few (d <= 12 x 256): dZ in dH and dW; with more
+//    consumers its lines must survive until the last of them has read them;
+//  - W in the forward-only call goes first (nothing else streams through L2 there).
+constexpr uint64_t kL2KeepBytes = 96ull << 20;
+constexpr int kFewConsumerTiles = 12;
+
+int keep_if_fits(uint64_t bytes) { return bytes <= kL2KeepBytes ? kL2EvictLast : kL2Normal; }
+
+// Row blocks per L2 group of the forward: the largest power of two up to 32 whose H rows
+// (128 per block, d elements of elem_bytes) take at most 24 MB, so the group stays in L2
+// beside the W tiles in flight and the stored exponentials (32 at d = 2560, 8 at d = 7168).
+// It only orders the units; no row's arithmetic depends on it.
+int forward_group_m(int32_t d, int elem_bytes) {
+  const uint64_t block_bytes = static_cast<uint64_t>(BM) * d * elem_bytes;
+  int g = 32;
+  while (g > 1 && g * block_bytes > (24ull << 20)) g >>= 1;
+  return g;
+}
+int first_if_few(int consumer_tiles) { return consumer_tiles <= kFewConsumerTiles ? kL2EvictFirst : kL2Normal; }
+
 GemmSched make_sched(int64_t m_rows, int64_t n_cols, int tiles_per_unit, int group_m, int64_t k) {
   GemmSched s;
+  s.l2_pol_a = kL2Normal;
+  s.l2_pol_b = kL2Normal;
   s.m_blocks = static_cast<int>(ceil_div(m_rows, BM));
   s.n_tiles = static_cast<int>(ceil_div(n_cols, BN));
   s.tiles_per_unit = tiles_per_unit;
@@ -221,7 +247,9 @@ rz_status run_forward(const rz_bf16* H, const rz_bf16* W, const int32_t* ids, in
   // rows past the range read as zeros, so no other rows' data enters the launch
   if (!make_operand_map(&mH, H, d, r0 + rows, static_cast<uint64_t>(d) * 2, BM)) return RZ_ERR_CUDA;
   if (!make_operand_map(&mW, W, d, V, static_cast<uint64_t>(d) * 2, BN)) return RZ_ERR_CUDA;
-  const GemmSched s = make_sched(rows, V, kSegTiles, 32, d);
+  GemmSched s = make_sched(rows, V, kSegTiles, forward_group_m(d, 2), d);
+  s.l2_pol_a = keep_if_fits(static_cast<uint64_t>(std::min<int64_t>(s.group_m * BM, rows)) * d * 2);
+  s.l2_pol_b = store_p ? kL2Normal : kL2EvictFirst;
   const OperandPos pos{static_cast<int>(r0), 0, 0, 0};
   float* part_m = at<float>(ws, L.part_m);
   float* part_s = at<float>(ws, L.part_s);
@@ -285,8 +313,10 @@ rz_status run_forward_fp8(const uint8_t* H8, const float* hs, const uint8_t* W8,
   if (!make_map(&mW, CU_TENSOR_MAP_DATA_TYPE_UINT8, W8, d, V, static_cast<uint64_t>(d), BK_FP8, BN,
                 CU_TENSOR_MAP_SWIZZLE_128B))
     return RZ_ERR_CUDA;
-  GemmSched s = make_sched(n, V, kSegTiles, 32, d);
+  GemmSched s = make_sched(n, V, kSegTiles, forward_group_m(d, 1), d);
   s.num_kb = static_cast<int>(ceil_div(d, BK_FP8));
+  s.l2_pol_a = keep_if_fits(static_cast<uint64_t>(std::min<int64_t>(s.group_m * BM, n)) * d);  // e4m3
+  s.l2_pol_b = kL2EvictFirst;
   const OperandPos pos{0, 0, 0, 0};
   EpiLse<false> e;
   std::memset(&e.p_map, 0, sizeof(e.p_map));
@@ -462,7 +492,8 @@ rz_status run_backward_chunk(const rz_bf16* H, const rz_bf16* W, const int32_t* 
       return RZ_ERR_CUDA;
     e.out_cols = d;
     e.out_rows = rows;
-    const GemmSched s = make_sched(rows, d, 1, 1, V);
+    GemmSched s = make_sched(rows, d, 1, 1, V);
+    s.l2_pol_a = first_if_few(s.n_tiles);  // dZ rows, read by the row block's d/256 tiles
     const OperandPos pos{0, 0, 0, 0};
     rec_begin(rec, RZ_KERNEL_DH, stream);
     if (launch_gemm<false, true>(mDzK, mWmn, s, pos, e, status, stream) != cudaSuccess) return RZ_ERR_CUDA;
@@ -480,7 +511,9 @@ rz_status run_backward_chunk(const rz_bf16* H, const rz_bf16* W, const int32_t* 
     e.out_cols = d;
     e.out_rows = V;
     e.accumulate = c0 > 0 ? 1 : 0;
-    const GemmSched s = make_sched(V, d, 1, 1, rows);
+    GemmSched s = make_sched(V, d, 1, 1, rows);
+    s.l2_pol_a = first_if_few(s.n_tiles);                                    // dZ^T
+    s.l2_pol_b = keep_if_fits(static_cast<uint64_t>(rows) * d * 2);          // the chunk's H
     const OperandPos pos{0, 0, 0, static_cast<int>(c0)};
     rec_begin(rec, RZ_KERNEL_DW, stream);
     if (launch_gemm<true, true>(mDzMn, mHmn, s, pos, e, status, stream) != cudaSuccess) return RZ_ERR_CUDA;

@@ -51,10 +51,6 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
 // arithmetic is the same code either way, so both variants give the same lse bits.
 template <bool STORE_P>
 struct EpiLse {
-  // A = H rows: the 32 row blocks of an L2 group are re-read by every vocabulary unit of
-  // the group, so they stay.  B = W tiles are shared by the group's CTAs in flight; with
-  // nothing else streaming through L2 they go first, making room for the H block.
-  static constexpr int kL2PolicyA = kL2EvictLast, kL2PolicyB = STORE_P ? kL2Normal : kL2EvictFirst;
   CUtensorMap p_map;  // STORE_P: fp16 [rows, V] (box 32 x 32, 64-byte swizzle)
   const int32_t* ids; // launch-relative
   int64_t rows;       // rows in this launch
@@ -205,9 +201,6 @@ struct EpiLse {
 
 // dH tile: fp32 accumulator -> bf16, TMA-stored into a [rows, d] map of the chunk.
 struct EpiDh {
-  // A = dZ rows stream through once (the 10 output tiles of a row block run side by side);
-  // letting them go first keeps the W tiles that the next wave of row blocks re-reads.
-  static constexpr int kL2PolicyA = kL2EvictFirst, kL2PolicyB = kL2Normal;
   CUtensorMap out_map;  // bf16 [rows, d], box 32 x 32, 64-byte swizzle
 
   struct State {};
@@ -238,9 +231,6 @@ struct EpiDh {
 // in chunk order) into the [V, d] fp32 map; every element gets exactly one store or add
 // per chunk, so the result is deterministic.
 struct EpiDw {
-  // A = dZ^T streams through once; B = the chunk's H (16384 x d bf16, 84 MB at d = 2560)
-  // is re-read by every wave of vocabulary blocks and fits in L2, so it stays.
-  static constexpr int kL2PolicyA = kL2EvictFirst, kL2PolicyB = kL2EvictLast;
   CUtensorMap out_map;  // fp32 [V, d], box 16 x 32, 64-byte swizzle
   int out_cols;
   int64_t out_rows;

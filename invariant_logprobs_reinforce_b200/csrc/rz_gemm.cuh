@@ -50,6 +50,8 @@ struct GemmSched {
   int group_m;         // units are ordered in groups of group_m row blocks (L2 locality)
   int num_units;       // m_blocks * units_n
   int num_kb;          // 64-wide K blocks per tile
+  int l2_pol_a;        // L2 eviction policy (L2Policy) of the A and B operand loads,
+  int l2_pol_b;        // chosen on the host from the operands' sizes and reuse
 
   // unit index -> (row block, N-unit).  Inside a group of group_m row blocks the row
   // block varies fastest; group_m = 1 gives row-block-major order with N fastest.
@@ -187,8 +189,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      const uint64_t pol_a = make_l2_policy<Epi::kL2PolicyA>();
-      const uint64_t pol_b = make_l2_policy<Epi::kL2PolicyB>();
+      const uint64_t pol_a = make_l2_policy_rt(sched.l2_pol_a);
+      const uint64_t pol_b = make_l2_policy_rt(sched.l2_pol_b);
       int issued_phase[kStages];
 #pragma unroll
       for (int s = 0; s < kStages; ++s) issued_phase[s] = -1;

@@ -99,6 +99,13 @@ __device__ __forceinline__ uint64_t make_l2_policy() {
   return p;
 }
 
+// The policy for a run-time choice (an L2Policy value).
+__device__ __forceinline__ uint64_t make_l2_policy_rt(int pol) {
+  if (pol == kL2EvictFirst) return make_l2_policy<kL2EvictFirst>();
+  if (pol == kL2EvictLast) return make_l2_policy<kL2EvictLast>();
+  return make_l2_policy<kL2Normal>();
+}
+
 // 2D tiled load of one box into shared memory, completing on `bar` (transaction bytes),
 // with the L2 policy `pol` (from make_l2_policy) on the lines it reads.
 __device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* bar, void* dst, int32_t x,
