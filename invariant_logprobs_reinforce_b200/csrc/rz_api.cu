@@ -221,6 +221,16 @@ int forward_group_m(int32_t d, int elem_bytes) {
 }
 int first_if_few(int consumer_tiles) { return consumer_tiles <= kFewConsumerTiles ? kL2EvictFirst : kL2Normal; }
 
+// Backward contractions with more than kFewConsumerTiles output tiles per row block (d >
+// 3072) run their N tiles in balanced groups of at most that many: a wave then streams
+// only its group's slice of W (dH) or H (dW), and a dZ row block has only the group's
+// tiles as consumers, at the price of reading dZ once per group.
+int backward_group_n(int n_tiles) {
+  if (n_tiles <= kFewConsumerTiles) return n_tiles;
+  const int groups = (n_tiles + kFewConsumerTiles - 1) / kFewConsumerTiles;
+  return (n_tiles + groups - 1) / groups;
+}
+
 GemmSched make_sched(int64_t m_rows, int64_t n_cols, int tiles_per_unit, int group_m, int64_t k) {
   GemmSched s;
   s.l2_pol_a = kL2Normal;
@@ -230,6 +240,7 @@ GemmSched make_sched(int64_t m_rows, int64_t n_cols, int tiles_per_unit, int gro
   s.tiles_per_unit = tiles_per_unit;
   s.units_n = static_cast<int>(ceil_div(s.n_tiles, tiles_per_unit));
   s.group_m = std::max(1, std::min(group_m, s.m_blocks));
+  s.group_n = s.units_n;
   s.num_units = s.m_blocks * s.units_n;
   s.num_kb = static_cast<int>(ceil_div(k, BK));
   return s;
@@ -493,7 +504,8 @@ rz_status run_backward_chunk(const rz_bf16* H, const rz_bf16* W, const int32_t* 
     e.out_cols = d;
     e.out_rows = rows;
     GemmSched s = make_sched(rows, d, 1, 1, V);
-    s.l2_pol_a = first_if_few(s.n_tiles);  // dZ rows, read by the row block's d/256 tiles
+    s.group_n = backward_group_n(s.n_tiles);
+    s.l2_pol_a = first_if_few(s.group_n);  // dZ rows, read by the group's tiles of the row block
     const OperandPos pos{0, 0, 0, 0};
     rec_begin(rec, RZ_KERNEL_DH, stream);
     if (launch_gemm<false, true>(mDzK, mWmn, s, pos, e, status, stream) != cudaSuccess) return RZ_ERR_CUDA;
@@ -512,8 +524,10 @@ rz_status run_backward_chunk(const rz_bf16* H, const rz_bf16* W, const int32_t* 
     e.out_rows = V;
     e.accumulate = c0 > 0 ? 1 : 0;
     GemmSched s = make_sched(V, d, 1, 1, rows);
-    s.l2_pol_a = first_if_few(s.n_tiles);                                    // dZ^T
-    s.l2_pol_b = keep_if_fits(static_cast<uint64_t>(rows) * d * 2);          // the chunk's H
+    s.group_n = backward_group_n(s.n_tiles);
+    s.l2_pol_a = first_if_few(s.group_n);  // dZ^T
+    // the group's columns of the chunk's H
+    s.l2_pol_b = keep_if_fits(static_cast<uint64_t>(rows) * std::min<int64_t>(d, s.group_n * BN) * 2);
     const OperandPos pos{0, 0, 0, static_cast<int>(c0)};
     rec_begin(rec, RZ_KERNEL_DW, stream);
     if (launch_gemm<true, true>(mDzMn, mHmn, s, pos, e, status, stream) != cudaSuccess) return RZ_ERR_CUDA;

@@ -48,14 +48,34 @@ struct GemmSched {
   int tiles_per_unit;  // consecutive N tiles processed by one unit
   int units_n;         // ceil(n_tiles / tiles_per_unit)
   int group_m;         // units are ordered in groups of group_m row blocks (L2 locality)
+  int group_n;         // with group_m = 1: groups of group_n N-units, each over all row
+                       // blocks before the next (group_n >= units_n: no N grouping)
   int num_units;       // m_blocks * units_n
   int num_kb;          // 64-wide K blocks per tile
   int l2_pol_a;        // L2 eviction policy (L2Policy) of the A and B operand loads,
   int l2_pol_b;        // chosen on the host from the operands' sizes and reuse
 
   // unit index -> (row block, N-unit).  Inside a group of group_m row blocks the row
-  // block varies fastest; group_m = 1 gives row-block-major order with N fastest.
+  // block varies fastest; group_m = 1 gives row-block-major order with N fastest, and
+  // with group_n < units_n that order runs group by group over the N-units (the last
+  // group holds the remainder).  Either way a bijection onto all units.
   __device__ __forceinline__ void unit_coords(int u, int& mb, int& nu) const {
+    if (group_m == 1 && group_n < units_n) {
+      const int full = units_n / group_n;   // groups of exactly group_n N-units
+      const int span = m_blocks * group_n;  // units per full group
+      const int g = u / span;
+      if (g < full) {
+        const int r = u - g * span;
+        mb = r / group_n;
+        nu = g * group_n + (r - mb * group_n);
+      } else {
+        const int rem = units_n - full * group_n;  // > 0 here: u < num_units
+        const int r = u - full * span;
+        mb = r / rem;
+        nu = full * group_n + (r - mb * rem);
+      }
+      return;
+    }
     const int per_group = group_m * units_n;
     const int g = u / per_group;
     const int r = u - g * per_group;
