@@ -2,11 +2,17 @@
 // TMA descriptor creation and the launch sequence of each entry point.
 //
 // Launch sequence of rz_loss_fwd_bwd (all on the caller's stream, no host sync):
-//   1. forward  : fused LM head + online log-sum-exp per (128-row block, 2048-column
-//                 vocabulary segment) -> per-segment partials; merge -> lp, lse
-//   2. loss     : per-response coefficient -A_i/(N L_i); per-token kappa and ratio; loss
-//   3. backward : for each chunk of 16384 tokens, in order:
-//                 dZ chunk (recomputed logits, bf16)  ->  dH rows = dZ W  ->  dW (+)= dZ^T H
+//   1. loss setup : group sums, per-response coefficients -A_i/(N L_i), block starts
+//   2. for each chunk of 16384 tokens, in order:
+//        forward  : fused LM head + online log-sum-exp per (128-row block, 2048-column
+//                   vocabulary segment), keeping e = exp(z - tile max) (fp16); merge -> lp, lse
+//        kappa    : per-token ratio and kappa, per-4096-token loss partials
+//        dZ       : kappa (onehot - e exp(tile max - lse)) as bf16, in place of e
+//        backward : dH rows = dZ W;  dW (+)= dZ^T H
+//   3. loss       : fixed-order sum of the partials
+// With the sequence gate a forward pass over every chunk runs first (the gate needs all
+// logprobs); rz_loss_fwd_bwd_streamed copies each chunk's rows of H from host memory on a
+// copy stream one chunk ahead.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -199,10 +205,12 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmSc
 
 // L2 eviction policies of the operand loads, from the operands' sizes and reuse (L2 126 MB):
 //  - an operand re-read by every wave of tiles stays (evict-last) while it fits in what
-//    the streams leave of L2: the forward's group of H row blocks, dW's chunk of H;
+//    the streams leave of L2: the forward's group of H row blocks, the columns of dW's
+//    chunk of H that one group of output tiles reads;
 //  - a streamed operand read by the output tiles of its row block side by side goes first
-//    (evict-first) while those tiles are few (d <= 12 x 256): dZ in dH and dW; with more
-//    consumers its lines must survive until the last of them has read them;
+//    (evict-first) while those tiles are few (at most 12; larger d runs its tiles in groups
+//    of at most 12, see backward_group_n): dZ in dH and dW; with more consumers its lines
+//    must survive until the last of them has read them;
 //  - W in the forward-only call goes first (nothing else streams through L2 there).
 constexpr uint64_t kL2KeepBytes = 96ull << 20;
 constexpr int kFewConsumerTiles = 12;

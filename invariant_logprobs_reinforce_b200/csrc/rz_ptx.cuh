@@ -1,5 +1,6 @@
-// rz_ptx.cuh -- thin inline-PTX wrappers for sm_100a: mbarriers, TMA tile loads,
-// tcgen05 (TMEM allocation, UMMA issue/commit, TMEM loads) and bounded waits.
+// rz_ptx.cuh -- thin inline-PTX wrappers for sm_100a: mbarriers, TMA tile loads (with L2
+// eviction policies), stores and reduce-adds, tcgen05 (TMEM allocation, UMMA issue/commit,
+// TMEM loads) and bounded waits.  No TMA operation here uses cluster multicast.
 //
 // Every wait in this library goes through mbar_wait(), which gives up after a
 // wall-clock limit (or when the CTA's abort flag is raised) instead of spinning

@@ -6,6 +6,19 @@
 //   token_kappa_kernel      unclipped ratio and kappa per token, per-block loss partials
 //   loss_final_kernel       fixed-order sum of the partials
 //   dz_from_p_kernel        dZ = kappa (onehot - softmax) from the forward's exponentials
+//   masked_count_kernel, gate_kernel
+//                           loss-stage options: counted tokens per response under a token
+//                           mask; the sequence gate on the geometric-mean ratio
+//   ratio_stats_*, response_mean_ratio_kernel
+//                           ratio diagnostics: KL estimators, min / max / deviation peak and
+//                           exact lower median (radix select), per-response mean ratio
+//   sumsq_kernel, sqrt_sum_kernel
+//                           gradient norms (fixed-order fp64 reductions)
+//   quantize_rows_e4m3_kernel
+//                           per-row e4m3 codes and scales for the fp8 forward
+//   sum_shards_kernel       rank-order sum of stacked shards (deterministic all-reduce)
+//   wait_timeout_selftest_kernel
+//                           the bounded mbarrier wait on a barrier nothing arrives on
 //
 // Definitions follow "vLLM says aligned kernels make asynchronous RL stable at lag 64"
 // (ainewsbites.com), section "REINFORCE Zero removes the mismatch first"; the fixed
