@@ -608,8 +608,21 @@ def cpu_oracle_sample(workload: str, budget_s: float = 15.0):
     k2 = int(max(2, min(512, 2 * round(0.5 * k * budget_s / max(t, 1e-3)))))
     t2 = run(k2)
     return {"value": k2 / t2, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "cpu_model": host_cpu_model(), "host_cpus": os.cpu_count(),
             "sample": f"{k2} tokens of {workload} (2 responses x {k2 // 2} tokens, d={d}, V={V}): "
                       f"fp64 lp, loss, dH and dW; {t2:.1f} s"}
+
+
+def host_cpu_model() -> str:
+    """The host CPU's model name (/proc/cpuinfo), or "unknown"."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def run_reference(args, rank, world):
