@@ -20,6 +20,7 @@ CASES = {
     "single_token": (1, 1, ("uniform", 1, 1), 256, 300, 204),
     "two_chunks": (2, 4, ("uniform", 2100, 2300), 64, 300, 205),
     "wide_d": (2, 2, ("uniform", 40, 70), 1600, 2100, 206),
+    "max_d": (1, 2, ("uniform", 30, 60), 32768, 600, 210),  # the largest d the library accepts
 }
 
 
