@@ -24,9 +24,29 @@ CASES = {
 }
 
 
+# exact response lengths at the backward's 16384-token chunk boundary: one full chunk, and
+# a full chunk plus a one-token chunk (one row in a 128-row tile; dW with K = 1)
+FIXED = {
+    "chunk_exact": ([8000, 8384], 64, 300, 211),
+    "chunk_plus_one": ([8000, 8385], 64, 300, 212),
+}
+CASES.update({k: None for k in FIXED})
+
+
+def _fixed_problem(lengths, d, V, seed):
+    off = np.zeros(len(lengths) + 1, np.int64)
+    off[1:] = np.cumsum(lengths)
+    n = int(off[-1])
+    seg = wl.Segments(off, np.zeros(len(lengths), np.int32), np.array([1.0, 0.0], np.float32), 1)
+    H, W = wl.draw_matrices(n, d, V, seed)
+    return wl.Problem(H, W, wl.draw_uniform_ids(n, V, seed), seg, d, V, ("normal", 0.05), seed)
+
+
 def _problem(name):
     if name == "tiny":
         return wl.tiny()
+    if name in FIXED:
+        return _fixed_problem(*FIXED[name])
     g, gs, lengths, d, V, seed = CASES[name]
     return wl.custom(g, gs, lengths, d, V, seed)
 
