@@ -104,3 +104,39 @@ def test_host_argument_checks_loss(rz):
     lib2 = rz.lib()
     assert lib2.rz_segment_loss(256, 512, 768, 1024, 1280, 10, 0, 1, 1536, 1792, None, 1 << 20, 1 << 40, None) == 1
     assert lib2.rz_segment_loss(256, 512, 768, 1024, 1280, 10, 2, 1, 1536, 1792, None, 1 << 20, 10, None) == 3
+
+
+def test_binding_fails_loudly_without_the_native_library():
+    """No fallback: with librz.so missing, the first call raises instead of computing."""
+    import subprocess
+    import sys
+    code = (
+        "import invariant_logprobs_reinforce_b200 as rz\n"
+        "rz._LIB_PATH = '/nonexistent/librz.so'\n"
+        "try:\n"
+        "    rz.rz_workspace_bytes_loss(100, 2, 1, 256, 4096)\n"
+        "except ImportError as e:\n"
+        "    print('raised', e)\n"
+    )
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, cwd=root, timeout=300)
+    assert out.returncode == 0, out.stderr
+    assert out.stdout.startswith("raised") and "not built" in out.stdout
+
+
+def test_host_argument_checks_streamed(rz):
+    lib = rz.lib()
+
+    def call(**kw):
+        a = dict(Hh=128, Hd=256, W=512, ids=1024, lr=2048, r=3072, off=4096, gid=5120, n=100, R=4, G=2, d=256,
+                 V=4096, loss=6144, dH=7168, dW=8192, ws=1 << 20, wsb=1 << 40)
+        a.update(kw)
+        return lib.rz_loss_fwd_bwd_streamed(a["Hh"], a["Hd"], a["W"], a["ids"], a["lr"], a["r"], a["off"], a["gid"],
+                                            a["n"], a["R"], a["G"], a["d"], a["V"], None, a["loss"], a["dH"],
+                                            a["dW"], None, None, a["ws"], a["wsb"], None)
+
+    assert call(Hh=None) == 1   # no host rows
+    assert call(Hd=None) == 1   # no device buffer
+    assert call(Hd=260) == 1    # device buffer not 16-byte aligned
+    assert call(d=96) == 2
+    assert call(wsb=100) == 3
