@@ -158,3 +158,29 @@ def test_on_policy_ratio_statistics_vanish():
     st, rm = o.ratio_stats(c["lp"], c["lp"], c["off"])
     assert st["k1"] == 0 and st["k2"] == 0 and st["k3"] == 0 and st["dev_max"] == 0
     np.testing.assert_array_equal(rm, 1.0)
+
+
+@pytest.mark.parametrize("n,masked", [(101, False), (100, False), (1001, True), (2, False), (1, False)])
+def test_ratio_statistics_against_brute_force(n, masked):
+    """Peak, exact lower median (rank floor((m-1)/2) of the m counted tokens), extremes, count
+    and per-response mean ratio against a direct sort / mean of |w - 1| and w."""
+    rng = np.random.default_rng(n)
+    lp = -rng.exponential(2.0, n)
+    lr = lp + rng.normal(0.0, 0.2, n)
+    cuts = np.sort(rng.choice(np.arange(1, n), size=min(4, n - 1), replace=False)) if n > 1 else np.array([], int)
+    off = np.concatenate([[0], cuts, [n]]).astype(np.int64)
+    mask = (rng.uniform(size=n) < 0.7).astype(np.uint8) if masked else None
+    st, rm = o.ratio_stats(lp, lr, off, mask=mask)
+    keep = np.ones(n, bool) if mask is None else mask.astype(bool)
+    w = np.exp(lp - lr)
+    dev = np.sort(np.abs(w[keep] - 1.0))
+    m = dev.size
+    assert st["count"] == m
+    assert st["dev_median"] == pytest.approx(dev[(m - 1) // 2], rel=1e-14)
+    assert st["dev_max"] == pytest.approx(dev[-1], rel=1e-14)
+    assert st["w_min"] == pytest.approx(w[keep].min(), rel=1e-14)
+    assert st["w_max"] == pytest.approx(w[keep].max(), rel=1e-14)
+    for i in range(len(off) - 1):
+        sel = keep[off[i]:off[i + 1]]
+        expect = w[off[i]:off[i + 1]][sel].mean() if sel.any() else 0.0
+        assert rm[i] == pytest.approx(expect, rel=1e-14, abs=0.0)
