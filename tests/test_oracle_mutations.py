@@ -1,0 +1,60 @@
+"""Mutation check of the oracle's pins (CPU only).  Each case plants one plausible mistake
+in a copy of oracle/oracle.c (every occurrence of the line), rebuilds that copy and runs the
+pins (tests/test_oracle_pins.py) against it: some pin must fail.  The unmutated copy is the
+control and must pass.  Every planted line must still exist verbatim, so the list cannot
+silently drift away from the oracle."""
+import os
+import shutil
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+MUTATIONS = {
+    "control": None,
+    "dropped 1/L_i": ("loss += A[i] * (wsum / L);", "loss += A[i] * wsum;"),
+    "dropped 1/N": ("*loss_out = -loss / N;", "*loss_out = -loss;"),
+    "flipped loss sign": ("*loss_out = -loss / N;", "*loss_out = loss / N;"),
+    "inverted ratio": ("const double w = exp(lp[t] - lp_rollout[t]);",
+                       "const double w = exp(lp_rollout[t] - lp[t]);"),
+    "global instead of group mean": ("A[i] = rewards[i] - sum[gid[i]] / (double)cnt[gid[i]];",
+                                     "A[i] = rewards[i] - sum[0] / (double)cnt[0];"),
+    "transposed W index": ("elem(W, (size_t)v * d + k, is_bf16);", "elem(W, (size_t)k * V + v, is_bf16);"),
+    "dropped softmax term in dZ": ("(v == ids[t] ? 1.0 : 0.0) - exp(z[v] - lse_rows[j])",
+                                   "(v == ids[t] ? 1.0 : 0.0)"),
+    "kappa without w": ("if (kappa_out) kappa_out[t] = -A[i] * w / (N * L);",
+                        "if (kappa_out) kappa_out[t] = -A[i] / (N * L);"),
+    "lp without lse": ("if (lp) lp[j] = z[ids[t]] - l;", "if (lp) lp[j] = z[ids[t]] - z[0];"),
+    "wrong dZ sign": ("const double dz = kappa[t] * ((v == ids[t] ? 1.0 : 0.0) - exp(z - lse[t]));",
+                      "const double dz = kappa[t] * ((v == ids[t] ? 1.0 : 0.0) + exp(z - lse[t]));"),
+}
+
+
+def _copy_tree(dst):
+    ignore = shutil.ignore_patterns("*.so", "__pycache__", "*.pyc")
+    shutil.copytree(os.path.join(ROOT, "oracle"), os.path.join(dst, "oracle"), ignore=ignore)
+    shutil.copytree(os.path.join(ROOT, "tests"), os.path.join(dst, "tests"), ignore=ignore)
+    for f in ("workloads.py", "pytest.ini"):
+        shutil.copy(os.path.join(ROOT, f), dst)
+
+
+@pytest.mark.parametrize("name", list(MUTATIONS))
+def test_pins_catch_a_planted_mistake(tmp_path, name):
+    _copy_tree(str(tmp_path))
+    src_path = tmp_path / "oracle" / "oracle.c"
+    if MUTATIONS[name] is not None:
+        old, new = MUTATIONS[name]
+        text = src_path.read_text()
+        assert old in text, f"planted line no longer in oracle.c: {old}"
+        src_path.write_text(text.replace(old, new))
+    r = subprocess.run([sys.executable, "-m", "pytest", "tests/test_oracle_pins.py", "-q", "-x",
+                        "-p", "no:cacheprovider"], cwd=str(tmp_path), capture_output=True, text=True,
+                       timeout=900, env=dict(os.environ, PYTHONPATH=str(tmp_path)))
+    tail = (r.stdout + r.stderr)[-1500:]
+    if name == "control":
+        assert r.returncode == 0, tail
+    else:
+        # 1 = tests ran and some failed (not a build, collection or usage error)
+        assert r.returncode == 1 and "failed" in r.stdout, tail
