@@ -1,8 +1,9 @@
 """Mutation check of the oracle's pins (CPU only).  Each case plants one plausible mistake
 in a copy of oracle/oracle.c (every occurrence of the line), rebuilds that copy and runs the
-pins (tests/test_oracle_pins.py) against it: some pin must fail.  The unmutated copy is the
-control and must pass.  Every planted line must still exist verbatim, so the list cannot
-silently drift away from the oracle."""
+pins against it (tests/test_oracle_pins.py for the method's core, tests/test_oracle_variants.py
+for the loss-stage variants and the ratio diagnostics): some pin must fail.  The unmutated
+copy is the control for each pin file and must pass.  Every planted line must still exist
+verbatim, so the list cannot silently drift away from the oracle."""
 import os
 import shutil
 import subprocess
@@ -30,6 +31,26 @@ MUTATIONS = {
     "wrong dZ sign": ("const double dz = kappa[t] * ((v == ids[t] ? 1.0 : 0.0) - exp(z - lse[t]));",
                       "const double dz = kappa[t] * ((v == ids[t] ? 1.0 : 0.0) + exp(z - lse[t]));"),
 }
+PINS = "tests/test_oracle_pins.py"
+
+VARIANT_MUTATIONS = {
+    "control": None,
+    "clip from below": ("if ((flags & ORACLE_CLIP) && w > clip_max) w = clip_max;",
+                        "if ((flags & ORACLE_CLIP) && w < clip_max) w = clip_max;"),
+    "inverted gate": ("keep = (g >= gate_lo && g <= gate_hi);", "keep = !(g >= gate_lo && g <= gate_hi);"),
+    "gate on the summed log-ratio": ("const double g = exp(logsum / L);", "const double g = exp(logsum);"),
+    "mask ignored in L_i": ("      if (counted) {\n        L += 1.0;", "      if (1) {\n        L += 1.0;"),
+    "global N ignored": ("const double N = n_resp_total > 0 ? (double)n_resp_total : (double)R;",
+                         "const double N = (double)R;"),
+    "upper median": ("const double med = dev[(m - 1) / 2];", "const double med = dev[m / 2];"),
+    "k3 without -x": ("k3 += w - 1.0 - x;", "k3 += w - 1.0;"),
+    "k1 sign": ("k1 += -x;", "k1 += x;"),
+    "peak over w": ("if (d > dmax) dmax = d;", "if (w > dmax) dmax = w;"),
+    "mask ignored in the statistics": ("      if (mask && !mask[t]) continue;\n      const double x = lp[t] - lp_rollout[t];",
+                                       "      const double x = lp[t] - lp_rollout[t];"),
+}
+VARIANT_PINS = "tests/test_oracle_variants.py"
+CASES = [(PINS, k) for k in MUTATIONS] + [(VARIANT_PINS, k) for k in VARIANT_MUTATIONS]
 
 
 def _copy_tree(dst):
@@ -40,16 +61,17 @@ def _copy_tree(dst):
         shutil.copy(os.path.join(ROOT, f), dst)
 
 
-@pytest.mark.parametrize("name", list(MUTATIONS))
-def test_pins_catch_a_planted_mistake(tmp_path, name):
+@pytest.mark.parametrize("pins,name", CASES)
+def test_pins_catch_a_planted_mistake(tmp_path, pins, name):
     _copy_tree(str(tmp_path))
     src_path = tmp_path / "oracle" / "oracle.c"
-    if MUTATIONS[name] is not None:
-        old, new = MUTATIONS[name]
+    mutation = (MUTATIONS if pins == PINS else VARIANT_MUTATIONS)[name]
+    if mutation is not None:
+        old, new = mutation
         text = src_path.read_text()
         assert old in text, f"planted line no longer in oracle.c: {old}"
         src_path.write_text(text.replace(old, new))
-    r = subprocess.run([sys.executable, "-m", "pytest", "tests/test_oracle_pins.py", "-q", "-x",
+    r = subprocess.run([sys.executable, "-m", "pytest", pins, "-q", "-x",
                         "-p", "no:cacheprovider"], cwd=str(tmp_path), capture_output=True, text=True,
                        timeout=900, env=dict(os.environ, PYTHONPATH=str(tmp_path)))
     tail = (r.stdout + r.stderr)[-1500:]
