@@ -15,7 +15,10 @@ from .build import LIB as _LIB_PATH
 __all__ = [
     "RZ_OK", "RZError", "lib", "rz_status_string", "rz_workspace_bytes_logprobs", "rz_workspace_bytes_loss",
     "rz_workspace_bytes_segment_loss", "rz_token_logprobs", "rz_loss_fwd_bwd", "rz_segment_loss",
-    "rz_read_device_status", "EXPORTED_SYMBOLS",
+    "rz_read_device_status", "rz_num_launches_loss", "rz_loss_fwd_bwd_timed", "rz_loss_fwd_bwd_ex",
+    "rz_loss_fwd_bwd_streamed", "rz_segment_loss_ex", "rz_ratio_stats", "rz_grad_norms", "rz_quantize_rows_e4m3",
+    "rz_token_logprobs_fp8", "rz_sum_shards_f32", "rz_selftest_wait_timeout", "rz_loss_options", "loss_options",
+    "EXPORTED_SYMBOLS", "STAT_NAMES", "KERNEL_KINDS",
 ]
 
 RZ_OK = 0
@@ -42,7 +45,10 @@ class rz_loss_options(ctypes.Structure):
 
 
 def loss_options(clip_max=None, gate=None, token_mask=None, n_resp_total=0):
-    """Build rz_loss_options: clip_max (float), gate ((lo, hi)), token_mask (uint8 CUDA tensor)."""
+    """Build rz_loss_options: clip_max (float), gate ((lo, hi)), token_mask (contiguous uint8 CUDA
+    tensor [n_tok], kept alive by the returned struct; its length is checked at each call)."""
+    if token_mask is not None:
+        _need(token_mask, _torch().uint8, "token_mask")
     o = rz_loss_options()
     o.flags, o.clip_max, o.gate_lo, o.gate_hi, o.token_mask = 0, 0.0, 0.0, 0.0, None
     if clip_max is not None:
@@ -54,8 +60,11 @@ def loss_options(clip_max=None, gate=None, token_mask=None, n_resp_total=0):
     if token_mask is not None:
         o.flags |= RZ_LOSS_TOKEN_MASK
         o.token_mask = token_mask.data_ptr()
+    o._token_mask = token_mask
     o.n_resp_total = int(n_resp_total)
     return o
+
+
 KERNEL_KINDS = ("lmhead_lse", "merge_lse", "response_coef", "token_kappa", "loss_final", "dz", "dh", "dw",
                 "block_first")
 
@@ -177,6 +186,83 @@ def _need(t, dtype, name, device=None):
     return t
 
 
+def _shape(t, shape, name):
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return t
+
+
+def _need_shaped(t, dtype, name, device, shape):
+    """_need plus an exact shape; None passes through (an omitted optional argument)."""
+    if t is None:
+        return None
+    return _shape(_need(t, dtype, name, device), shape, name)
+
+
+def _matrix(t, dtype, name, device=None):
+    _need(t, dtype, name, device)
+    if t.dim() != 2:
+        raise ValueError(f"{name} must be 2-D, got shape {tuple(t.shape)}")
+    return t.shape
+
+
+def _segments(lp_rollout, rewards, seg_offsets, group_ids, n, dev):
+    """Checks the per-token rollout logprobs and the response / group description; returns R."""
+    torch = _torch()
+    _need_shaped(lp_rollout, torch.float32, "lp_rollout", dev, (n,))
+    _need(rewards, torch.float32, "rewards", dev)
+    if rewards.dim() != 1:
+        raise ValueError("rewards must be 1-D [n_resp]")
+    R = rewards.shape[0]
+    _need_shaped(seg_offsets, torch.int64, "seg_offsets", dev, (R + 1,))
+    _need_shaped(group_ids, torch.int32, "group_ids", dev, (R,))
+    return R
+
+
+def _token_vector(t, name):
+    """A per-token fp32 vector on a CUDA device; returns (n, device)."""
+    _need(t, _torch().float32, name)
+    if t.dim() != 1:
+        raise ValueError(f"{name} must be 1-D [n_tok]")
+    return t.shape[0], t.device
+
+
+def _loss_inputs(H, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids, H_name="H"):
+    """Checks the loss entry points' device inputs; returns (device, n, d, V, R)."""
+    torch = _torch()
+    n, d = _matrix(H, torch.bfloat16, H_name)
+    dev = H.device
+    V, dw = _matrix(W_head, torch.bfloat16, "W_head", dev)
+    if dw != d:
+        raise ValueError(f"W_head has d = {dw}, H has d = {d}")
+    _need_shaped(token_ids, torch.int32, "token_ids", dev, (n,))
+    R = _segments(lp_rollout, rewards, seg_offsets, group_ids, n, dev)
+    return dev, n, d, V, R
+
+
+def _loss_outputs(dev, n, d, V, loss=None, dH=None, dW=None, lp=None, kappa=None):
+    torch = _torch()
+    _need_shaped(loss, torch.float32, "loss", dev, (1,))
+    _need_shaped(dH, torch.bfloat16, "dH", dev, (n, d))
+    _need_shaped(dW, torch.float32, "dW", dev, (V, d))
+    _need_shaped(lp, torch.float32, "lp_out", dev, (n,))
+    _need_shaped(kappa, torch.float32, "kappa_out", dev, (n,))
+
+
+def _options_ref(options, n, dev):
+    """ctypes reference to rz_loss_options after checking its token mask against this call."""
+    if options is None:
+        return None
+    if not isinstance(options, rz_loss_options):
+        raise TypeError("options must be an rz_loss_options (see loss_options)")
+    if options.flags & RZ_LOSS_TOKEN_MASK:
+        m = getattr(options, "_token_mask", None)
+        if m is None or m.data_ptr() != (options.token_mask or 0):
+            raise ValueError("options carry a token mask without its tensor; build them with loss_options()")
+        _need_shaped(m, _torch().uint8, "token_mask", dev, (n,))
+    return ctypes.byref(options)
+
+
 def _workspace(nbytes, workspace, device):
     torch = _torch()
     if workspace is None:
@@ -200,14 +286,14 @@ def rz_token_logprobs(H, W_head, token_ids, lp_out=None, lse_out=None, workspace
     lse_out is given).
     """
     torch = _torch()
-    _need(H, torch.bfloat16, "H")
+    n, d = _matrix(H, torch.bfloat16, "H")
     dev = H.device
-    _need(W_head, torch.bfloat16, "W_head", dev)
-    _need(token_ids, torch.int32, "token_ids", dev)
-    n, d = H.shape
-    V = W_head.shape[0]
-    if W_head.shape[1] != d or token_ids.shape != (n,):
-        raise ValueError("shape mismatch")
+    V, dw = _matrix(W_head, torch.bfloat16, "W_head", dev)
+    if dw != d:
+        raise ValueError(f"W_head has d = {dw}, H has d = {d}")
+    _need_shaped(token_ids, torch.int32, "token_ids", dev, (n,))
+    _need_shaped(lp_out, torch.float32, "lp_out", dev, (n,))
+    _need_shaped(lse_out, torch.float32, "lse_out", dev, (n,))
     lp = lp_out if lp_out is not None else torch.empty(n, dtype=torch.float32, device=dev)
     lse = lse_out if lse_out is not None else (torch.empty(n, dtype=torch.float32, device=dev) if want_lse else None)
     ws_bytes = rz_workspace_bytes_logprobs(n, d, V)
@@ -223,19 +309,8 @@ def rz_loss_fwd_bwd(H, W_head, token_ids, lp_rollout, rewards, seg_offsets, grou
                     want_kappa=True):
     """Forward + REINFORCE Zero loss + backward.  Returns dict(loss, dH, dW, lp, kappa, workspace)."""
     torch = _torch()
-    _need(H, torch.bfloat16, "H")
-    dev = H.device
-    _need(W_head, torch.bfloat16, "W_head", dev)
-    _need(token_ids, torch.int32, "token_ids", dev)
-    _need(lp_rollout, torch.float32, "lp_rollout", dev)
-    _need(rewards, torch.float32, "rewards", dev)
-    _need(seg_offsets, torch.int64, "seg_offsets", dev)
-    _need(group_ids, torch.int32, "group_ids", dev)
-    n, d = H.shape
-    V = W_head.shape[0]
-    R = rewards.shape[0]
-    if seg_offsets.shape != (R + 1,) or group_ids.shape != (R,) or lp_rollout.shape != (n,):
-        raise ValueError("shape mismatch")
+    dev, n, d, V, R = _loss_inputs(H, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids)
+    _loss_outputs(dev, n, d, V, loss, dH, dW, lp_out, kappa_out)
     loss = loss if loss is not None else torch.empty(1, dtype=torch.float32, device=dev)
     dH = dH if dH is not None else torch.empty((n, d), dtype=torch.bfloat16, device=dev)
     dW = dW if dW is not None else torch.empty((V, d), dtype=torch.float32, device=dev)
@@ -265,9 +340,12 @@ def rz_loss_fwd_bwd_timed(events, H, W_head, token_ids, lp_rollout, rewards, seg
     have been recorded once (so their handles exist).  Returns the kernel kind of each
     recorded launch (indices into KERNEL_KINDS).
     """
-    n, d = H.shape
-    V = W_head.shape[0]
-    R = rewards.shape[0]
+    dev, n, d, V, R = _loss_inputs(H, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids)
+    _loss_outputs(dev, n, d, V, loss, dH, dW, lp_out, kappa_out)
+    for name, t in (("loss", loss), ("dH", dH), ("dW", dW)):
+        if t is None:
+            raise ValueError(f"{name} is required")
+    _need(workspace, _torch().uint8, "workspace", dev)
     cap = len(events) // 2
     handles = (ctypes.c_void_p * (2 * cap))(*[ctypes.c_void_p(e.cuda_event) for e in events[:2 * cap]])
     kinds = (ctypes.c_int32 * max(cap, 1))()
@@ -284,14 +362,11 @@ def rz_segment_loss(lp, lp_rollout, rewards, seg_offsets, group_ids, n_groups, l
                     w_out=None, want_w=False, workspace=None, stream=None):
     """The loss stage alone from given logprobs.  Returns dict(loss, kappa, w, workspace)."""
     torch = _torch()
-    _need(lp, torch.float32, "lp")
-    dev = lp.device
-    _need(lp_rollout, torch.float32, "lp_rollout", dev)
-    _need(rewards, torch.float32, "rewards", dev)
-    _need(seg_offsets, torch.int64, "seg_offsets", dev)
-    _need(group_ids, torch.int32, "group_ids", dev)
-    n = lp.shape[0]
-    R = rewards.shape[0]
+    n, dev = _token_vector(lp, "lp")
+    R = _segments(lp_rollout, rewards, seg_offsets, group_ids, n, dev)
+    _need_shaped(loss, torch.float32, "loss", dev, (1,))
+    _need_shaped(kappa_out, torch.float32, "kappa_out", dev, (n,))
+    _need_shaped(w_out, torch.float32, "w_out", dev, (n,))
     loss = loss if loss is not None else torch.empty(1, dtype=torch.float32, device=dev)
     kappa_out = kappa_out if kappa_out is not None else torch.empty(n, dtype=torch.float32, device=dev)
     if w_out is None and want_w:
@@ -315,11 +390,8 @@ def rz_loss_fwd_bwd_ex(H, W_head, token_ids, lp_rollout, rewards, seg_offsets, g
                        workspace=None, stream=None):
     """rz_loss_fwd_bwd with rz_loss_options (see loss_options).  Returns the same dict."""
     torch = _torch()
-    _need(H, torch.bfloat16, "H")
-    dev = H.device
-    n, d = H.shape
-    V = W_head.shape[0]
-    R = rewards.shape[0]
+    dev, n, d, V, R = _loss_inputs(H, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids)
+    opt = _options_ref(options, n, dev)
     out = dict(loss=torch.empty(1, dtype=torch.float32, device=dev),
                dH=torch.empty((n, d), dtype=torch.bfloat16, device=dev),
                dW=torch.empty((V, d), dtype=torch.float32, device=dev),
@@ -327,8 +399,7 @@ def rz_loss_fwd_bwd_ex(H, W_head, token_ids, lp_rollout, rewards, seg_offsets, g
                kappa=torch.empty(n, dtype=torch.float32, device=dev))
     ws = _workspace(rz_workspace_bytes_loss(n, R, n_groups, d, V), workspace, dev)
     code = lib().rz_loss_fwd_bwd_ex(_ptr(H), _ptr(W_head), _ptr(token_ids), _ptr(lp_rollout), _ptr(rewards),
-                                    _ptr(seg_offsets), _ptr(group_ids), n, R, n_groups, d, V,
-                                    ctypes.byref(options) if options is not None else None, _ptr(out["loss"]),
+                                    _ptr(seg_offsets), _ptr(group_ids), n, R, n_groups, d, V, opt, _ptr(out["loss"]),
                                     _ptr(out["dH"]), _ptr(out["dW"]), _ptr(out["lp"]), _ptr(out["kappa"]), _ptr(ws),
                                     ws.numel(), _stream_handle(stream))
     _check(code, "rz_loss_fwd_bwd_ex")
@@ -342,16 +413,17 @@ def rz_loss_fwd_bwd_streamed(H_host, H_dev, W_head, token_ids, lp_rollout, rewar
     overlap the compute) into the device buffer H_dev, chunk by chunk.  `out` (the dict this returns) may be
     passed back in to reuse its buffers.  H_host must stay unchanged until the work on the stream is done."""
     torch = _torch()
-    _need(H_dev, torch.bfloat16, "H_dev")
-    if H_host.dtype != torch.bfloat16 or H_host.device.type != "cpu" or not H_host.is_contiguous():
-        raise ValueError("H_host must be a contiguous CPU bf16 tensor")
+    dev, n, d, V, R = _loss_inputs(H_dev, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids, "H_dev")
+    if not isinstance(H_host, torch.Tensor) or H_host.dtype != torch.bfloat16:
+        raise TypeError("H_host must be a bf16 torch.Tensor")
+    if H_host.device.type != "cpu" or not H_host.is_contiguous():
+        raise ValueError("H_host must be a contiguous CPU tensor")
     if tuple(H_host.shape) != tuple(H_dev.shape):
         raise ValueError("H_host and H_dev must have the same shape")
-    dev = H_dev.device
-    n, d = H_dev.shape
-    V = W_head.shape[0]
-    R = rewards.shape[0]
-    if out is None:
+    opt = _options_ref(options, n, dev)
+    if out is not None:
+        _loss_outputs(dev, n, d, V, out["loss"], out["dH"], out["dW"], out.get("lp"), out.get("kappa"))
+    else:
         out = dict(loss=torch.empty(1, dtype=torch.float32, device=dev),
                    dH=torch.empty((n, d), dtype=torch.bfloat16, device=dev),
                    dW=torch.empty((V, d), dtype=torch.float32, device=dev),
@@ -359,8 +431,8 @@ def rz_loss_fwd_bwd_streamed(H_host, H_dev, W_head, token_ids, lp_rollout, rewar
                    kappa=torch.empty(n, dtype=torch.float32, device=dev))
     ws = _workspace(rz_workspace_bytes_loss(n, R, n_groups, d, V), workspace, dev)
     code = lib().rz_loss_fwd_bwd_streamed(_ptr(H_host), _ptr(H_dev), _ptr(W_head), _ptr(token_ids), _ptr(lp_rollout),
-                                          _ptr(rewards), _ptr(seg_offsets), _ptr(group_ids), n, R, n_groups, d, V,
-                                          ctypes.byref(options) if options is not None else None, _ptr(out["loss"]),
+                                          _ptr(rewards), _ptr(seg_offsets), _ptr(group_ids), n, R, n_groups, d, V, opt,
+                                          _ptr(out["loss"]),
                                           _ptr(out["dH"]), _ptr(out["dW"]), _ptr(out.get("lp")), _ptr(out.get("kappa")),
                                           _ptr(ws), ws.numel(), _stream_handle(stream))
     _check(code, "rz_loss_fwd_bwd_streamed")
@@ -372,15 +444,15 @@ def rz_segment_loss_ex(lp, lp_rollout, rewards, seg_offsets, group_ids, n_groups
                        workspace=None, stream=None):
     """rz_segment_loss with rz_loss_options.  Returns dict(loss, kappa, w, workspace)."""
     torch = _torch()
-    dev = lp.device
-    n = lp.shape[0]
-    R = rewards.shape[0]
+    n, dev = _token_vector(lp, "lp")
+    R = _segments(lp_rollout, rewards, seg_offsets, group_ids, n, dev)
+    opt = _options_ref(options, n, dev)
     loss = torch.empty(1, dtype=torch.float32, device=dev)
     kappa = torch.empty(n, dtype=torch.float32, device=dev)
     w = torch.empty(n, dtype=torch.float32, device=dev) if want_w else None
     ws = _workspace(rz_workspace_bytes_segment_loss(n, R, n_groups), workspace, dev)
     code = lib().rz_segment_loss_ex(_ptr(lp), _ptr(lp_rollout), _ptr(rewards), _ptr(seg_offsets), _ptr(group_ids), n,
-                                    R, n_groups, ctypes.byref(options) if options is not None else None, _ptr(loss),
+                                    R, n_groups, opt, _ptr(loss),
                                     _ptr(kappa), _ptr(w), _ptr(ws), ws.numel(), _stream_handle(stream))
     _check(code, "rz_segment_loss_ex")
     return dict(loss=loss, kappa=kappa, w=w, workspace=ws)
@@ -389,8 +461,12 @@ def rz_segment_loss_ex(lp, lp_rollout, rewards, seg_offsets, group_ids, n_groups
 def rz_ratio_stats(lp, lp_rollout, seg_offsets, token_mask=None, want_resp_mean=True, workspace=None, stream=None):
     """Ratio diagnostics.  Returns (stats tensor [9] fp64 on device, per-response mean ratio or None)."""
     torch = _torch()
-    dev = lp.device
-    n = lp.shape[0]
+    n, dev = _token_vector(lp, "lp")
+    _need_shaped(lp_rollout, torch.float32, "lp_rollout", dev, (n,))
+    _need(seg_offsets, torch.int64, "seg_offsets", dev)
+    if seg_offsets.dim() != 1 or seg_offsets.shape[0] < 1:
+        raise ValueError("seg_offsets must be 1-D [n_resp + 1]")
+    _need_shaped(token_mask, torch.uint8, "token_mask", dev, (n,))
     R = seg_offsets.shape[0] - 1
     stats = torch.empty(9, dtype=torch.float64, device=dev)
     rm = torch.empty(R, dtype=torch.float32, device=dev) if want_resp_mean else None
@@ -404,9 +480,11 @@ def rz_ratio_stats(lp, lp_rollout, seg_offsets, token_mask=None, want_resp_mean=
 def rz_grad_norms(dH, dW, workspace=None, stream=None):
     """(||dH||, ||dW||) as an fp64 device tensor [2]."""
     torch = _torch()
-    dev = dW.device
-    n, d = dH.shape
-    V = dW.shape[0]
+    n, d = _matrix(dH, torch.bfloat16, "dH")
+    dev = dH.device
+    V, dw = _matrix(dW, torch.float32, "dW", dev)
+    if dw != d:
+        raise ValueError(f"dW has d = {dw}, dH has d = {d}")
     out = torch.empty(2, dtype=torch.float64, device=dev)
     ws = _workspace(int(lib().rz_workspace_bytes_grad_norms()), workspace, dev)
     code = lib().rz_grad_norms(_ptr(dH), _ptr(dW), n, d, V, _ptr(out), _ptr(ws), ws.numel(), _stream_handle(stream))
@@ -417,8 +495,7 @@ def rz_grad_norms(dH, dW, workspace=None, stream=None):
 def rz_quantize_rows_e4m3(X, stream=None):
     """bf16 [rows, d] -> (e4m3 codes as uint8 [rows, d], fp32 per-row scales [rows])."""
     torch = _torch()
-    _need(X, torch.bfloat16, "X")
-    rows, d = X.shape
+    rows, d = _matrix(X, torch.bfloat16, "X")
     q = torch.empty((rows, d), dtype=torch.uint8, device=X.device)
     sc = torch.empty(rows, dtype=torch.float32, device=X.device)
     _check(lib().rz_quantize_rows_e4m3(_ptr(X), rows, d, _ptr(q), _ptr(sc), _stream_handle(stream)),
@@ -430,10 +507,16 @@ def rz_token_logprobs_fp8(H8, h_scale, W8, w_scale, token_ids, lp_out=None, lse_
                           stream=None, want_lse=True):
     """Token logprobs from e4m3 operands with per-row scales.  Returns (lp, lse)."""
     torch = _torch()
-    _need(H8, torch.uint8, "H8")
+    n, d = _matrix(H8, torch.uint8, "H8")
     dev = H8.device
-    n, d = H8.shape
-    V = W8.shape[0]
+    V, dw = _matrix(W8, torch.uint8, "W8", dev)
+    if dw != d:
+        raise ValueError(f"W8 has d = {dw}, H8 has d = {d}")
+    _need_shaped(h_scale, torch.float32, "h_scale", dev, (n,))
+    _need_shaped(w_scale, torch.float32, "w_scale", dev, (V,))
+    _need_shaped(token_ids, torch.int32, "token_ids", dev, (n,))
+    _need_shaped(lp_out, torch.float32, "lp_out", dev, (n,))
+    _need_shaped(lse_out, torch.float32, "lse_out", dev, (n,))
     lp = lp_out if lp_out is not None else torch.empty(n, dtype=torch.float32, device=dev)
     lse = lse_out if lse_out is not None else (torch.empty(n, dtype=torch.float32, device=dev) if want_lse else None)
     ws = _workspace(rz_workspace_bytes_logprobs(n, d, V), workspace, dev)
@@ -446,8 +529,8 @@ def rz_token_logprobs_fp8(H8, h_scale, W8, w_scale, token_ids, lp_out=None, lse_
 def rz_sum_shards_f32(stacked, out=None, stream=None):
     """Rank-order sum of the rows of a [nshards, count] fp32 CUDA tensor (fp64 accumulation)."""
     torch = _torch()
-    _need(stacked, torch.float32, "stacked")
-    nshards, count = stacked.shape
+    nshards, count = _matrix(stacked, torch.float32, "stacked")
+    _need_shaped(out, torch.float32, "out", stacked.device, (count,))
     out = out if out is not None else torch.empty(count, dtype=torch.float32, device=stacked.device)
     _check(lib().rz_sum_shards_f32(_ptr(stacked), nshards, count, _ptr(out), _stream_handle(stream)),
            "rz_sum_shards_f32")
