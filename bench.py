@@ -29,7 +29,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-METRIC = "fwd+bwd logprob/loss tokens/s on 1 B200"
+METRIC = "fwd+bwd logprob/loss tokens/s on 1 B200, % BF16 tensor peak, batch-invariance diff=0"
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -343,6 +343,10 @@ def run_rz(args, rank, world, local_rank):
         fwd8_ms = max_over_ranks(fwd8_ms, dev)
     del H8, W8
 
+    invariance = run_batch_invariance(rz, torch, dev, stream, H, W, ids, lp, wsf, prob.seed)
+    if dist:
+        invariance["diff"] = int(max_over_ranks(float(invariance["diff"]), dev))
+
     loss_stage = None
     if not args.no_loss_stage:
         loss_stage = run_loss_stage(rz, torch, dev, stream)
@@ -374,8 +378,44 @@ def run_rz(args, rank, world, local_rank):
         dominant=dom, achieved=ach, peak=peak_tflops, peak_src=peak_src,
         traffic=traffic_for(dom, tens[dom]["rows"] / tens[dom]["launches"]),
         fwd_ms=fwd_ms, fwd_tok_s=world * n / (fwd_ms * 1e-3), launches=launches_total, e2e=e2e, cfg=cfg,
-        loss_stage=loss_stage, fwd8_ms=fwd8_ms,
+        loss_stage=loss_stage, fwd8_ms=fwd8_ms, invariance=invariance,
     )
+
+
+def run_batch_invariance(rz, torch, dev, stream, H, W, ids, lp_step, ws, seed, n_alone=256, window=16384):
+    """The metric's "diff = 0", measured on the bench's own batch after the timed region: the
+    timed step's lp (from rz_loss_fwd_bwd) against the same rows from rz_token_logprobs
+    (a) alone, batch size 1, for n_alone sampled rows; (b) in prefill chunks of 64, 512 and
+    2048 rows over a window of the batch; (c) inside a permuted copy of the whole batch.
+    Counts the rows whose 32 bits differ anywhere."""
+    n = H.shape[0]
+    ref = lp_step.view(torch.int32)
+    g = torch.Generator()
+    g.manual_seed(seed)
+    rows = torch.randperm(n, generator=g)[:min(n_alone, n)].sort().values
+    lp1 = torch.empty(rows.numel(), dtype=torch.float32, device=dev)
+    for j, r in enumerate(rows.tolist()):
+        rz.rz_token_logprobs(H[r:r + 1], W, ids[r:r + 1], lp_out=lp1[j:j + 1], workspace=ws, stream=stream,
+                             want_lse=False)
+    differing = {"alone": int((lp1.view(torch.int32) != ref[rows.to(dev)]).sum())}
+    w0 = int(torch.randint(0, max(0, n - window) + 1, (1,), generator=g))
+    w1 = min(n, w0 + window)
+    lpc = torch.empty(w1 - w0, dtype=torch.float32, device=dev)
+    for c in (64, 512, 2048):
+        for c0 in range(w0, w1, c):
+            c1 = min(w1, c0 + c)
+            rz.rz_token_logprobs(H[c0:c1], W, ids[c0:c1], lp_out=lpc[c0 - w0:c1 - w0], workspace=ws, stream=stream,
+                                 want_lse=False)
+        differing[f"chunks_{c}"] = int((lpc.view(torch.int32) != ref[w0:w1]).sum())
+    perm = torch.randperm(n, generator=g).to(dev)
+    lpp = torch.empty(n, dtype=torch.float32, device=dev)
+    rz.rz_token_logprobs(H[perm].contiguous(), W, ids[perm].contiguous(), lp_out=lpp, workspace=ws, stream=stream,
+                         want_lse=False)
+    differing["permuted"] = int((lpp.view(torch.int32) != ref[perm]).sum())
+    return {"diff": sum(differing.values()), "rows_differing": differing,
+            "rows_checked": {"alone": rows.numel(), "chunks": 3 * (w1 - w0), "permuted": n},
+            "compared": "bits of the timed step's lp against rz_token_logprobs: rows alone, prefill chunks "
+                        f"of 64/512/2048 over rows {w0}..{w1 - 1}, the whole batch permuted"}
 
 
 def run_loss_stage(rz, torch, dev, stream, n_tok=1 << 26, reps=200):
@@ -708,6 +748,7 @@ def main():
                              "tensor_frac_2dV": res["n_tok"] * 2 * res["d"] * res["V"] / (res["fwd8_ms"] * 1e-3)
                              / (2 * res["peak"] * 1e12),
                              "peak_note": "e4m3 peak = 2 x the measured sustained bf16 peak (nominal ratio)"},
+            "batch_invariance": res["invariance"],
             "kernels": res["kernels"],
             "loss_stage": res["loss_stage"],
             "gpu_launches": res["launches"],

@@ -1,6 +1,7 @@
 """Host-side logic of bench.py (CPU only): the roofline's traffic record is used only while
 the recorded source digest matches the sources, the per-launch row accounting of the timed
-step, the algorithmic work per launch, and the clock reader without a GPU."""
+step, the algorithmic work per launch, the clock reader without a GPU, and the batch-invariance
+check's slicing and counting (with a CPU stand-in for the forward)."""
 import json
 import os
 import sys
@@ -65,3 +66,54 @@ def test_clock_reader_without_a_gpu_reports_nothing():
 
 def test_host_cpu_model_is_a_string():
     assert isinstance(bench.host_cpu_model(), str) and bench.host_cpu_model()
+
+
+class _RowwiseForward:
+    """CPU stand-in for rz_token_logprobs with the same slicing contract; `batch_term` makes
+    each row's value depend on how many rows share the call (a batch-variant forward)."""
+
+    def __init__(self, batch_term=0.0):
+        self.batch_term = batch_term
+        self.calls = 0
+
+    def rz_token_logprobs(self, H, W, ids, lp_out=None, workspace=None, stream=None, want_lse=True):
+        import torch
+        assert H.shape[0] == ids.shape[0] == lp_out.shape[0] and H.shape[1] == W.shape[1]
+        z = H.double() @ W.double().T
+        lp = z.gather(1, ids.long()[:, None])[:, 0] - torch.logsumexp(z, 1)
+        lp_out.copy_((lp + self.batch_term * (H.shape[0] > 1)).float())
+        self.calls += 1
+        return lp_out, None
+
+
+def _invariance_case(n, batch_term):
+    import torch
+    g = torch.Generator()
+    g.manual_seed(0)
+    H = torch.randn(n, 16, generator=g).to(torch.bfloat16)
+    W = torch.randn(40, 16, generator=g).to(torch.bfloat16)
+    ids = torch.randint(0, 40, (n,), generator=g, dtype=torch.int32)
+    fwd = _RowwiseForward(batch_term)
+    lp_step = torch.empty(n)
+    fwd.rz_token_logprobs(H, W, ids, lp_out=lp_step)
+    return fwd, bench.run_batch_invariance(fwd, torch, torch.device("cpu"), None, H, W, ids, lp_step, None, seed=5,
+                                           n_alone=20, window=300)
+
+
+@pytest.mark.parametrize("n", [1000, 130])
+def test_batch_invariance_check_reports_zero_for_a_rowwise_forward(n):
+    fwd, inv = _invariance_case(n, 0.0)
+    assert inv["diff"] == 0 and set(inv["rows_differing"].values()) == {0}
+    w = min(n, 300)
+    assert inv["rows_checked"] == {"alone": 20, "chunks": 3 * w, "permuted": n}
+    # 20 single rows, the window in chunks of 64 / 512 / 2048, one permuted batch (plus the step)
+    assert fwd.calls == 1 + 20 + sum(-(-w // c) for c in (64, 512, 2048)) + 1
+
+
+def test_batch_invariance_check_counts_rows_of_a_batch_variant_forward():
+    n = 1000
+    _, inv = _invariance_case(n, 0.5)
+    # computed alone, a row loses the batch term and differs; every batched row keeps it
+    assert inv["rows_differing"]["alone"] == 20
+    assert inv["rows_differing"]["chunks_64"] == 0 and inv["rows_differing"]["permuted"] == 0
+    assert inv["diff"] == 20
