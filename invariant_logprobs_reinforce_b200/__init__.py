@@ -17,7 +17,8 @@ __all__ = [
     "rz_workspace_bytes_segment_loss", "rz_token_logprobs", "rz_loss_fwd_bwd", "rz_segment_loss",
     "rz_read_device_status", "rz_num_launches_loss", "rz_loss_fwd_bwd_timed", "rz_loss_fwd_bwd_ex",
     "rz_loss_fwd_bwd_streamed", "rz_segment_loss_ex", "rz_ratio_stats", "rz_grad_norms", "rz_quantize_rows_e4m3",
-    "rz_token_logprobs_fp8", "rz_sum_shards_f32", "rz_selftest_wait_timeout", "rz_loss_options", "loss_options",
+    "rz_token_logprobs_fp8", "rz_sum_shards_f32", "rz_selftest_wait_timeout", "rz_token_logprobs_noalloc",
+    "rz_workspace_bytes_ratio_stats", "rz_workspace_bytes_grad_norms", "rz_loss_options", "loss_options",
     "EXPORTED_SYMBOLS", "STAT_NAMES", "KERNEL_KINDS",
 ]
 
@@ -151,6 +152,14 @@ def rz_workspace_bytes_loss(n_tok: int, n_resp: int, n_groups: int, d: int, V: i
 
 def rz_workspace_bytes_segment_loss(n_tok: int, n_resp: int, n_groups: int) -> int:
     return int(lib().rz_workspace_bytes_segment_loss(n_tok, n_resp, n_groups))
+
+
+def rz_workspace_bytes_ratio_stats(n_tok: int, n_resp: int) -> int:
+    return int(lib().rz_workspace_bytes_ratio_stats(n_tok, n_resp))
+
+
+def rz_workspace_bytes_grad_norms() -> int:
+    return int(lib().rz_workspace_bytes_grad_norms())
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -302,6 +311,27 @@ def rz_token_logprobs(H, W_head, token_ids, lp_out=None, lse_out=None, workspace
                                    ws.numel(), _stream_handle(stream))
     _check(code, "rz_token_logprobs")
     return lp, lse
+
+
+def rz_token_logprobs_noalloc(H, W_head, token_ids, lp_out, lse_out=None, stream=None):
+    """rz_token_logprobs from the library's fixed scratch instead of a workspace: the caller
+    passes every output buffer, and neither this wrapper nor the library allocates.  Calls
+    that may overlap on the GPU must be serialised by the caller (they share the scratch).
+    Returns (lp_out, lse_out)."""
+    torch = _torch()
+    n, d = _matrix(H, torch.bfloat16, "H")
+    dev = H.device
+    V, dw = _matrix(W_head, torch.bfloat16, "W_head", dev)
+    if dw != d:
+        raise ValueError(f"W_head has d = {dw}, H has d = {d}")
+    _need_shaped(token_ids, torch.int32, "token_ids", dev, (n,))
+    if lp_out is None:
+        raise ValueError("lp_out is required (this entry point allocates nothing)")
+    _need_shaped(lp_out, torch.float32, "lp_out", dev, (n,))
+    _need_shaped(lse_out, torch.float32, "lse_out", dev, (n,))
+    _check(lib().rz_token_logprobs_noalloc(_ptr(H), _ptr(W_head), _ptr(token_ids), n, d, V, _ptr(lp_out),
+                                           _ptr(lse_out), _stream_handle(stream)), "rz_token_logprobs_noalloc")
+    return lp_out, lse_out
 
 
 def rz_loss_fwd_bwd(H, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids, n_groups, loss=None,
@@ -470,7 +500,7 @@ def rz_ratio_stats(lp, lp_rollout, seg_offsets, token_mask=None, want_resp_mean=
     R = seg_offsets.shape[0] - 1
     stats = torch.empty(9, dtype=torch.float64, device=dev)
     rm = torch.empty(R, dtype=torch.float32, device=dev) if want_resp_mean else None
-    ws = _workspace(int(lib().rz_workspace_bytes_ratio_stats(n, R)), workspace, dev)
+    ws = _workspace(rz_workspace_bytes_ratio_stats(n, R), workspace, dev)
     code = lib().rz_ratio_stats(_ptr(lp), _ptr(lp_rollout), _ptr(seg_offsets), n, R, _ptr(token_mask), _ptr(stats),
                                 _ptr(rm), _ptr(ws), ws.numel(), _stream_handle(stream))
     _check(code, "rz_ratio_stats")
@@ -486,7 +516,7 @@ def rz_grad_norms(dH, dW, workspace=None, stream=None):
     if dw != d:
         raise ValueError(f"dW has d = {dw}, dH has d = {d}")
     out = torch.empty(2, dtype=torch.float64, device=dev)
-    ws = _workspace(int(lib().rz_workspace_bytes_grad_norms()), workspace, dev)
+    ws = _workspace(rz_workspace_bytes_grad_norms(), workspace, dev)
     code = lib().rz_grad_norms(_ptr(dH), _ptr(dW), n, d, V, _ptr(out), _ptr(ws), ws.numel(), _stream_handle(stream))
     _check(code, "rz_grad_norms")
     return out

@@ -58,6 +58,13 @@ def test_every_prototype_is_parsed():
     assert set(protos) == set(rz.EXPORTED_SYMBOLS)
 
 
+def test_every_declared_call_has_a_python_function_of_the_same_name():
+    import invariant_logprobs_reinforce_b200 as rz
+    missing = [name for name in _prototypes() if not callable(getattr(rz, name, None))]
+    assert not missing, missing
+    assert set(_prototypes()) <= set(rz.__all__)
+
+
 @pytest.mark.parametrize("name", sorted(_prototypes()))
 def test_binding_signature_matches_the_header(lib, name):
     ret, params = _prototypes()[name]

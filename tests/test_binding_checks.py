@@ -93,6 +93,9 @@ def _calls():
             lambda x: dict(lp_out=torch.zeros(n), lse_out=torch.zeros(n))),
         "rz_sum_shards_f32": (rz.rz_sum_shards_f32, lambda x: [torch.zeros((4, 33))],
                               lambda x: dict(out=torch.zeros(33))),
+        "rz_token_logprobs_noalloc": (rz.rz_token_logprobs_noalloc,
+                                      lambda x: [x["H"], x["W_head"], x["token_ids"], torch.zeros(n)],
+                                      lambda x: dict(lse_out=torch.zeros(n))),
     }
 
 

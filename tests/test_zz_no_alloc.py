@@ -62,6 +62,17 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(rz):
         assert torch.equal(lse.view(torch.int32), ref_lse.view(torch.int32))
 
 
+def test_python_wrapper_is_the_same_call(rz):
+    H, W, ids = _problem(500, 512, 9000, 3)
+    lp = torch.empty(500, device="cuda")
+    lse = torch.empty(500, device="cuda")
+    rz.rz_token_logprobs_noalloc(H, W, ids, lp, lse)
+    ref_lp, ref_lse = rz.rz_token_logprobs(H, W, ids)
+    torch.cuda.synchronize()
+    assert torch.equal(lp.view(torch.int32), ref_lp.view(torch.int32))
+    assert torch.equal(lse.view(torch.int32), ref_lse.view(torch.int32))
+
+
 def test_noalloc_rejects_calls_beyond_its_scratch(rz):
     d, V = 256, 151936
     segs = -(-V // 2048)
