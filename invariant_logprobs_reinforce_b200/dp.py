@@ -17,6 +17,7 @@ summation can be injected only for testing the orchestration on CPU ranks.
 """
 from __future__ import annotations
 
+import numpy as np
 import torch
 import torch.distributed as dist
 
@@ -55,16 +56,59 @@ def global_response_count(n_resp_local: int, device, group=None) -> int:
     return int(t.item())
 
 
+def shard_groups(seg_offsets, group_ids, world: int):
+    """Split a batch into `world` shards of whole groups, balanced by tokens (host logic).
+
+    Each group's responses must form one contiguous run (the layout the group-mean advantage
+    is computed over).  Shard r ends at the group boundary whose token offset is closest to
+    (r + 1) n_tok / world, keeping at least one group for every shard after it; needs at
+    least `world` groups.  Returns one dict per rank: its token range [tok_lo, tok_hi), its
+    response range [resp_lo, resp_hi), its seg_offsets rebased to 0 and its group ids
+    renumbered 0 .. n_groups - 1 in order of appearance."""
+    off = np.asarray(seg_offsets, dtype=np.int64)
+    gid = np.asarray(group_ids, dtype=np.int64)
+    R = gid.shape[0]
+    if off.shape != (R + 1,) or R == 0:
+        raise ValueError("seg_offsets must have n_resp + 1 entries, n_resp >= 1")
+    starts = np.flatnonzero(np.r_[True, gid[1:] != gid[:-1]])  # first response of each run
+    if np.unique(gid[starts]).shape[0] != starts.shape[0]:
+        raise ValueError("a group's responses must be contiguous")
+    n_runs = starts.shape[0]
+    if n_runs < world:
+        raise ValueError(f"{n_runs} groups cannot fill {world} shards")
+    bounds = np.r_[starts, R]  # response index of every group boundary
+    n_tok = int(off[-1])
+    cut = [0]
+    for r in range(1, world):
+        lo, hi = cut[-1] + 1, n_runs - (world - r)  # boundary indices still allowed
+        cand = np.arange(lo, hi + 1)
+        target = r * n_tok / world
+        cut.append(int(cand[np.argmin(np.abs(off[bounds[cand]] - target))]))
+    cut.append(n_runs)
+    shards = []
+    for r in range(world):
+        r0, r1 = int(bounds[cut[r]]), int(bounds[cut[r + 1]])
+        t0, t1 = int(off[r0]), int(off[r1])
+        local = gid[r0:r1]
+        _, first = np.unique(local, return_index=True)
+        order = np.argsort(np.argsort(first))  # rank of each distinct id by first appearance
+        ids = order[np.searchsorted(np.unique(local), local)].astype(np.int32)
+        shards.append(dict(tok_lo=t0, tok_hi=t1, resp_lo=r0, resp_hi=r1, seg_offsets=off[r0:r1 + 1] - t0,
+                           group_ids=ids, n_groups=int(first.shape[0])))
+    return shards
+
+
 def dp_loss_fwd_bwd(H, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids, n_groups, group=None,
-                    options=None):
-    """One data-parallel step: this rank's shard (whole groups) through rz_loss_fwd_bwd_ex with
-    N = the global response count, then dW and the loss summed deterministically.  dH stays
-    local (its rows are this rank's tokens).  Returns the rz_loss_fwd_bwd dict with the
-    global loss and dW."""
+                    options=None, sum_shards=None):
+    """One data-parallel step: this rank's shard (whole groups, e.g. from shard_groups) through
+    rz_loss_fwd_bwd_ex with N = the global response count, then dW and the loss summed
+    deterministically.  dH stays local (its rows are this rank's tokens).  Returns the
+    rz_loss_fwd_bwd dict with the global loss and dW.  `sum_shards` is for testing the
+    orchestration on CPU ranks only (see deterministic_all_reduce)."""
     n_total = global_response_count(rewards.shape[0], rewards.device, group)
     opts = options if options is not None else loss_options()
     opts.n_resp_total = n_total
     out = rz_loss_fwd_bwd_ex(H, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids, n_groups, opts)
-    out["dW"] = deterministic_all_reduce(out["dW"], group)
-    out["loss"] = deterministic_all_reduce(out["loss"], group)
+    out["dW"] = deterministic_all_reduce(out["dW"], group, sum_shards)
+    out["loss"] = deterministic_all_reduce(out["loss"], group, sum_shards)
     return out
