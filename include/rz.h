@@ -235,7 +235,7 @@ rz_status rz_ratio_stats(const float* lp, const float* lp_rollout, const int64_t
 /*
  * Frobenius norms of the gradients: norms_out[0] = ||dH|| (bf16 [n_tok, d]),
  * norms_out[1] = ||dW|| (fp32 [V, d]), fp64, device; fixed-order reductions (deterministic).
- * The pages report the largest gradient norm before clipping ("vLLM says aligned
+ * The pages report the peak pre-clipping gradient norm ("vLLM says aligned
  * kernels…", section "Reported results include 2.40 times higher throughput").
  */
 size_t rz_workspace_bytes_grad_norms(void);
@@ -244,7 +244,7 @@ rz_status rz_grad_norms(const rz_bf16* dH, const float* dW, int64_t n_tok, int32
 
 /*
  * Low-precision forward: token logprobs from e4m3 (fp8) operands with per-row scales, the
- * pages' "low-precision compute" of the rollout side ("vLLM Train-Inference Consistency
+ * pages' reduced-precision arithmetic on the rollout side ("vLLM Train-Inference Consistency
  * Release Notes", section "The Technical Challenge"; "vLLM says aligned kernels…", section
  * "Zero mismatch expands to newer models": FP8 weights), under the same batch-invariance
  * contract as rz_token_logprobs.

@@ -14,8 +14,9 @@
  *       (token logprob = log-softmax of the LM-head logits, gathered at the token);
  *     - the ratio is the learner probability divided by the recorded rollout probability,
  *       with no clipping:  w_t = exp(lp_t - lp_rollout_t);
- *     - the advantage of a response is its reward minus the mean reward of its group;
- *     - tokens are averaged within a response; no value model, no rejection gates;
+ *     - a response's advantage is r_i less the average r over the responses of its group;
+ *     - the per-token terms of a response are combined by a mean over that response's
+ *       tokens; there is no value model and no gate rejects any response;
  *     - the objective is plain REINFORCE (importance weighted).
  *
  * Definitions written out (everything in fp64, inputs widened exactly):
@@ -295,8 +296,8 @@ int oracle_num_threads(void) {
 /* ------------------------------------------------------------------------------------
  * Variants of the loss stage (the baselines the pages contrast REINFORCE Zero with) and
  * diagnostics of the ratio.  Readings, as the pages give no formulas:
- *   - truncated IS ("clipping the importance weights can introduce bias", [A] section
- *     "REINFORCE Zero removes the mismatch first"): w -> min(w, clip_max) in the
+ *   - truncated IS (the clipped-weight baseline, which the page says biases the gradient;
+ *     [A] section "REINFORCE Zero removes the mismatch first"): w -> min(w, clip_max) in the
  *     coefficient of each token's gradient, held constant;
  *   - sequence gate (the standard-kernel baseline on OSWorld, [A] section "Zero mismatch
  *     expands to newer models"): response i is kept iff gate_lo <= exp(mean_t (lp - lp_rollout))
