@@ -1,8 +1,9 @@
 """Mutation check of the oracle's pins (CPU only).  Each case plants one plausible mistake
 in a copy of oracle/oracle.c (every occurrence of the line), rebuilds that copy and runs the
 pins against it (tests/test_oracle_pins.py for the method's core, tests/test_oracle_variants.py
-for the loss-stage variants and the ratio diagnostics): some pin must fail.  The unmutated
-copy is the control for each pin file and must pass.  Every planted line must still exist
+for the loss-stage variants and the ratio diagnostics; the e4m3 helpers in oracle/__init__.py
+against tests/test_oracle_fp8.py): some pin must fail.  The unmutated copy is the control for
+each pin file and must pass.  Every planted line must still exist
 verbatim, so the list cannot silently drift away from the oracle."""
 import os
 import shutil
@@ -50,7 +51,20 @@ VARIANT_MUTATIONS = {
                                        "      const double x = lp[t] - lp_rollout[t];"),
 }
 VARIANT_PINS = "tests/test_oracle_variants.py"
-CASES = [(PINS, k) for k in MUTATIONS] + [(VARIANT_PINS, k) for k in VARIANT_MUTATIONS]
+
+FP8_MUTATIONS = {
+    "control": None,
+    "e4m3 range of the fnuz variant": ("E4M3_MAX = 448.0", "E4M3_MAX = 240.0"),
+    "decoded as e5m2": ("torch.float8_e4m3fn).double()", "torch.float8_e5m2).double()"),
+    "no zero-row guard": ("torch.where(m > 0, m / torch.tensor(E4M3_MAX, dtype=torch.float32), torch.ones_like(m))",
+                          "m / torch.tensor(E4M3_MAX, dtype=torch.float32)"),
+    "scale from the row mean": ("m = x.abs().amax(dim=1)", "m = x.abs().mean(dim=1)"),
+    "sign dropped": ("y = (x / sc[:, None])", "y = (x.abs() / sc[:, None])"),
+}
+FP8_PINS = "tests/test_oracle_fp8.py"
+TARGETS = {PINS: ("oracle.c", MUTATIONS), VARIANT_PINS: ("oracle.c", VARIANT_MUTATIONS),
+           FP8_PINS: ("__init__.py", FP8_MUTATIONS)}
+CASES = [(pins, k) for pins, (_, table) in TARGETS.items() for k in table]
 
 
 def _copy_tree(dst):
@@ -64,12 +78,13 @@ def _copy_tree(dst):
 @pytest.mark.parametrize("pins,name", CASES)
 def test_pins_catch_a_planted_mistake(tmp_path, pins, name):
     _copy_tree(str(tmp_path))
-    src_path = tmp_path / "oracle" / "oracle.c"
-    mutation = (MUTATIONS if pins == PINS else VARIANT_MUTATIONS)[name]
+    target, table = TARGETS[pins]
+    src_path = tmp_path / "oracle" / target
+    mutation = table[name]
     if mutation is not None:
         old, new = mutation
         text = src_path.read_text()
-        assert old in text, f"planted line no longer in oracle.c: {old}"
+        assert old in text, f"planted line no longer in oracle/{target}: {old}"
         src_path.write_text(text.replace(old, new))
     r = subprocess.run([sys.executable, "-m", "pytest", pins, "-q", "-x",
                         "-p", "no:cacheprovider"], cwd=str(tmp_path), capture_output=True, text=True,
