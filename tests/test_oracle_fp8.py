@@ -1,4 +1,4 @@
-"""Pins of the oracle's e4m3 helpers (CPU only) against the OCP 8-bit floating-point
+"""Pins of the oracle's e4m3 helpers and of its fp64-operand path (CPU only): the helpers against the OCP 8-bit floating-point
 definition of E4M3 ("fn" variant: no infinities, one NaN pattern per sign), written out
 here bit by bit, and against brute force over all 256 codes.  The pages name FP8 weights
 and reduced-precision arithmetic on the rollout side but fix no format or scaling; the
@@ -94,3 +94,34 @@ def test_hand_worked_ties(x, code):
 def test_zero_row_has_scale_one_and_zero_codes():
     q, sc = oracle.quantize_rows_e4m3(_bf16_rows(np.zeros((2, 64), np.float32)))
     assert np.all(sc == 1.0) and np.all((q & 0x7F) == 0)
+
+
+def test_fp64_operands_are_used_as_given():
+    """The fp8 parity test hands the oracle fp64 operands (decoded codes times scales).  With
+    H_t = e_k the logits are the head's column k exactly, so lp and lse have closed forms;
+    the head's values are not fp32 or bf16 numbers, so any narrowing of the fp64 input path
+    would show."""
+    from scipy.special import logsumexp
+    rng = np.random.default_rng(5)
+    V, d = 40, 8
+    W = rng.standard_normal((V, d)) * (1 + 1e-12)   # not representable in fp32
+    assert np.any(W.astype(np.float32).astype(np.float64) != W)
+    ks = np.array([0, 5, 7], np.int64)
+    H = np.zeros((3, d))
+    H[np.arange(3), ks] = 1.0
+    ids = np.array([3, 39, 0], np.int32)
+    lp, lse = oracle.token_logprobs(H, W, ids)
+    for t, k in enumerate(ks):
+        ref = logsumexp(W[:, k])
+        assert abs(lse[t] - ref) <= 1e-14 * max(1.0, abs(ref))
+        assert abs(lp[t] - (W[ids[t], k] - ref)) <= 1e-14 * max(1.0, abs(ref))
+
+
+def test_fp64_and_bf16_bit_operands_agree_on_bf16_values():
+    rng = np.random.default_rng(6)
+    Hb = wl.bf16_bits(rng.standard_normal((20, 64)).astype(np.float32))
+    Wb = wl.bf16_bits((rng.standard_normal((300, 64)) / 8).astype(np.float32))
+    ids = rng.integers(0, 300, 20).astype(np.int32)
+    a = oracle.token_logprobs(Hb, Wb, ids)
+    b = oracle.token_logprobs(wl.bits_to_f32(Hb).astype(np.float64), wl.bits_to_f32(Wb).astype(np.float64), ids)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
