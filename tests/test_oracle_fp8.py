@@ -1,8 +1,9 @@
-"""Pins of the oracle's e4m3 helpers and of its fp64-operand path (CPU only): the helpers against the OCP 8-bit floating-point
-definition of E4M3 ("fn" variant: no infinities, one NaN pattern per sign), written out
-here bit by bit, and against brute force over all 256 codes.  The pages name FP8 weights
-and reduced-precision arithmetic on the rollout side but fix no format or scaling; the
-reading is per-row absmax scaling to the e4m3 range, round to nearest even."""
+"""Pins of the oracle's e4m3 helpers and of its fp64-operand path (CPU only).  The helpers
+are checked against the OCP 8-bit floating-point definition of E4M3 ("fn" variant: no
+infinities, one NaN pattern per sign), written out here bit by bit, and against brute force
+over all 256 codes.  The pages name FP8 weights and reduced-precision arithmetic on the
+rollout side but fix no format or scaling; the reading is per-row absmax scaling to the
+e4m3 range, round to nearest even."""
 import math
 
 import numpy as np
