@@ -288,6 +288,23 @@ def test_p6_dW_columns_sum_to_zero(oracle):
     assert np.abs(col).max() < 1e-12 * max(1.0, np.abs(out["dW"]).sum(axis=0).max())
 
 
+def test_p7_dH_is_kappa_times_target_row_minus_softmax_mean_row(oracle):
+    """dH_t = kappa_t (W[y_t] - sum_v p_tv W[v]): the factored form, with p from scipy's
+    softmax of logits formed here in fp64 (not the oracle's lse); only kappa comes from the
+    oracle (pinned by the finite differences)."""
+    from scipy.special import softmax
+    p = wl.tiny()
+    lp, _ = oracle.token_logprobs(p.H, p.W, p.ids)
+    lr = wl.rollout_logprobs_with_lag(lp, p.noise, p.seed)
+    out = oracle.loss_fwd_bwd(p.H, p.W, p.ids, lr, p.seg.rewards, p.seg.seg_offsets, p.seg.group_ids,
+                              p.seg.n_groups)
+    Hf = wl.bits_to_f32(p.H).astype(np.float64)
+    Wf = wl.bits_to_f32(p.W).astype(np.float64)
+    P = softmax(Hf @ Wf.T, axis=1)
+    ref = out["kappa"][:, None] * (Wf[p.ids] - P @ Wf)
+    assert np.abs(out["dH"] - ref).max() <= 1e-12 * np.abs(ref).max()
+
+
 def test_dh_dw_row_subsets_match_full(oracle):
     p = _tiny_problem()
     out = oracle.loss_fwd_bwd(p["H"], p["W"], p["ids"], p["lp_rollout"], p["rewards"], p["seg_offsets"],
