@@ -4,7 +4,6 @@ checked over random shapes, group layouts, lengths, rewards and lags (hypothesis
 section "REINFORCE Zero removes the mismatch first" (group-mean advantage, per-response
 token mean, unclipped ratio)."""
 import numpy as np
-import pytest
 from hypothesis import given, settings, strategies as st
 
 import workloads as wl
