@@ -1,6 +1,5 @@
 """Boundary behaviour on the GPU: device-checked inputs set status bits and never trap,
 argument errors enqueue nothing, optional outputs may be omitted, empty calls are no-ops."""
-import numpy as np
 import pytest
 import torch
 

@@ -2,7 +2,6 @@
 kernels are the ones of rz_loss_fwd_bwd_ex, so every output must be bit-identical to the
 call with H already on the device; the tests start from a device buffer full of garbage, so
 a chunk computed before its copy landed would show."""
-import numpy as np
 import pytest
 import torch
 
