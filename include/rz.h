@@ -39,6 +39,9 @@
  *   - Device-checked inputs (a violation sets a bit of the device status and never
  *     traps): 0 <= token_ids[t] < V (the row's lp becomes NaN); seg_offsets[0] = 0,
  *     seg_offsets strictly increasing, seg_offsets[n_resp] = n_tok; 0 <= group_ids < n_groups.
+ *     After a failed device check the loss path's outputs carry no meaning: a NaN logprob
+ *     or coefficient spreads into its response's kappa, the loss, its dH rows and all of
+ *     dW.  Read the status (rz_read_device_status) before using them.
  */
 #ifndef RZ_H_
 #define RZ_H_
