@@ -2,7 +2,8 @@
 in a copy of oracle/oracle.c (every occurrence of the line), rebuilds that copy and runs the
 pins against it (tests/test_oracle_pins.py for the method's core, tests/test_oracle_variants.py
 for the loss-stage variants and the ratio diagnostics; the e4m3 helpers in oracle/__init__.py
-against tests/test_oracle_fp8.py): some pin must fail.  The unmutated copy is the control for
+against tests/test_oracle_fp8.py; the MXFP4 reference in oracle/mxfp4.py against
+tests/test_oracle_mxfp4.py): some pin must fail.  The unmutated copy is the control for
 each pin file and must pass.  Every planted line must still exist
 verbatim, so the list cannot silently drift away from the oracle."""
 import os
@@ -62,8 +63,18 @@ FP8_MUTATIONS = {
     "sign dropped": ("y = (x / sc[:, None])", "y = (x.abs() / sc[:, None])"),
 }
 FP8_PINS = "tests/test_oracle_fp8.py"
+
+MXFP4_MUTATIONS = {
+    "control": None,
+    "E2M1 top exponent 1": ("E2M1_EMAX = 2", "E2M1_EMAX = 1"),
+    "ceiling block exponent": ("Xe = (e.astype(np.int64) - 1) - E2M1_EMAX", "Xe = e.astype(np.int64) - E2M1_EMAX"),
+    "ties to odd": ("even = tie & (np.arange(8) % 2 == 0)", "even = tie & (np.arange(8) % 2 == 1)"),
+    "sign dropped": ("return mag | (np.signbit(y).astype(np.uint8) << 3)", "return mag"),
+    "E8M0 bias 128": ("return codes, (Xe + 127).astype(np.uint8)", "return codes, (Xe + 128).astype(np.uint8)"),
+}
+MXFP4_PINS = "tests/test_oracle_mxfp4.py"
 TARGETS = {PINS: ("oracle.c", MUTATIONS), VARIANT_PINS: ("oracle.c", VARIANT_MUTATIONS),
-           FP8_PINS: ("__init__.py", FP8_MUTATIONS)}
+           FP8_PINS: ("__init__.py", FP8_MUTATIONS), MXFP4_PINS: ("mxfp4.py", MXFP4_MUTATIONS)}
 CASES = [(pins, k) for pins, (_, table) in TARGETS.items() for k in table]
 
 
@@ -75,23 +86,44 @@ def _copy_tree(dst):
         shutil.copy(os.path.join(ROOT, f), dst)
 
 
-@pytest.mark.parametrize("pins,name", CASES)
-def test_pins_catch_a_planted_mistake(tmp_path, pins, name):
-    _copy_tree(str(tmp_path))
+def _run_case(root, pins, name):
+    """Plant one mistake in a fresh copy under `root` and run its pin file there; returns
+    (returncode, stdout, output tail)."""
+    _copy_tree(root)
     target, table = TARGETS[pins]
-    src_path = tmp_path / "oracle" / target
+    src_path = os.path.join(root, "oracle", target)
     mutation = table[name]
     if mutation is not None:
         old, new = mutation
-        text = src_path.read_text()
-        assert old in text, f"planted line no longer in oracle/{target}: {old}"
-        src_path.write_text(text.replace(old, new))
-    r = subprocess.run([sys.executable, "-m", "pytest", pins, "-q", "-x",
-                        "-p", "no:cacheprovider"], cwd=str(tmp_path), capture_output=True, text=True,
-                       timeout=900, env=dict(os.environ, PYTHONPATH=str(tmp_path)))
-    tail = (r.stdout + r.stderr)[-1500:]
+        with open(src_path) as f:
+            text = f.read()
+        if old not in text:
+            return None, "", f"planted line no longer in oracle/{target}: {old}"
+        with open(src_path, "w") as f:
+            f.write(text.replace(old, new))
+    # one OpenMP thread per copy: the copies run side by side
+    env = dict(os.environ, PYTHONPATH=root, OMP_NUM_THREADS="1")
+    r = subprocess.run([sys.executable, "-m", "pytest", pins, "-q", "-x", "-p", "no:cacheprovider"], cwd=root,
+                       capture_output=True, text=True, timeout=900, env=env)
+    return r.returncode, r.stdout, (r.stdout + r.stderr)[-1500:]
+
+
+@pytest.fixture(scope="module")
+def outcomes(tmp_path_factory):
+    """Every case, each in its own copy, run concurrently (independent subprocesses)."""
+    from concurrent.futures import ThreadPoolExecutor
+    roots = {case: str(tmp_path_factory.mktemp("mut")) for case in CASES}
+    with ThreadPoolExecutor(max_workers=max(1, min(len(CASES), os.cpu_count() or 1))) as pool:
+        futures = {case: pool.submit(_run_case, roots[case], *case) for case in CASES}
+        return {case: f.result() for case, f in futures.items()}
+
+
+@pytest.mark.parametrize("pins,name", CASES)
+def test_pins_catch_a_planted_mistake(outcomes, pins, name):
+    code, stdout, tail = outcomes[(pins, name)]
+    assert code is not None, tail
     if name == "control":
-        assert r.returncode == 0, tail
+        assert code == 0, tail
     else:
         # 1 = tests ran and some failed (not a build, collection or usage error)
-        assert r.returncode == 1 and "failed" in r.stdout, tail
+        assert code == 1 and "failed" in stdout, tail
