@@ -46,12 +46,6 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
     return LIB
 
 
-if __name__ == "__main__":
-    import sys
-    build(force="--force" in sys.argv, verbose=True,
-          extra_flags=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else [])
-
-
 def source_digest(family: str = "all") -> str:
     """sha256 prefix over the sources that define a kernel family.
 
@@ -71,3 +65,9 @@ def source_digest(family: str = "all") -> str:
         with open(p, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
+
+
+if __name__ == "__main__":
+    import sys
+    build(force="--force" in sys.argv, verbose=True,
+          extra_flags=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else [])
