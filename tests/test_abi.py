@@ -140,3 +140,139 @@ def test_host_argument_checks_streamed(rz):
     assert call(Hd=260) == 1    # device buffer not 16-byte aligned
     assert call(d=96) == 2
     assert call(wsb=100) == 3
+
+
+def _opts(rz, **kw):
+    o = rz.rz_loss_options()
+    o.flags, o.clip_max, o.gate_lo, o.gate_hi, o.token_mask, o.n_resp_total = 0, 0.0, 0.0, 0.0, None, 0
+    for k, v in kw.items():
+        setattr(o, k, v)
+    return o
+
+
+def _bad_options(rz):
+    C, G, M = rz.RZ_LOSS_CLIP_IS, rz.RZ_LOSS_SEQ_GATE, rz.RZ_LOSS_TOKEN_MASK
+    return [
+        _opts(rz, flags=8),                              # unknown flag bit
+        _opts(rz, flags=C, clip_max=0.0),                # clip_max must be > 0
+        _opts(rz, flags=C, clip_max=float("nan")),
+        _opts(rz, flags=G, gate_lo=2.0, gate_hi=1.0),    # empty gate interval
+        _opts(rz, flags=M, token_mask=None),             # mask flag without a mask
+        _opts(rz, flags=M, token_mask=4098),             # mask not 4-byte aligned
+        _opts(rz, n_resp_total=-1),
+    ]
+
+
+def test_host_checks_of_the_loss_options(rz):
+    import ctypes
+    lib = rz.lib()
+
+    def ex(opt, d=256, wsb=1 << 40):
+        return lib.rz_loss_fwd_bwd_ex(256, 512, 1024, 2048, 3072, 4096, 5120, 100, 4, 2, d, 4096,
+                                      ctypes.byref(opt), 6144, 7168, 8192, None, None, 1 << 20, wsb, None)
+
+    def seg_ex(opt, wsb=1 << 40):
+        return lib.rz_segment_loss_ex(256, 512, 768, 1024, 1280, 10, 2, 1, ctypes.byref(opt), 1536, 1792, None,
+                                      1 << 20, wsb, None)
+
+    for o in _bad_options(rz):
+        assert ex(o) == 1 and seg_ex(o) == 1
+        assert ex(o, d=96) == 1  # the options are checked before the shape
+    good = _opts(rz, flags=rz.RZ_LOSS_CLIP_IS | rz.RZ_LOSS_SEQ_GATE | rz.RZ_LOSS_TOKEN_MASK, clip_max=2.0,
+                 gate_lo=0.5, gate_hi=2.0, token_mask=4096, n_resp_total=7)
+    assert ex(good, d=96) == 2
+    assert ex(good, wsb=100) == 3 and seg_ex(good, wsb=10) == 3
+
+
+def test_host_checks_of_the_diagnostics(rz):
+    lib = rz.lib()
+    assert rz.rz_workspace_bytes_ratio_stats(0, 1) == 0 and rz.rz_workspace_bytes_ratio_stats(10, 0) == 0
+    assert rz.rz_workspace_bytes_ratio_stats(1 << 20, 100) > 0
+    assert rz.rz_workspace_bytes_grad_norms() >= 2 * 8 * 148
+
+    def stats(**kw):
+        a = dict(lp=256, lr=512, off=768, n=100, R=3, mask=None, out=1024, rm=None, ws=1 << 20, wsb=1 << 40)
+        a.update(kw)
+        return lib.rz_ratio_stats(a["lp"], a["lr"], a["off"], a["n"], a["R"], a["mask"], a["out"], a["rm"],
+                                  a["ws"], a["wsb"], None)
+
+    assert stats(n=0) == 1 and stats(R=0) == 1 and stats(lp=None) == 1 and stats(out=None) == 1
+    assert stats(off=772) == 1   # int64 offsets not 8-byte aligned
+    assert stats(out=1028) == 1  # fp64 outputs not 8-byte aligned
+    assert stats(rm=1026) == 1 and stats(ws=(1 << 20) + 64) == 1
+    assert stats(wsb=100) == 3
+
+    def norms(**kw):
+        a = dict(dH=256, dW=512, n=10, d=64, V=100, out=1024, ws=1 << 20, wsb=1 << 40)
+        a.update(kw)
+        return lib.rz_grad_norms(a["dH"], a["dW"], a["n"], a["d"], a["V"], a["out"], a["ws"], a["wsb"], None)
+
+    assert norms(n=-1) == 1 and norms(d=0) == 1 and norms(V=-1) == 1 and norms(out=None) == 1
+    assert norms(dH=None) == 1 and norms(dW=None) == 1 and norms(out=1028) == 1
+    assert norms(wsb=8) == 3
+
+
+def test_host_checks_of_the_fp8_forward(rz):
+    lib = rz.lib()
+    assert lib.rz_quantize_rows_e4m3(256, -1, 64, 512, 1024, None) == 1
+    assert lib.rz_quantize_rows_e4m3(256, 10, 0, 512, 1024, None) == 1
+    assert lib.rz_quantize_rows_e4m3(None, 0, 64, None, None, None) == 0   # no rows: a no-op
+    assert lib.rz_quantize_rows_e4m3(None, 10, 64, 512, 1024, None) == 1
+    assert lib.rz_quantize_rows_e4m3(256, 10, 64, 512, 1026, None) == 1    # scales not 4-byte aligned
+
+    def fwd(**kw):
+        a = dict(H=256, hs=512, W=1024, ws_=2048, ids=3072, n=100, d=256, V=4096, lp=4096 + 256, lse=None,
+                 ws=1 << 20, wsb=1 << 40)
+        a.update(kw)
+        return lib.rz_token_logprobs_fp8(a["H"], a["hs"], a["W"], a["ws_"], a["ids"], a["n"], a["d"], a["V"], a["lp"],
+                                         a["lse"], a["ws"], a["wsb"], None)
+
+    assert fwd(d=192) == 2 and fwd(d=100) == 2 and fwd(V=0) == 2  # d a multiple of 128
+    assert fwd(n=-1) == 1
+    assert fwd(n=0, H=None, hs=None, W=None, ws_=None, ids=None, lp=None, ws=None) == 0
+    assert fwd(H=None) == 1 and fwd(hs=None) == 1 and fwd(H=264) == 1 and fwd(ws_=2050) == 1
+    assert fwd(wsb=100) == 3
+
+
+def test_host_checks_of_the_shard_sum_selftest_noalloc_and_timed(rz):
+    import ctypes
+    lib = rz.lib()
+    assert lib.rz_sum_shards_f32(256, 0, 10, 512, None) == 1
+    assert lib.rz_sum_shards_f32(256, 2, -1, 512, None) == 1
+    assert lib.rz_sum_shards_f32(None, 2, 0, None, None) == 0   # nothing to sum
+    assert lib.rz_sum_shards_f32(None, 2, 10, 512, None) == 1
+    assert lib.rz_sum_shards_f32(256, 2, 10, 514, None) == 1
+
+    waited = ctypes.c_uint64(0)
+    assert lib.rz_selftest_wait_timeout(1000, None, 256, ctypes.byref(waited), None) == 1
+    assert lib.rz_selftest_wait_timeout(1000, 1 << 20, 100, ctypes.byref(waited), None) == 1
+    assert lib.rz_selftest_wait_timeout(10_000_000_001, 1 << 20, 256, ctypes.byref(waited), None) == 1
+    assert lib.rz_selftest_wait_timeout(1000, (1 << 20) + 16, 256, ctypes.byref(waited), None) == 1
+
+    def noalloc(**kw):
+        a = dict(H=256, W=512, ids=1024, n=100, d=256, V=4096, lp=2048, lse=None)
+        a.update(kw)
+        return lib.rz_token_logprobs_noalloc(a["H"], a["W"], a["ids"], a["n"], a["d"], a["V"], a["lp"], a["lse"],
+                                             None)
+
+    assert noalloc(n=-1) == 1 and noalloc(d=96) == 2
+    assert noalloc(n=0, H=None, W=None, ids=None, lp=None) == 0
+    assert noalloc(H=None) == 1 and noalloc(lp=2050) == 1
+    # beyond the fixed 32 MiB scratch: 4 n (2 ceil(V / 2048) + 1) bytes plus the status word
+    assert noalloc(n=1 << 20, V=151936) == 3
+
+    count = ctypes.c_int32(-5)
+    kinds = (ctypes.c_int32 * 4)()
+    events = (ctypes.c_void_p * 8)()
+
+    def timed(n=100, ev=events, cap=4):
+        return lib.rz_loss_fwd_bwd_timed(256, 512, 1024, 2048, 3072, 4096, 5120, n, 4, 2, 256, 4096, 6144, 7168,
+                                         8192, None, None, 1 << 20, 1 << 40, None, ev, kinds, cap,
+                                         ctypes.byref(count))
+
+    assert timed(ev=None) == 1 and timed(cap=-1) == 1
+    assert timed(n=0) == 1 and count.value == 0   # nothing recorded on an argument error
+    assert lib.rz_num_launches_loss(0) == 0
+    # 3 loss-stage launches, 6 per 16384-token chunk
+    assert [lib.rz_num_launches_loss(n) for n in (1, 16384, 16385)] == [9, 9, 15]
+    assert lib.rz_read_device_status(None, None, None) == 1
