@@ -1,6 +1,7 @@
 """The seeded input recipes (workloads.py) on CPU: each configuration's response structure,
 lengths, rewards and token count as stated in the workload table, determinism under its
-seed, the fp32 -> bf16 rounding, the lag noise, and whole-group truncation under a cap."""
+seed, the fp32 -> bf16 rounding, the lag noise, whole-group truncation under a cap, and the
+temperature-1 sampler's token frequencies."""
 import numpy as np
 import pytest
 
@@ -77,3 +78,21 @@ def test_token_cap_keeps_whole_groups():
     R = p.seg.seg_offsets.shape[0] - 1
     assert R % gs == 0 and R >= gs
     assert p.n_tok == int(p.seg.seg_offsets[-1])
+
+
+def test_sampler_draws_tokens_at_temperature_one():
+    """Gumbel-max: the frequency of each token for a repeated row matches softmax(z)."""
+    import torch
+    V, reps = 6, 30000
+    z_target = torch.tensor([0.0, 1.0, -1.0, 2.0, 0.5, -3.0])
+    # H = e_0 and W[:, 0] = z: the logits of every row are z (exact in bf16)
+    H = torch.zeros((reps, 8), dtype=torch.bfloat16)
+    H[:, 0] = 1.0
+    W = torch.zeros((V, 8), dtype=torch.bfloat16)
+    W[:, 0] = z_target.to(torch.bfloat16)
+    ids = wl.rollout_sample_ids(H, W, seed=5, chunk=4096)
+    freq = np.bincount(ids.numpy(), minlength=V) / reps
+    p = torch.softmax(z_target.double(), 0).numpy()
+    # binomial standard error at 30000 draws is below 0.003 for every p
+    assert np.all(np.abs(freq - p) < 5 * np.sqrt(p * (1 - p) / reps) + 1e-4), (freq, p)
+    assert np.array_equal(ids.numpy(), wl.rollout_sample_ids(H, W, seed=5, chunk=4096).numpy())
