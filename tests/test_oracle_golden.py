@@ -1,4 +1,4 @@
-"""Oracle regression record and an independent numpy restatement (CPU only).
+"""Oracle regression record, an independent numpy restatement and thread-count independence (CPU only).
 
 tiny_oracle.json was written by tests/golden/make_golden.py from the oracle alone; the
 test guards the oracle against silent drift.  The numpy restatement below is a second,
@@ -70,3 +70,33 @@ def test_numpy_restatement_agrees(oracle):
     for k in ("dH", "dW"):
         err = np.linalg.norm(out[k] - ref[k]) / np.linalg.norm(ref[k])
         assert err < 1e-12, (k, err)
+
+
+def test_oracle_results_do_not_depend_on_its_thread_count(tmp_path):
+    """The oracle parallelises over independent rows only (no reductions across threads),
+    so one thread and all threads give the same bits."""
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = (
+        "import sys, numpy as np, oracle, workloads as wl\n"
+        "p = wl.tiny()\n"
+        "lp, _ = oracle.token_logprobs(p.H, p.W, p.ids)\n"
+        "lr = wl.rollout_logprobs_with_lag(lp, p.noise, p.seed)\n"
+        "o = oracle.loss_fwd_bwd(p.H, p.W, p.ids, lr, p.seg.rewards, p.seg.seg_offsets, p.seg.group_ids,\n"
+        "                        p.seg.n_groups)\n"
+        "np.savez(sys.argv[1], loss=o['loss'], lp=o['lp'], kappa=o['kappa'], dH=o['dH'], dW=o['dW'],\n"
+        "         threads=oracle.num_threads())\n"
+    )
+    outs = {}
+    for threads in ("1", str(max(2, os.cpu_count() or 2))):
+        f = str(tmp_path / f"t{threads}.npz")
+        env = dict(os.environ, OMP_NUM_THREADS=threads, PYTHONPATH=root)
+        r = subprocess.run([sys.executable, "-c", code, f], cwd=root, env=env, capture_output=True, text=True,
+                           timeout=600)
+        assert r.returncode == 0, r.stderr[-2000:]
+        outs[threads] = np.load(f)
+    a, b = outs.values()
+    assert int(a["threads"]) == 1 and int(b["threads"]) > 1
+    for k in ("loss", "lp", "kappa", "dH", "dW"):
+        assert a[k].tobytes() == b[k].tobytes(), k
