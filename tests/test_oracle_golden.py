@@ -1,4 +1,4 @@
-"""Oracle regression record, an independent numpy restatement and thread-count independence (CPU only).
+"""Oracle regression record, a numpy restatement, thread-count independence (CPU only).
 
 tiny_oracle.json was written by tests/golden/make_golden.py from the oracle alone; the
 test guards the oracle against silent drift.  The numpy restatement below is a second,
