@@ -44,8 +44,13 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-loss-stage", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the other synthetic workloads (invariance head, lag64, moe_head at 2^20 tokens)")
     ap.add_argument("--sweep", action="store_true",
                     help="tokens-per-call sweep 2^12..2^20 of the workload (forward and forward+backward)")
+    ap.add_argument("--dp", action="store_true",
+                    help="data-parallel step: the one batch split into whole groups across the ranks, dW and the "
+                         "loss summed with the deterministic all-reduce (strong scaling)")
     ap.add_argument("--n-tok-cap", type=int, default=None,
                     help="keep only the leading whole groups that fit (small profiling cases)")
     return ap.parse_args()
@@ -357,6 +362,11 @@ def run_rz(args, rank, world, local_rank):
 
     peaks, peak_src = load_peaks()
     peak_tflops = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    other = None
+    if not args.no_workloads:
+        del ws, dH, dW
+        torch.cuda.empty_cache()
+        other = run_workloads(rz, torch, dev, stream, peak_tflops)
     tens = {k: v for k, v in per.items() if v["flops"] > 0}
     dom = max(tens, key=lambda k: tens[k]["ms"])
     ach = tens[dom]["flops"] / (tens[dom]["ms"] * 1e-3) / 1e12
@@ -378,7 +388,7 @@ def run_rz(args, rank, world, local_rank):
         dominant=dom, achieved=ach, peak=peak_tflops, peak_src=peak_src,
         traffic=traffic_for(dom, tens[dom]["rows"] / tens[dom]["launches"]),
         fwd_ms=fwd_ms, fwd_tok_s=world * n / (fwd_ms * 1e-3), launches=launches_total, e2e=e2e, cfg=cfg,
-        loss_stage=loss_stage, fwd8_ms=fwd8_ms, invariance=invariance,
+        loss_stage=loss_stage, fwd8_ms=fwd8_ms, invariance=invariance, workloads=other,
     )
 
 
@@ -504,15 +514,19 @@ def run_loss_stage(rz, torch, dev, stream, n_tok=1 << 26, reps=200):
 
 
 def run_e2e(rz, torch, dev, stream, H, W, ids, lp_roll, rewards, off, gid, G, n, d, V, args, world=1):
-    """The same step through the public call with inputs in pinned host memory: H2D of every
-    input and D2H of the loss and logprobs inside the timed region.  W and the small inputs
-    are copied first; H goes through rz_loss_fwd_bwd_streamed, which copies it chunk by chunk
-    on its own stream while the previous chunk computes."""
+    """The same step through the public calls from host inputs to host results: every input
+    copied host -> device and every result (dH, dW, lp, loss) device -> host inside the timed
+    region, all host buffers pinned.  W and the small inputs are copied first (the first
+    forward needs all of W); rz_loss_fwd_bwd_host_io copies H chunk by chunk on one stream and
+    each chunk's dH rows back on another while the next chunk computes, then dW after the
+    last chunk; lp and the loss follow."""
     host = {k: t.cpu().pin_memory() for k, t in
             dict(H=H, W=W, ids=ids, lp_roll=lp_roll, rewards=rewards, off=off, gid=gid).items()}
     dbuf = {k: torch.empty_like(t, device=dev) for k, t in host.items()}
     loss_h = torch.empty(1, dtype=torch.float32).pin_memory()
     lp_h = torch.empty(n, dtype=torch.float32).pin_memory()
+    dH_h = torch.empty((n, d), dtype=torch.bfloat16).pin_memory()
+    dW_h = torch.empty((V, d), dtype=torch.float32).pin_memory()
     R = rewards.shape[0]
     ws = torch.empty(rz.rz_workspace_bytes_loss(n, R, G, d, V), dtype=torch.uint8, device=dev)
     out = dict(loss=torch.empty(1, dtype=torch.float32, device=dev),
@@ -524,14 +538,16 @@ def run_e2e(rz, torch, dev, stream, H, W, ids, lp_roll, rewards, off, gid, G, n,
         for k in host:
             if k != "H":
                 dbuf[k].copy_(host[k], non_blocking=True)
-        rz.rz_loss_fwd_bwd_streamed(host["H"], dbuf["H"], dbuf["W"], dbuf["ids"], dbuf["lp_roll"], dbuf["rewards"],
-                                    dbuf["off"], dbuf["gid"], G, out=out, workspace=ws, stream=stream)
+        rz.rz_loss_fwd_bwd_host_io(host["H"], dbuf["H"], dbuf["W"], dbuf["ids"], dbuf["lp_roll"], dbuf["rewards"],
+                                   dbuf["off"], dbuf["gid"], G, dH_host=dH_h, dW_host=dW_h, out=out, workspace=ws,
+                                   stream=stream)
         loss_h.copy_(out["loss"], non_blocking=True)
         lp_h.copy_(out["lp"], non_blocking=True)
 
     for _ in range(1):
         step()
     torch.cuda.synchronize()
+    ok = bool(torch.equal(dW_h.view(torch.int32), out["dW"].cpu().view(torch.int32)))
     steps = max(2, min(args.steps, 3))
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
@@ -544,9 +560,161 @@ def run_e2e(rz, torch, dev, stream, H, W, ids, lp_roll, rewards, off, gid, G, n,
     if world > 1:  # every rank copies its own inputs: the job's time is the slowest rank's
         ms = max_over_ranks(ms, dev)
     h2d = world * sum(t.numel() * t.element_size() for t in host.values())
-    d2h = world * (loss_h.numel() * 4 + lp_h.numel() * 4)
+    d2h = world * sum(t.numel() * t.element_size() for t in (loss_h, lp_h, dH_h, dW_h))
     return {"value": world * n / (ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
-            "d2h_bytes_per_step": int(d2h), "ms_per_step": ms, "bytes_note": "summed over all ranks"}
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": ms, "host_results_equal_device": ok,
+            "bytes_note": "summed over all ranks; in: H, W, ids, lp_rollout, rewards, offsets, group ids; "
+                          "out: dH, dW, lp, loss"}
+
+
+def _time_calls(torch, stream, fn, reps, warm=1):
+    """Mean milliseconds per call of fn() over `reps` calls (CUDA events on `stream`)."""
+    for _ in range(warm):
+        fn()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def run_workloads(rz, torch, dev, stream, peak_tflops):
+    """The other synthetic workloads, each through the same public calls as the headline:
+    - invariance (d=1536, V=151936): the forward over its 4096 rows in one call, and the
+      decode-shaped calls of 1 and 64 rows it is also checked with (microseconds per call);
+    - lag64 (d=2560, V=151936, 256 responses of 1K-16K tokens, all ~1.44M tokens): forward
+      alone and forward + loss + backward;
+    - moe_head (d=7168, V=129280) at 2^20 tokens (the largest call of its sweep): the same.
+    Tensor fractions are against the sustained bf16 peak: 2dV FLOP per token forward, 6dV
+    forward + loss + backward."""
+    import workloads as wl
+    res = {}
+    cfg = wl.CONFIGS["invariance"]
+    d, V = cfg["d"], cfg["V"]
+    H, W = wl.draw_matrices(cfg["n_rows"], d, V, cfg["seed"], device=str(dev))
+    ids = torch.from_numpy(wl.draw_uniform_ids(cfg["n_rows"], V, cfg["seed"])).to(dev)
+    n = H.shape[0]
+    lp = torch.empty(n, dtype=torch.float32, device=dev)
+    ws = torch.empty(rz.rz_workspace_bytes_logprobs(n, d, V), dtype=torch.uint8, device=dev)
+    ms = _time_calls(torch, stream, lambda: rz.rz_token_logprobs(H, W, ids, lp_out=lp, workspace=ws, stream=stream,
+                                                                  want_lse=False), 20, 3)
+    ent = {"fwd_tok_s": n / (ms * 1e-3), "fwd_frac": n * 2 * d * V / (ms * 1e-3) / (peak_tflops * 1e12)}
+    for rows in (1, 64):
+        ms_r = _time_calls(torch, stream, lambda: rz.rz_token_logprobs(
+            H[:rows], W, ids[:rows], lp_out=lp[:rows], workspace=ws, stream=stream, want_lse=False), 50, 3)
+        ent[f"us_per_call_{rows}_rows"] = ms_r * 1e3
+    res["invariance_d1536"] = ent
+    del H, W, ids, lp, ws
+
+    for name, cap in (("lag64", None), ("moe_head", 1 << 20)):
+        prob = wl.full_config(name, device=str(dev), n_tok_cap=cap)
+        seg = prob.seg
+        n, d, V = prob.n_tok, prob.d, prob.V
+        lp0, _ = rz.rz_token_logprobs(prob.H, prob.W, prob.ids, want_lse=False)
+        torch.cuda.synchronize()
+        lr = torch.from_numpy(wl.rollout_logprobs_with_lag(lp0.cpu().numpy(), prob.noise, prob.seed)).to(dev)
+        t_r = torch.from_numpy(seg.rewards).to(dev)
+        t_off = torch.from_numpy(seg.seg_offsets).to(dev)
+        t_gid = torch.from_numpy(seg.group_ids).to(dev)
+        out = dict(loss=torch.empty(1, device=dev), dH=torch.empty((n, d), dtype=torch.bfloat16, device=dev),
+                   dW=torch.empty((V, d), dtype=torch.float32, device=dev))
+        ws = torch.empty(rz.rz_workspace_bytes_loss(n, seg.n_resp, seg.n_groups, d, V), dtype=torch.uint8,
+                         device=dev)
+        wsf = torch.empty(rz.rz_workspace_bytes_logprobs(n, d, V), dtype=torch.uint8, device=dev)
+        ms_f = _time_calls(torch, stream, lambda: rz.rz_token_logprobs(prob.H, prob.W, prob.ids, lp_out=lp0,
+                                                                        workspace=wsf, stream=stream,
+                                                                        want_lse=False), 2)
+        ms_b = _time_calls(torch, stream, lambda: rz.rz_loss_fwd_bwd(
+            prob.H, prob.W, prob.ids, lr, t_r, t_off, t_gid, seg.n_groups, loss=out["loss"], dH=out["dH"],
+            dW=out["dW"], want_lp=False, want_kappa=False, workspace=ws, stream=stream), 2)
+        code, _ = rz.rz_read_device_status(ws)
+        res[f"{name}_{n}_tok"] = {
+            "d": d, "V": V, "n_resp": seg.n_resp, "status_ok": code == 0,
+            "fwd_tok_s": n / (ms_f * 1e-3), "fwd_frac": n * 2 * d * V / (ms_f * 1e-3) / (peak_tflops * 1e12),
+            "fwd_bwd_tok_s": n / (ms_b * 1e-3),
+            "fwd_bwd_frac_6dV": n * 6 * d * V / (ms_b * 1e-3) / (peak_tflops * 1e12)}
+        del prob, lr, out, ws, wsf, lp0
+        torch.cuda.empty_cache()
+    return res
+
+
+def dp_shard(seg, world: int, rank: int):
+    """This rank's part of the batch for the data-parallel mode: whole groups balanced by
+    tokens (dp.shard_groups), with the global response count every rank's N must use."""
+    from invariant_logprobs_reinforce_b200 import dp
+    sh = dp.shard_groups(seg.seg_offsets, seg.group_ids, world)[rank]
+    rewards = seg.rewards[sh["resp_lo"]:sh["resp_hi"]].copy()
+    return sh, rewards, seg.n_resp
+
+
+def run_dp(args, rank, world, local_rank):
+    """The data-parallel step over one batch of the workload: rank r takes its shard of whole
+    groups and runs dp.dp_loss_fwd_bwd (the shard through rz_loss_fwd_bwd_ex with N = the
+    global response count, then the deterministic all-reduce of dW and the loss: all-to-all,
+    rank-order fp64 sum in librz, all-gather).  Timed on the device, max over ranks; value =
+    the batch's tokens / that time.  Also checks that every rank ends with the same dW bits."""
+    import torch
+    import torch.distributed as tdist
+    import workloads as wl
+    import invariant_logprobs_reinforce_b200 as rz
+    from invariant_logprobs_reinforce_b200 import build as rzbuild
+    from invariant_logprobs_reinforce_b200 import dp
+    rzbuild.build()
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream()
+    prob = wl.full_config(args.workload, device=str(dev), n_tok_cap=args.n_tok_cap)
+    seg = prob.seg
+    d, V = prob.d, prob.V
+    lp0, _ = rz.rz_token_logprobs(prob.H, prob.W, prob.ids, want_lse=False)
+    torch.cuda.synchronize()
+    lr_all = torch.from_numpy(wl.rollout_logprobs_with_lag(lp0.cpu().numpy(), prob.noise, prob.seed)).to(dev)
+    sh, rewards, n_total = dp_shard(seg, world, rank)
+    t0, t1 = sh["tok_lo"], sh["tok_hi"]
+    H, ids, lr = prob.H[t0:t1].contiguous(), prob.ids[t0:t1].contiguous(), lr_all[t0:t1].contiguous()
+    t_r = torch.from_numpy(rewards).to(dev)
+    t_off = torch.from_numpy(sh["seg_offsets"]).to(dev)
+    t_gid = torch.from_numpy(sh["group_ids"]).to(dev)
+    n = t1 - t0
+    ws = torch.empty(rz.rz_workspace_bytes_loss(n, rewards.shape[0], sh["n_groups"], d, V), dtype=torch.uint8,
+                     device=dev)
+
+    def step():
+        return dp.dp_loss_fwd_bwd(H, prob.W, ids, lr, t_r, t_off, t_gid, sh["n_groups"], workspace=ws,
+                                  n_resp_total=n_total)
+
+    for _ in range(args.warmup):
+        out = step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.5)
+    tdist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        out = step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    tdist.barrier()
+    clk = clocks.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1), dev) / args.steps
+    code, bits = rz.rz_read_device_status(ws)
+    # the same dW bits on every rank: compare a checksum of the bit patterns
+    csum = torch.tensor([int(out["dW"].view(torch.int32).to(torch.int64).sum().item()),
+                         int(out["loss"].view(torch.int32).item())], dtype=torch.int64, device=dev)
+    allsums = [torch.empty_like(csum) for _ in range(world)]
+    tdist.all_gather(allsums, csum)
+    same = all(torch.equal(allsums[0], x) for x in allsums)
+    launches = rz.rz_num_launches_loss(n) + 2  # + the rank-order sums of dW and the loss
+    return dict(value=seg.n_tok / (ms * 1e-3), ms_per_step=ms, n_tok=seg.n_tok, shard_tokens=n, d=d, V=V,
+                status_ok=code == 0 and bits == 0, dW_same_bits_on_all_ranks=same, clocks=clk,
+                launches=int(max_over_ranks(float(launches * args.steps), dev)), n_resp=seg.n_resp,
+                n_groups=seg.n_groups)
 
 
 # --------------------------------------------------------------------------- sweep
@@ -692,6 +860,88 @@ def run_reference(args, rank, world):
     return line
 
 
+def _round(x, sig=4):
+    """Floats rounded to `sig` significant digits (nested), to keep the line short."""
+    if isinstance(x, float):
+        return float(f"{x:.{sig}g}") if math.isfinite(x) else x
+    if isinstance(x, dict):
+        return {k: _round(v, sig) for k, v in x.items()}
+    if isinstance(x, (list, tuple)):
+        return [_round(v, sig) for v in x]
+    return x
+
+
+def make_line(args, world, res, cpu):
+    """The JSON line: the contract's keys first, the detailed records next, and the compact
+    headline figures last (a consumer that keeps only the end of the output still has them)."""
+    cfg = res["cfg"]
+    peak = res["peak"]
+    frac = res["achieved"] / peak
+    d, V, n = res["d"], res["V"], res["n_tok"]
+    line = {
+        "metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {
+            "workload": f"{args.workload}: d={d}, V={V}, {res['G']} groups x {res['R'] // res['G']} responses, "
+                        f"lengths {cfg['lengths'][0]} {cfg['lengths'][1]}-{cfg['lengths'][2]}, n_tok={n} per GPU",
+            "n_tok": n, "d": d, "V": V, "n_resp": res["R"], "n_groups": res["G"],
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "inputs larger than L2 (H %.2f GB, W %.2f GB)" % (n * d * 2 / 1e9, V * d * 2 / 1e9),
+        },
+        "roofline": {"bound": "tensor", "kernel": res["dominant"], "achieved": res["achieved"], "peak": peak,
+                     "unit": "TFLOP/s", "frac": frac, "traffic": res["traffic"],
+                     "peak_source": f"bf16_tflops_sustained of {res['peak_src']}"},
+        "clocks": res["clocks"],
+        "gpu_launches": res["launches"],
+        "e2e": res["e2e"],
+        "cpu_baseline": cpu,
+        # detailed records
+        "kernels": _round(res["kernels"]),
+        "batch_invariance": res["invariance"],
+        "loss_stage": _round(res["loss_stage"]),
+        # compact headline figures, last
+        "tensor_frac_6dV": _round(res["value"] / world * 6 * d * V / (peak * 1e12)),
+        "fwd_only": _round({"tokens_per_s": res["fwd_tok_s"], "ms_per_step": res["fwd_ms"],
+                            "tensor_frac_2dV": res["fwd_tok_s"] / world * 2 * d * V / (peak * 1e12)}),
+        "fwd_only_fp8": _round({"tokens_per_s": n * world / (res["fwd8_ms"] * 1e-3), "ms_per_step": res["fwd8_ms"],
+                                "tensor_frac_2dV": n * 2 * d * V / (res["fwd8_ms"] * 1e-3) / (2 * peak * 1e12),
+                                "peak": "2 x sustained bf16 (nominal e4m3 ratio)"}),
+    }
+    ls = res["loss_stage"]
+    if ls is not None:
+        line["loss_stage_frac"] = _round({"segment_loss": ls["frac"], "clip_mask": ls["variant_clip_mask"]["frac"],
+                                          "ratio_stats": ls["ratio_stats"]["frac"], "sm_mhz": ls["sm_mhz"]})
+    line["workloads"] = _round(res["workloads"])
+    return line
+
+
+def make_dp_line(args, world, r):
+    """The JSON line of the data-parallel mode (strong scaling over one fixed batch)."""
+    return {
+        "metric": METRIC, "value": r["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{args.workload}: d={r['d']}, V={r['V']}, {r['n_resp']} responses in "
+                               f"{r['n_groups']} groups, n_tok={r['n_tok']} for the whole job",
+                   "parallelism": f"data-parallel x{world}: whole groups per rank, dW and loss summed by a "
+                                  f"deterministic all-reduce (all-to-all, rank-order fp64 sum, all-gather)",
+                   "shard_tokens_rank0": r["shard_tokens"]},
+        "clocks": r["clocks"], "gpu_launches": r["launches"], "status_ok": r["status_ok"],
+        "dW_same_bits_on_all_ranks": r["dW_same_bits_on_all_ranks"],
+        "roofline": None, "e2e": None, "cpu_baseline": None,
+        "note": "the data-parallel mode reports throughput and cross-rank consistency; the default mode "
+                "carries the roofline, e2e and cpu_baseline",
+    }
+
+
+def free_port() -> int:
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
 # --------------------------------------------------------------------------- main
 
 def main():
@@ -710,53 +960,32 @@ def main():
             print(json.dumps({"sweep": run_sweep(args, local_rank)}), flush=True)
         return 0
 
-    if world > 1:
+    if world > 1 or args.dp:
         import datetime
         import torch
         import torch.distributed as tdist
         torch.cuda.set_device(local_rank)
-        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+        if world == 1:  # a one-rank group for the data-parallel mode on one GPU
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            os.environ.setdefault("MASTER_PORT", str(free_port()))
+            os.environ.setdefault("RANK", "0")
+            os.environ.setdefault("WORLD_SIZE", "1")
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                  device_id=torch.device("cuda", local_rank))
+    if args.dp:
+        r = run_dp(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(make_dp_line(args, world, r)), flush=True)
+        import torch.distributed as tdist
+        tdist.barrier()
+        tdist.destroy_process_group()
+        return 0
     res = run_rz(args, rank, world, local_rank)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_sample(args.workload)
     if rank == 0:
-        cfg = res["cfg"]
-        frac = res["achieved"] / res["peak"]
-        line = {
-            "metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {
-                "workload": f"{args.workload}: d={res['d']}, V={res['V']}, {res['G']} groups x "
-                            f"{res['R'] // res['G']} responses, lengths {cfg['lengths'][0]} "
-                            f"{cfg['lengths'][1]}-{cfg['lengths'][2]}, n_tok={res['n_tok']} per GPU",
-                "n_tok": res["n_tok"], "d": res["d"], "V": res["V"], "n_resp": res["R"], "n_groups": res["G"],
-                "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                "l2": "inputs larger than L2 (H %.2f GB, W %.2f GB)" % (res["n_tok"] * res["d"] * 2 / 1e9,
-                                                                      res["V"] * res["d"] * 2 / 1e9),
-            },
-            "roofline": {"bound": "tensor", "kernel": res["dominant"], "achieved": res["achieved"],
-                         "peak": res["peak"], "unit": "TFLOP/s", "frac": frac, "traffic": res["traffic"],
-                         "peak_source": f"bf16_tflops_sustained of {res['peak_src']}"},
-            "tensor_frac_6dV": res["value"] / world * 6 * res["d"] * res["V"] / (res["peak"] * 1e12),
-            "fwd_only": {"tokens_per_s": res["fwd_tok_s"], "ms_per_step": res["fwd_ms"],
-                         "tensor_frac_2dV": res["fwd_tok_s"] / world * 2 * res["d"] * res["V"] / (res["peak"] * 1e12)},
-            "fwd_only_fp8": {"tokens_per_s": res["n_tok"] * world / (res["fwd8_ms"] * 1e-3),
-                             "ms_per_step": res["fwd8_ms"],
-                             "tensor_frac_2dV": res["n_tok"] * 2 * res["d"] * res["V"] / (res["fwd8_ms"] * 1e-3)
-                             / (2 * res["peak"] * 1e12),
-                             "peak_note": "e4m3 peak = 2 x the measured sustained bf16 peak (nominal ratio)"},
-            "batch_invariance": res["invariance"],
-            "kernels": res["kernels"],
-            "loss_stage": res["loss_stage"],
-            "gpu_launches": res["launches"],
-            "clocks": res["clocks"],
-            "e2e": res["e2e"],
-            "cpu_baseline": cpu,
-        }
-        print(json.dumps(line), flush=True)
+        print(json.dumps(make_line(args, world, res, cpu)), flush=True)
     if world > 1:
         import torch.distributed as tdist
         tdist.barrier()

@@ -209,6 +209,30 @@ rz_status rz_loss_fwd_bwd_streamed(const rz_bf16* H_host, rz_bf16* H_dev, const 
                                    const rz_loss_options* options, float* loss, rz_bf16* dH, float* dW,
                                    float* lp_out, float* kappa_out, void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * rz_loss_fwd_bwd_streamed with the gradients also delivered to HOST memory: the whole step
+ * from host inputs to host results, for a trainer that keeps activations and gradients in
+ * host memory.  On top of the streamed call, each 16384-token chunk's rows of dH are copied
+ * to dH_host right after that chunk's dH contraction (on a device-to-host stream of its own,
+ * one per device, created on first use, so the copy of chunk c overlaps the compute of
+ * chunk c + 1 and the host-to-device copy of the next chunk's H), and dW to dW_host after
+ * the last chunk's dW contraction.  Every copy is finished before any work enqueued on
+ * `stream` after this call starts, so a stream synchronisation after the call means the
+ * host buffers hold the results.
+ *
+ *   dH_host  host, [n_tok, d] bf16, nullable (no dH copy); pinned for the copies to overlap
+ *   dW_host  host, [V, d] fp32, nullable (no dW copy); pinned for the copy to run asynchronously
+ *   every other argument as rz_loss_fwd_bwd_streamed (dH and dW still receive the device copies).
+ * Errors: as rz_loss_fwd_bwd_streamed, plus RZ_ERR_CUDA when the device-to-host stream, its
+ * event or a copy cannot be created or enqueued.
+ */
+rz_status rz_loss_fwd_bwd_host_io(const rz_bf16* H_host, rz_bf16* H_dev, const rz_bf16* W_head,
+                                  const int32_t* token_ids, const float* lp_rollout, const float* rewards,
+                                  const int64_t* seg_offsets, const int32_t* group_ids, int64_t n_tok, int32_t n_resp,
+                                  int32_t n_groups, int32_t d, int32_t V, const rz_loss_options* options,
+                                  float* loss, rz_bf16* dH, float* dW, float* lp_out, float* kappa_out,
+                                  rz_bf16* dH_host, float* dW_host, void* workspace, size_t ws_bytes, void* stream);
+
 /* rz_segment_loss with loss-stage options (same workspace size). */
 rz_status rz_segment_loss_ex(const float* lp, const float* lp_rollout, const float* rewards,
                              const int64_t* seg_offsets, const int32_t* group_ids, int64_t n_tok, int32_t n_resp,
@@ -295,15 +319,17 @@ rz_status rz_selftest_wait_timeout(uint64_t limit_ns, void* workspace, size_t ws
 /* Kernel kinds reported per launch by rz_loss_fwd_bwd_timed. */
 #define RZ_KERNEL_LMHEAD_LSE 0    /* fused LM head + online log-sum-exp + gather (tensor cores) */
 #define RZ_KERNEL_MERGE_LSE 1     /* fixed-order merge of the vocabulary-segment partials       */
-#define RZ_KERNEL_RESPONSE_COEF 2 /* group means and -A_i / (N L_i)                             */
-#define RZ_KERNEL_TOKEN_KAPPA 3   /* ratio and kappa per token, per-block loss partials          */
-#define RZ_KERNEL_LOSS_FINAL 4    /* fixed-order sum of the loss partials                        */
-#define RZ_KERNEL_DZ 5            /* recomputed logits -> dZ chunk (tensor cores)                */
+#define RZ_KERNEL_RESPONSE_COEF 2 /* loss setup: checks, group means, -A_i / (N L_i), block starts */
+#define RZ_KERNEL_TOKEN_KAPPA 3   /* ratio and kappa per token, loss partials; the call's last
+                                     block also sums the partials into the loss                 */
+#define RZ_KERNEL_LOSS_FINAL 4    /* not reported: the loss is summed inside RZ_KERNEL_TOKEN_KAPPA */
+#define RZ_KERNEL_DZ 5            /* kept exponentials -> dZ chunk in place (HBM pass)           */
 #define RZ_KERNEL_DH 6            /* dH chunk = dZ W (tensor cores)                              */
 #define RZ_KERNEL_DW 7            /* dW (+)= dZ^T H (tensor cores)                               */
-#define RZ_KERNEL_BLOCK_FIRST 8   /* first response of each 4096-token block of the loss stage   */
+#define RZ_KERNEL_BLOCK_FIRST 8   /* not reported: the block starts come from RZ_KERNEL_RESPONSE_COEF */
 
-/* Number of kernel launches one rz_loss_fwd_bwd call makes for n_tok tokens (0 if n_tok < 1). */
+/* Number of launches rz_loss_fwd_bwd_timed records for n_tok tokens (0 if n_tok < 1): the
+ * loss setup, then six per 16384-token chunk (forward, merge, kappa, dZ, dH, dW). */
 int32_t rz_num_launches_loss(int64_t n_tok);
 
 /*
@@ -343,16 +369,38 @@ rz_status rz_loss_fwd_bwd_timed(const rz_bf16* H, const rz_bf16* W_head, const i
  * RZ_ERR_WORKSPACE_TOO_SMALL and enqueue nothing; split them into several calls.
  *
  * The first call on each device looks up the scratch address (cudaGetSymbolAddress)
- * and caches it; make that first call before any stream capture begins.  All calls
- * share the one array: calls whose GPU work can overlap (different streams, or
- * different host threads) race on it and must be serialised by the caller.  Each call
- * clears the scratch's status word; out-of-range token ids still give NaN logprobs,
- * but the status word is internal (rz_read_device_status does not apply).  Nothing
- * here calls cudaMalloc, cudaFree or any allocating routine.
+ * and caches it with the device's CUDA context; make that first call before any stream
+ * capture begins.  If the context is destroyed and recreated (cudaDeviceReset, or a
+ * released primary context), the next call sees the new context and looks the address
+ * up again, so make that call outside a capture as well.  The device that is current when
+ * the call is made must be the one that holds H, W_head, token_ids and the outputs, and
+ * `stream` must belong to it.  All calls share the one array: calls whose GPU work can
+ * overlap (different streams, or different host threads) race on it and must be
+ * serialised by the caller.  Each call clears the scratch's status word.  The status word
+ * is internal (rz_read_device_status does not apply), so problems show in the outputs:
+ * an out-of-range token id gives that row a NaN logprob, and a kernel wait that gave up
+ * gives NaN in every lp and lse of the call.  Nothing here calls cudaMalloc, cudaFree or
+ * any allocating routine.
  */
 rz_status rz_token_logprobs_noalloc(const rz_bf16* H, const rz_bf16* W_head, const int32_t* token_ids,
                                     int64_t n_tok, int32_t d, int32_t V, float* lp_out, float* lse_out,
                                     void* stream);
+
+/*
+ * Self-test of what a forward call returns after one of its waits gave up.  Runs
+ * rz_token_logprobs on `workspace` (use_noalloc_scratch == 0) or rz_token_logprobs_noalloc
+ * (use_noalloc_scratch != 0; workspace and ws_bytes are ignored) with one extra bounded
+ * wait, on a barrier nothing arrives on and with a 1 ms limit, enqueued right after the
+ * call clears its status word.  That wait gives up and sets RZ_DEV_WAIT_TIMEOUT exactly as
+ * a wait inside the forward's kernels would; the forward then runs normally and its merge,
+ * seeing the bit, writes NaN to every lp_out and lse_out (nullable) element.  With a
+ * workspace, rz_read_device_status then returns RZ_ERR_DEVICE_TIMEOUT.  Arguments, checks
+ * and errors otherwise as the call it runs.  No GPU fault or hang is involved.
+ */
+rz_status rz_selftest_forward_after_timeout(int32_t use_noalloc_scratch, const rz_bf16* H, const rz_bf16* W_head,
+                                            const int32_t* token_ids, int64_t n_tok, int32_t d, int32_t V,
+                                            float* lp_out, float* lse_out, void* workspace, size_t ws_bytes,
+                                            void* stream);
 
 /*
  * Synchronises `stream`, then reads the device status word of `workspace`.

@@ -8,6 +8,7 @@ librz.so is missing or no CUDA device is present, the calls raise.
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 
 from .build import LIB as _LIB_PATH
@@ -16,9 +17,10 @@ __all__ = [
     "RZ_OK", "RZError", "lib", "rz_status_string", "rz_workspace_bytes_logprobs", "rz_workspace_bytes_loss",
     "rz_workspace_bytes_segment_loss", "rz_token_logprobs", "rz_loss_fwd_bwd", "rz_segment_loss",
     "rz_read_device_status", "rz_num_launches_loss", "rz_loss_fwd_bwd_timed", "rz_loss_fwd_bwd_ex",
-    "rz_loss_fwd_bwd_streamed", "rz_segment_loss_ex", "rz_ratio_stats", "rz_grad_norms", "rz_quantize_rows_e4m3",
+    "rz_loss_fwd_bwd_streamed", "rz_loss_fwd_bwd_host_io", "rz_segment_loss_ex", "rz_ratio_stats", "rz_grad_norms", "rz_quantize_rows_e4m3",
     "rz_token_logprobs_fp8", "rz_sum_shards_f32", "rz_selftest_wait_timeout", "rz_token_logprobs_noalloc",
-    "rz_workspace_bytes_ratio_stats", "rz_workspace_bytes_grad_norms", "rz_loss_options", "loss_options",
+    "rz_workspace_bytes_ratio_stats", "rz_workspace_bytes_grad_norms", "rz_selftest_forward_after_timeout",
+    "rz_loss_options", "loss_options",
     "EXPORTED_SYMBOLS", "STAT_NAMES", "KERNEL_KINDS",
 ]
 
@@ -31,9 +33,11 @@ EXPORTED_SYMBOLS = (
     "rz_status_string", "rz_workspace_bytes_logprobs", "rz_workspace_bytes_loss", "rz_workspace_bytes_segment_loss",
     "rz_token_logprobs", "rz_loss_fwd_bwd", "rz_segment_loss", "rz_read_device_status", "rz_num_launches_loss",
     "rz_loss_fwd_bwd_timed", "rz_token_logprobs_noalloc", "rz_loss_fwd_bwd_ex", "rz_loss_fwd_bwd_streamed",
+    "rz_loss_fwd_bwd_host_io",
     "rz_segment_loss_ex",
     "rz_workspace_bytes_ratio_stats", "rz_ratio_stats", "rz_workspace_bytes_grad_norms", "rz_grad_norms",
     "rz_quantize_rows_e4m3", "rz_token_logprobs_fp8", "rz_sum_shards_f32", "rz_selftest_wait_timeout",
+    "rz_selftest_forward_after_timeout",
 )
 RZ_LOSS_CLIP_IS, RZ_LOSS_SEQ_GATE, RZ_LOSS_TOKEN_MASK = 1, 2, 4
 STAT_NAMES = ("k1", "k2", "k3", "w_min", "w_max", "dev_max", "dev_median", "dev_peak_over_median", "count")
@@ -113,6 +117,9 @@ def lib() -> ctypes.CDLL:
         L.rz_loss_fwd_bwd_streamed.argtypes = [P, P, P, P, P, P, P, P, i64, i32, i32, i32, i32,
                                                 ctypes.POINTER(rz_loss_options), P, P, P, P, P, P, sz, P]
         L.rz_loss_fwd_bwd_streamed.restype = ctypes.c_int
+        L.rz_loss_fwd_bwd_host_io.argtypes = [P, P, P, P, P, P, P, P, i64, i32, i32, i32, i32,
+                                               ctypes.POINTER(rz_loss_options), P, P, P, P, P, P, P, P, sz, P]
+        L.rz_loss_fwd_bwd_host_io.restype = ctypes.c_int
         L.rz_segment_loss_ex.argtypes = [P, P, P, P, P, i64, i32, i32, ctypes.POINTER(rz_loss_options), P, P, P, P,
                                           sz, P]
         L.rz_segment_loss_ex.restype = ctypes.c_int
@@ -132,6 +139,8 @@ def lib() -> ctypes.CDLL:
         L.rz_sum_shards_f32.restype = ctypes.c_int
         L.rz_selftest_wait_timeout.argtypes = [ctypes.c_uint64, P, sz, ctypes.POINTER(ctypes.c_uint64), P]
         L.rz_selftest_wait_timeout.restype = ctypes.c_int
+        L.rz_selftest_forward_after_timeout.argtypes = [i32, P, P, P, i64, i32, i32, P, P, P, sz, P]
+        L.rz_selftest_forward_after_timeout.restype = ctypes.c_int
         L.rz_read_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_int32)]
         L.rz_read_device_status.restype = ctypes.c_int
         _lib = L
@@ -174,10 +183,28 @@ def _ptr(t):
 
 
 def _stream_handle(stream):
+    """The stream to enqueue on: `stream`, else the current stream of the current device
+    (the entry points make the tensors' device current first, see _on_tensor_device)."""
     torch = _torch()
     if stream is None:
         stream = torch.cuda.current_stream()
+    elif stream.device != torch.device("cuda", torch.cuda.current_device()):
+        raise ValueError(f"stream is on {stream.device}, the tensors on cuda:{torch.cuda.current_device()}")
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _on_tensor_device(fn):
+    """Run an entry point with the device of its first CUDA tensor argument current: the
+    library launches on the current device, which must be the one that holds the data."""
+    @functools.wraps(fn)
+    def wrapper(*args, **kwargs):
+        torch = _torch()
+        for a in (*args, *kwargs.values()):
+            if isinstance(a, torch.Tensor) and a.is_cuda:
+                with torch.cuda.device(a.device):
+                    return fn(*args, **kwargs)
+        return fn(*args, **kwargs)
+    return wrapper
 
 
 def _need(t, dtype, name, device=None):
@@ -287,6 +314,7 @@ def _check(code, what):
 
 # ----------------------------------------------------------------------------- entry points
 
+@_on_tensor_device
 def rz_token_logprobs(H, W_head, token_ids, lp_out=None, lse_out=None, workspace=None, stream=None,
                       want_lse=True):
     """Token logprobs of the sampled tokens (bf16 H [n,d], bf16 W [V,d], int32 ids [n]).
@@ -313,6 +341,7 @@ def rz_token_logprobs(H, W_head, token_ids, lp_out=None, lse_out=None, workspace
     return lp, lse
 
 
+@_on_tensor_device
 def rz_token_logprobs_noalloc(H, W_head, token_ids, lp_out, lse_out=None, stream=None):
     """rz_token_logprobs from the library's fixed scratch instead of a workspace: the caller
     passes every output buffer, and neither this wrapper nor the library allocates.  Calls
@@ -334,6 +363,7 @@ def rz_token_logprobs_noalloc(H, W_head, token_ids, lp_out, lse_out=None, stream
     return lp_out, lse_out
 
 
+@_on_tensor_device
 def rz_loss_fwd_bwd(H, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids, n_groups, loss=None,
                     dH=None, dW=None, lp_out=None, kappa_out=None, workspace=None, stream=None, want_lp=True,
                     want_kappa=True):
@@ -362,6 +392,7 @@ def rz_num_launches_loss(n_tok: int) -> int:
     return int(lib().rz_num_launches_loss(n_tok))
 
 
+@_on_tensor_device
 def rz_loss_fwd_bwd_timed(events, H, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids, n_groups,
                           loss, dH, dW, lp_out, kappa_out, workspace, stream=None):
     """rz_loss_fwd_bwd recording a CUDA event pair around every kernel launch.
@@ -388,6 +419,7 @@ def rz_loss_fwd_bwd_timed(events, H, W_head, token_ids, lp_rollout, rewards, seg
     return [int(kinds[i]) for i in range(count.value)]
 
 
+@_on_tensor_device
 def rz_segment_loss(lp, lp_rollout, rewards, seg_offsets, group_ids, n_groups, loss=None, kappa_out=None,
                     w_out=None, want_w=False, workspace=None, stream=None):
     """The loss stage alone from given logprobs.  Returns dict(loss, kappa, w, workspace)."""
@@ -409,6 +441,7 @@ def rz_segment_loss(lp, lp_rollout, rewards, seg_offsets, group_ids, n_groups, l
     return dict(loss=loss, kappa=kappa_out, w=w_out, workspace=ws)
 
 
+@_on_tensor_device
 def rz_read_device_status(workspace, stream=None):
     """Synchronise the stream and return (status code, raw RZ_DEV_* bits) of a workspace."""
     bits = ctypes.c_int32(0)
@@ -416,6 +449,7 @@ def rz_read_device_status(workspace, stream=None):
     return int(code), int(bits.value)
 
 
+@_on_tensor_device
 def rz_loss_fwd_bwd_ex(H, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids, n_groups, options,
                        workspace=None, stream=None):
     """rz_loss_fwd_bwd with rz_loss_options (see loss_options).  Returns the same dict."""
@@ -437,6 +471,7 @@ def rz_loss_fwd_bwd_ex(H, W_head, token_ids, lp_rollout, rewards, seg_offsets, g
     return out
 
 
+@_on_tensor_device
 def rz_loss_fwd_bwd_streamed(H_host, H_dev, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids, n_groups,
                              options=None, out=None, workspace=None, stream=None):
     """rz_loss_fwd_bwd_ex with H read from host memory (H_host: CPU bf16 tensor, pinned for the copies to
@@ -470,6 +505,51 @@ def rz_loss_fwd_bwd_streamed(H_host, H_dev, W_head, token_ids, lp_rollout, rewar
     return out
 
 
+@_on_tensor_device
+def rz_loss_fwd_bwd_host_io(H_host, H_dev, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids, n_groups,
+                            dH_host=None, dW_host=None, options=None, out=None, workspace=None, stream=None):
+    """rz_loss_fwd_bwd_streamed that also copies the gradients to host memory: dH_host (CPU bf16 [n, d]) chunk by
+    chunk as each chunk's dH is produced, dW_host (CPU fp32 [V, d]) after the last chunk; either may be None.
+    Pin them (and H_host) for the copies to overlap the compute.  Returns the same dict as the streamed call, plus
+    dH_host and dW_host; the host buffers hold the results once the stream's work is done."""
+    torch = _torch()
+    dev, n, d, V, R = _loss_inputs(H_dev, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids, "H_dev")
+    if not isinstance(H_host, torch.Tensor) or H_host.dtype != torch.bfloat16:
+        raise TypeError("H_host must be a bf16 torch.Tensor")
+    if H_host.device.type != "cpu" or not H_host.is_contiguous():
+        raise ValueError("H_host must be a contiguous CPU tensor")
+    if tuple(H_host.shape) != tuple(H_dev.shape):
+        raise ValueError("H_host and H_dev must have the same shape")
+    for name, t, dt, shape in (("dH_host", dH_host, torch.bfloat16, (n, d)), ("dW_host", dW_host, torch.float32, (V, d))):
+        if t is None:
+            continue
+        if not isinstance(t, torch.Tensor) or t.dtype != dt:
+            raise TypeError(f"{name} must be a {dt} torch.Tensor")
+        if t.device.type != "cpu" or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CPU tensor")
+        _shape(t, shape, name)
+    opt = _options_ref(options, n, dev)
+    if out is not None:
+        _loss_outputs(dev, n, d, V, out["loss"], out["dH"], out["dW"], out.get("lp"), out.get("kappa"))
+    else:
+        out = dict(loss=torch.empty(1, dtype=torch.float32, device=dev),
+                   dH=torch.empty((n, d), dtype=torch.bfloat16, device=dev),
+                   dW=torch.empty((V, d), dtype=torch.float32, device=dev),
+                   lp=torch.empty(n, dtype=torch.float32, device=dev),
+                   kappa=torch.empty(n, dtype=torch.float32, device=dev))
+    ws = _workspace(rz_workspace_bytes_loss(n, R, n_groups, d, V), workspace, dev)
+    code = lib().rz_loss_fwd_bwd_host_io(_ptr(H_host), _ptr(H_dev), _ptr(W_head), _ptr(token_ids), _ptr(lp_rollout),
+                                         _ptr(rewards), _ptr(seg_offsets), _ptr(group_ids), n, R, n_groups, d, V, opt,
+                                         _ptr(out["loss"]), _ptr(out["dH"]), _ptr(out["dW"]), _ptr(out.get("lp")),
+                                         _ptr(out.get("kappa")), _ptr(dH_host), _ptr(dW_host), _ptr(ws), ws.numel(),
+                                         _stream_handle(stream))
+    _check(code, "rz_loss_fwd_bwd_host_io")
+    out["workspace"] = ws
+    out["dH_host"], out["dW_host"] = dH_host, dW_host
+    return out
+
+
+@_on_tensor_device
 def rz_segment_loss_ex(lp, lp_rollout, rewards, seg_offsets, group_ids, n_groups, options, want_w=False,
                        workspace=None, stream=None):
     """rz_segment_loss with rz_loss_options.  Returns dict(loss, kappa, w, workspace)."""
@@ -488,6 +568,7 @@ def rz_segment_loss_ex(lp, lp_rollout, rewards, seg_offsets, group_ids, n_groups
     return dict(loss=loss, kappa=kappa, w=w, workspace=ws)
 
 
+@_on_tensor_device
 def rz_ratio_stats(lp, lp_rollout, seg_offsets, token_mask=None, want_resp_mean=True, workspace=None, stream=None):
     """Ratio diagnostics.  Returns (stats tensor [9] fp64 on device, per-response mean ratio or None)."""
     torch = _torch()
@@ -507,6 +588,7 @@ def rz_ratio_stats(lp, lp_rollout, seg_offsets, token_mask=None, want_resp_mean=
     return stats, rm
 
 
+@_on_tensor_device
 def rz_grad_norms(dH, dW, workspace=None, stream=None):
     """(||dH||, ||dW||) as an fp64 device tensor [2]."""
     torch = _torch()
@@ -522,6 +604,7 @@ def rz_grad_norms(dH, dW, workspace=None, stream=None):
     return out
 
 
+@_on_tensor_device
 def rz_quantize_rows_e4m3(X, stream=None):
     """bf16 [rows, d] -> (e4m3 codes as uint8 [rows, d], fp32 per-row scales [rows])."""
     torch = _torch()
@@ -533,6 +616,7 @@ def rz_quantize_rows_e4m3(X, stream=None):
     return q, sc
 
 
+@_on_tensor_device
 def rz_token_logprobs_fp8(H8, h_scale, W8, w_scale, token_ids, lp_out=None, lse_out=None, workspace=None,
                           stream=None, want_lse=True):
     """Token logprobs from e4m3 operands with per-row scales.  Returns (lp, lse)."""
@@ -556,6 +640,7 @@ def rz_token_logprobs_fp8(H8, h_scale, W8, w_scale, token_ids, lp_out=None, lse_
     return lp, lse
 
 
+@_on_tensor_device
 def rz_sum_shards_f32(stacked, out=None, stream=None):
     """Rank-order sum of the rows of a [nshards, count] fp32 CUDA tensor (fp64 accumulation)."""
     torch = _torch()
@@ -576,3 +661,26 @@ def rz_selftest_wait_timeout(limit_ns: int, stream=None):
                                           _stream_handle(stream)), "rz_selftest_wait_timeout")
     code, bits = rz_read_device_status(ws, stream)
     return code, bits, int(waited.value)
+
+
+@_on_tensor_device
+def rz_selftest_forward_after_timeout(H, W_head, token_ids, use_noalloc_scratch=False, stream=None):
+    """Run the forward (with a workspace, or from the allocation-free scratch) with one wait
+    that gives up enqueued before its kernels.  Returns (lp, lse, status code, status bits);
+    the status is that of the workspace (0, 0 for the scratch, whose status is internal)."""
+    torch = _torch()
+    n, d = _matrix(H, torch.bfloat16, "H")
+    dev = H.device
+    V, dw = _matrix(W_head, torch.bfloat16, "W_head", dev)
+    if dw != d:
+        raise ValueError(f"W_head has d = {dw}, H has d = {d}")
+    _need_shaped(token_ids, torch.int32, "token_ids", dev, (n,))
+    lp = torch.empty(n, dtype=torch.float32, device=dev)
+    lse = torch.empty(n, dtype=torch.float32, device=dev)
+    ws = None if use_noalloc_scratch else _workspace(rz_workspace_bytes_logprobs(n, d, V), None, dev)
+    code = lib().rz_selftest_forward_after_timeout(1 if use_noalloc_scratch else 0, _ptr(H), _ptr(W_head),
+                                                   _ptr(token_ids), n, d, V, _ptr(lp), _ptr(lse), _ptr(ws),
+                                                   0 if ws is None else ws.numel(), _stream_handle(stream))
+    _check(code, "rz_selftest_forward_after_timeout")
+    status = (0, 0) if ws is None else rz_read_device_status(ws, stream)
+    return lp, lse, status[0], status[1]

@@ -18,6 +18,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -180,21 +181,41 @@ void rec_end(Recorder* r, cudaStream_t s) {
 // ---------------------------------------------------------------- launches
 
 int sm_count() {
-  static int cache[kMaxDevices] = {0};
+  static std::atomic<int> cache[kMaxDevices];  // zero-initialised (static storage)
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (dev < kMaxDevices && cache[dev] > 0) return cache[dev];
+  if (dev >= 0 && dev < kMaxDevices) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
   int sms = 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  if (dev < kMaxDevices) cache[dev] = sms;
+  if (dev >= 0 && dev < kMaxDevices) cache[dev].store(sms, std::memory_order_relaxed);
   return sms;
 }
 
-template <bool A_MN, bool B_MN, class Epi>
+// The engine's dynamic shared memory is above the 48 KB default, so each kernel
+// instantiation needs its limit raised once per device; the devices done are kept as bits
+// of a per-instantiation word (setting it twice from racing threads is harmless).
+template <bool A_MN, bool B_MN, class Epi, bool FP8>
+cudaError_t ensure_gemm_smem_attr() {
+  static std::atomic<uint64_t> done{0};
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+  if (bit != 0 && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  err = cudaFuncSetAttribute(gemm_tc_kernel<A_MN, B_MN, Epi, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kGemmSmemBytes);
+  if (err == cudaSuccess && bit != 0) done.fetch_or(bit, std::memory_order_acq_rel);
+  return err;
+}
+
+template <bool A_MN, bool B_MN, class Epi, bool FP8 = false>
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmSched& s, const OperandPos& p,
                         const Epi& e, int* status, cudaStream_t stream) {
-  auto kernel = gemm_tc_kernel<A_MN, B_MN, Epi>;
-  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes);
+  auto kernel = gemm_tc_kernel<A_MN, B_MN, Epi, FP8>;
+  cudaError_t err = ensure_gemm_smem_attr<A_MN, B_MN, Epi, FP8>();
   if (err != cudaSuccess) return err;
   const int sms = sm_count();
   if (sms <= 0) return cudaErrorInvalidDevice;
@@ -351,14 +372,8 @@ rz_status run_forward_fp8(const uint8_t* H8, const float* hs, const uint8_t* W8,
   e.row_scale = hs;
   e.col_scale = wsc;
   e.col_scale_vec = aligned(wsc, 16) ? 1 : 0;
-  auto kernel = gemm_tc_kernel<false, false, EpiLse<false>, true>;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBytes) != cudaSuccess)
+  if (launch_gemm<false, false, EpiLse<false>, true>(mH, mW, s, pos, e, status, stream) != cudaSuccess)
     return RZ_ERR_CUDA;
-  const int sms = sm_count();
-  if (sms <= 0) return RZ_ERR_CUDA;
-  kernel<<<std::max(1, std::min(s.num_units, sms)), kGemmThreads, kGemmSmemBytes, stream>>>(mH, mW, s, pos, e,
-                                                                                          status);
-  if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
   merge_lse_kernel<<<static_cast<unsigned>(ceil_div(n, 256)), 256, 0, stream>>>(
       e.part_m, e.part_s, L.part_ld, e.zy, ids, n, V, num_segments(V), lp, lse, status);
   return cudaGetLastError() == cudaSuccess ? RZ_OK : RZ_ERR_CUDA;
@@ -405,30 +420,20 @@ rz_status run_loss_setup(const float* rewards, const int64_t* off, const int32_t
                          int32_t G, const LossOpts& opt, void* ws, const Layout& L, cudaStream_t stream,
                          Recorder* rec) {
   int* status = at<int>(ws, L.status);
-  int* flags = status + 1;  // cleared together with the status word
-  double* gsum = at<double>(ws, L.gsum);
-  int* gcnt = at<int>(ws, L.gcnt);
-  const unsigned rb = static_cast<unsigned>(ceil_div(R, kCoefThreads));
-  rec_begin(rec, RZ_KERNEL_RESPONSE_COEF, stream);
-  coef_runs_kernel<<<rb, kCoefThreads, 0, stream>>>(rewards, off, gid, R, G, n, gsum, gcnt, flags, status);
-  if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
-  coef_groups_kernel<<<static_cast<unsigned>(ceil_div(G, kCoefThreads)), kCoefThreads, 0, stream>>>(
-      rewards, gid, R, G, gsum, gcnt, flags);
-  if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
+  int* flags = status + 1;  // unsorted flag, then the tickets; cleared with the status word
   int* counted = nullptr;
+  rec_begin(rec, RZ_KERNEL_RESPONSE_COEF, stream);
   if (opt.mask != nullptr) {
     counted = at<int>(ws, L.counted);
     masked_count_kernel<<<static_cast<unsigned>(ceil_div(R, 8)), 256, 0, stream>>>(opt.mask, off, R, counted);
     if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
   }
-  coef_kernel<<<rb, kCoefThreads, 0, stream>>>(rewards, off, gid, R, G, opt.N, counted, gsum, gcnt,
-                                               at<float>(ws, L.coef));
-  if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
-  rec_end(rec, stream);
   const int nb = kappa_blocks(n);
-  rec_begin(rec, RZ_KERNEL_BLOCK_FIRST, stream);
-  block_first_kernel<<<static_cast<unsigned>(ceil_div(nb, 256)), 256, 0, stream>>>(off, R, n, nb,
-                                                                                   at<int>(ws, L.bfirst));
+  const unsigned grid = static_cast<unsigned>(ceil_div(std::max<int64_t>(R, nb), kSetupThreads));
+  loss_setup_kernel<<<grid, kSetupThreads, 0, stream>>>(rewards, off, gid, R, G, n, opt.N, counted,
+                                                        at<double>(ws, L.gsum), at<int>(ws, L.gcnt),
+                                                        at<float>(ws, L.coef), nb, at<int>(ws, L.bfirst), flags,
+                                                        flags + 1, status);
   if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
   rec_end(rec, stream);
   return RZ_OK;
@@ -443,25 +448,18 @@ rz_status run_gate(const float* lp, const float* lp_roll, const int64_t* off, in
   return cudaGetLastError() == cudaSuccess ? RZ_OK : RZ_ERR_CUDA;
 }
 
-// Loss stage, part 2: kappa and ratio for the 4096-token blocks [blk0, blk0 + nblk).
+// Loss stage, part 2: kappa and ratio for the 4096-token blocks [blk0, blk0 + nblk); the
+// block that finishes last of all the call's blocks writes the loss.
 rz_status run_kappa(const float* lp, const float* lp_roll, const int64_t* off, int64_t n, int32_t R, int blk0,
-                    int nblk, const LossOpts& opt, float* kappa, float* w_out, void* ws, const Layout& L,
+                    int nblk, const LossOpts& opt, float* kappa, float* w_out, float* loss, void* ws, const Layout& L,
                     cudaStream_t stream, Recorder* rec) {
   const int vec_ok = aligned(lp, 16) && aligned(lp_roll, 16) && aligned(kappa, 16) &&
                      (w_out == nullptr || aligned(w_out, 16)) && (opt.mask == nullptr || aligned(opt.mask, 4));
   rec_begin(rec, RZ_KERNEL_TOKEN_KAPPA, stream);
   token_kappa_kernel<<<nblk, kKappaThreads, 0, stream>>>(lp, lp_roll, off, R, at<float>(ws, L.coef),
                                                          at<int>(ws, L.bfirst), n, blk0, vec_ok, opt.mask,
-                                                         opt.clip_max, kappa, w_out, at<double>(ws, L.bsum));
-  if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
-  rec_end(rec, stream);
-  return RZ_OK;
-}
-
-// Loss stage, part 3: loss = fixed-order sum of the per-block partials.
-rz_status run_loss_final(int64_t n, float* loss, void* ws, const Layout& L, cudaStream_t stream, Recorder* rec) {
-  rec_begin(rec, RZ_KERNEL_LOSS_FINAL, stream);
-  loss_final_kernel<<<1, 1024, 0, stream>>>(at<double>(ws, L.bsum), kappa_blocks(n), loss);
+                                                         opt.clip_max, kappa, w_out, at<double>(ws, L.bsum),
+                                                         kappa_blocks(n), at<int>(ws, L.status) + 3, loss);
   if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
   rec_end(rec, stream);
   return RZ_OK;
@@ -477,17 +475,84 @@ rz_status run_segment_loss(const float* lp, const float* lp_roll, const float* r
     r = run_gate(lp, lp_roll, off, R, opt, ws, L, stream);
     if (r != RZ_OK) return r;
   }
-  r = run_kappa(lp, lp_roll, off, n, R, 0, kappa_blocks(n), opt, kappa, w_out, ws, L, stream, rec);
-  if (r != RZ_OK) return r;
-  return run_loss_final(n, loss, ws, L, stream, rec);
+  return run_kappa(lp, lp_roll, off, n, R, 0, kappa_blocks(n), opt, kappa, w_out, loss, ws, L, stream, rec);
 }
 
+// A non-blocking stream per device for device-to-host copies of results, created on
+// first use (separate from the host-to-device stream, so both copy directions overlap).
+cudaStream_t d2h_stream_for_current_device() {
+  static std::mutex mu;
+  static cudaStream_t streams[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (streams[dev] == nullptr && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess)
+    streams[dev] = nullptr;
+  return streams[dev];
+}
+
+// Results copied to host memory as they are produced (rz_loss_fwd_bwd_host_io): each
+// chunk's dH rows right after that chunk's dH contraction, dW after the last chunk's dW
+// contraction, on the device-to-host stream, so the copies of chunk c run while chunk
+// c + 1 computes.  finish() makes the compute stream wait for every copy, so the call's
+// work on that stream completes only once the host buffers hold the results.
+struct HostExport {
+  rz_bf16* dH_host;  // nullable
+  float* dW_host;    // nullable
+  cudaStream_t copy = nullptr;
+  cudaEvent_t ev = nullptr;
+
+  HostExport(rz_bf16* dh, float* dw) : dH_host(dh), dW_host(dw) {}
+  HostExport(const HostExport&) = delete;
+  HostExport& operator=(const HostExport&) = delete;
+  ~HostExport() {
+    if (ev != nullptr) cudaEventDestroy(ev);  // released once its pending records complete
+  }
+
+  rz_status start() {
+    copy = d2h_stream_for_current_device();
+    if (copy == nullptr) return RZ_ERR_CUDA;
+    if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) {
+      ev = nullptr;
+      return RZ_ERR_CUDA;
+    }
+    return RZ_OK;
+  }
+
+  // Copy `bytes` from device `src` to host `dst` once the work enqueued on `st` so far is done.
+  rz_status copy_after(cudaStream_t st, void* dst, const void* src, size_t bytes) {
+    if (cudaEventRecord(ev, st) != cudaSuccess || cudaStreamWaitEvent(copy, ev, 0) != cudaSuccess ||
+        cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToHost, copy) != cudaSuccess)
+      return RZ_ERR_CUDA;
+    return RZ_OK;
+  }
+
+  rz_status after_dh(cudaStream_t st, const rz_bf16* dH, int64_t c0, int64_t rows, int32_t d) {
+    if (dH_host == nullptr) return RZ_OK;
+    const size_t off = static_cast<size_t>(c0) * static_cast<size_t>(d);
+    return copy_after(st, dH_host + off, dH + off, static_cast<size_t>(rows) * d * sizeof(rz_bf16));
+  }
+
+  rz_status after_dw(cudaStream_t st, const float* dW, int32_t V, int32_t d) {
+    if (dW_host == nullptr) return RZ_OK;
+    return copy_after(st, dW_host, dW, static_cast<size_t>(V) * d * sizeof(float));
+  }
+
+  // Work enqueued on `st` after this waits for every copy enqueued so far.
+  rz_status finish(cudaStream_t st) {
+    if (cudaEventRecord(ev, copy) != cudaSuccess || cudaStreamWaitEvent(st, ev, 0) != cudaSuccess)
+      return RZ_ERR_CUDA;
+    return RZ_OK;
+  }
+};
+
 // Backward of one chunk of rows [c0, c0 + rows), after its forward (e, tile maxima) and
-// its kappa: dZ in place, dH rows = dZ W, dW (+)= dZ^T H.
+// its kappa: dZ in place, dH rows = dZ W, dW (+)= dZ^T H.  With `out`, the chunk's dH rows
+// are copied to host memory right after their contraction.
 rz_status run_backward_chunk(const rz_bf16* H, const rz_bf16* W, const int32_t* ids, int64_t c0, int64_t rows,
                              int32_t d, int32_t V, const float* lp, const float* lse, const float* kappa,
                              rz_bf16* dH, float* dW, void* ws, const Layout& L, cudaStream_t stream,
-                             Recorder* rec) {
+                             Recorder* rec, HostExport* out = nullptr) {
   int* status = at<int>(ws, L.status);
   uint16_t* dz = at<uint16_t>(ws, L.dz);
   const int64_t ldz = padded_vocab(V);
@@ -518,6 +583,10 @@ rz_status run_backward_chunk(const rz_bf16* H, const rz_bf16* W, const int32_t* 
     rec_begin(rec, RZ_KERNEL_DH, stream);
     if (launch_gemm<false, true>(mDzK, mWmn, s, pos, e, status, stream) != cudaSuccess) return RZ_ERR_CUDA;
     rec_end(rec, stream);
+    if (out != nullptr) {
+      const rz_status r = out->after_dh(stream, dH, c0, rows, d);
+      if (r != RZ_OK) return r;
+    }
   }
   // dW (+)= dZ^T H: A = dZ^T (MN-major: V contiguous), B = H chunk (MN-major: d contiguous)
   {
@@ -580,21 +649,54 @@ RZ_API size_t rz_workspace_bytes_segment_loss(int64_t n_tok, int32_t n_resp, int
   return make_layout(n_tok, n_resp, n_groups, 1, Path::LossStage).total;
 }
 
-RZ_API rz_status rz_token_logprobs(const rz_bf16* H, const rz_bf16* W_head, const int32_t* token_ids, int64_t n_tok,
-                            int32_t d, int32_t V, float* lp_out, float* lse_out, void* workspace,
-                            size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Host checks of the forward entry points (workspace checked by the caller).
+rz_status check_forward_args(const rz_bf16* H, const rz_bf16* W_head, const int32_t* token_ids, int64_t n_tok,
+                             int32_t d, int32_t V, const float* lp_out, const float* lse_out) {
   if (n_tok < 0 || n_tok >= (int64_t{1} << 31)) return RZ_ERR_INVALID_ARG;
   if (!shape_ok(d, V)) return RZ_ERR_UNSUPPORTED_SHAPE;
   if (n_tok == 0) return RZ_OK;
-  if (!H || !W_head || !token_ids || !lp_out || !workspace) return RZ_ERR_INVALID_ARG;
+  if (!H || !W_head || !token_ids || !lp_out) return RZ_ERR_INVALID_ARG;
   if (!aligned(H, 16) || !aligned(W_head, 16) || !aligned(token_ids, 4) || !aligned(lp_out, 4) ||
-      (lse_out && !aligned(lse_out, 4)) || !aligned(workspace, kAlign))
+      (lse_out && !aligned(lse_out, 4)))
     return RZ_ERR_INVALID_ARG;
+  return RZ_OK;
+}
+
+// The forward on a checked workspace: clear the status word, then the LM head + online
+// log-sum-exp and the merge.  inject_timeout (self-test only) enqueues, right after the
+// clear, one bounded wait on a barrier nothing arrives on (1 ms limit), which sets the
+// timeout bit exactly as a wait inside the forward that gave up would.
+rz_status forward_on_workspace(const rz_bf16* H, const rz_bf16* W_head, const int32_t* token_ids, int64_t n_tok,
+                               int32_t d, int32_t V, float* lp_out, float* lse_out, void* ws, const Layout& L,
+                               cudaStream_t st, bool inject_timeout) {
+  if (cudaMemsetAsync(at<int>(ws, L.status), 0, 16, st) != cudaSuccess) return RZ_ERR_CUDA;
+  if (inject_timeout) {
+    // the status piece is 256 bytes: the waited time goes to byte 16, past the two words
+    wait_timeout_selftest_kernel<<<1, 32, 0, st>>>(1000000ull, at<int>(ws, L.status),
+                                                   at<unsigned long long>(ws, L.status + 16));
+    if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
+  }
+  return run_forward(H, W_head, token_ids, 0, n_tok, d, V, lp_out, lse_out, ws, L, false, st, nullptr);
+}
+
+}  // namespace
+
+extern "C" {
+
+RZ_API rz_status rz_token_logprobs(const rz_bf16* H, const rz_bf16* W_head, const int32_t* token_ids, int64_t n_tok,
+                            int32_t d, int32_t V, float* lp_out, float* lse_out, void* workspace,
+                            size_t ws_bytes, void* stream) {
+  const rz_status c = check_forward_args(H, W_head, token_ids, n_tok, d, V, lp_out, lse_out);
+  if (c != RZ_OK || n_tok == 0) return c;
+  if (!workspace || !aligned(workspace, kAlign)) return RZ_ERR_INVALID_ARG;
   const Layout L = make_layout(n_tok, 0, 0, V, Path::Forward);
   if (ws_bytes < L.total) return RZ_ERR_WORKSPACE_TOO_SMALL;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(at<int>(workspace, L.status), 0, 16, st) != cudaSuccess) return RZ_ERR_CUDA;
-  return run_forward(H, W_head, token_ids, 0, n_tok, d, V, lp_out, lse_out, workspace, L, false, st, nullptr);
+  return forward_on_workspace(H, W_head, token_ids, n_tok, d, V, lp_out, lse_out, workspace, L,
+                              static_cast<cudaStream_t>(stream), false);
 }
 
 namespace {
@@ -705,7 +807,7 @@ rz_status loss_fwd_bwd_impl(const rz_bf16* H, const rz_bf16* W_head, const int32
                           const int32_t* group_ids, int64_t n_tok, int32_t n_resp, int32_t n_groups, int32_t d,
                           int32_t V, const rz_loss_options* options, float* loss, rz_bf16* dH, float* dW,
                           float* lp_out, float* kappa_out, void* workspace, size_t ws_bytes, void* stream,
-                          Recorder* rec, HostRows* host_rows = nullptr) {
+                          Recorder* rec, HostRows* host_rows = nullptr, HostExport* host_out = nullptr) {
   if (n_tok < 1 || n_tok >= (int64_t{1} << 31) || n_resp < 1 || n_groups < 1) return RZ_ERR_INVALID_ARG;
   LossOpts opt;
   if (!resolve_options(options, n_resp, &opt)) return RZ_ERR_INVALID_ARG;
@@ -727,6 +829,10 @@ rz_status loss_fwd_bwd_impl(const rz_bf16* H, const rz_bf16* W_head, const int32
   float* kappa = kappa_out ? kappa_out : at<float>(workspace, L.kappa);
   rz_status r = run_loss_setup(rewards, seg_offsets, group_ids, n_tok, n_resp, n_groups, opt, workspace, L, st, rec);
   if (r != RZ_OK) return r;
+  if (host_out != nullptr) {
+    r = host_out->start();
+    if (r != RZ_OK) return r;
+  }
   if (host_rows != nullptr) {  // the first chunk (every chunk for the gate's first pass)
     r = host_rows->start(st);
     if (r == RZ_OK) r = host_rows->enqueue(opt.gate ? n_tok : std::min<int64_t>(kChunkTokens, n_tok));
@@ -756,17 +862,21 @@ rz_status loss_fwd_bwd_impl(const rz_bf16* H, const rz_bf16* W_head, const int32
     if (r != RZ_OK) return r;
     const int blk0 = static_cast<int>(c0 / kKappaBlockTokens);
     const int nblk = static_cast<int>(ceil_div(rows, kKappaBlockTokens));
-    r = run_kappa(lp, lp_rollout, seg_offsets, n_tok, n_resp, blk0, nblk, opt, kappa, nullptr, workspace, L, st,
-                  rec);
+    r = run_kappa(lp, lp_rollout, seg_offsets, n_tok, n_resp, blk0, nblk, opt, kappa, nullptr, loss, workspace, L,
+                  st, rec);
     if (r != RZ_OK) return r;
-    r = run_backward_chunk(H, W_head, token_ids, c0, rows, d, V, lp, lse, kappa, dH, dW, workspace, L, st, rec);
+    r = run_backward_chunk(H, W_head, token_ids, c0, rows, d, V, lp, lse, kappa, dH, dW, workspace, L, st, rec,
+                           host_out);
     if (r != RZ_OK) return r;
     if (host_rows != nullptr && c0 + rows < n_tok) {
       r = host_rows->wait(st);  // before the next chunk's kernels
       if (r != RZ_OK) return r;
     }
   }
-  return run_loss_final(n_tok, loss, workspace, L, st, rec);
+  if (host_out == nullptr) return RZ_OK;
+  r = host_out->after_dw(st, dW, V, d);
+  if (r != RZ_OK) return r;
+  return host_out->finish(st);
 }
 
 }  // namespace
@@ -808,9 +918,24 @@ RZ_API rz_status rz_loss_fwd_bwd_streamed(const rz_bf16* H_host, rz_bf16* H_dev,
                            nullptr, &rows);
 }
 
+RZ_API rz_status rz_loss_fwd_bwd_host_io(const rz_bf16* H_host, rz_bf16* H_dev, const rz_bf16* W_head,
+                                         const int32_t* token_ids, const float* lp_rollout, const float* rewards,
+                                         const int64_t* seg_offsets, const int32_t* group_ids, int64_t n_tok,
+                                         int32_t n_resp, int32_t n_groups, int32_t d, int32_t V,
+                                         const rz_loss_options* options, float* loss, rz_bf16* dH, float* dW,
+                                         float* lp_out, float* kappa_out, rz_bf16* dH_host, float* dW_host,
+                                         void* workspace, size_t ws_bytes, void* stream) {
+  if (H_host == nullptr) return RZ_ERR_INVALID_ARG;
+  HostRows rows(H_host, H_dev, d);
+  HostExport out(dH_host, dW_host);
+  return loss_fwd_bwd_impl(H_dev, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids, n_tok, n_resp,
+                           n_groups, d, V, options, loss, dH, dW, lp_out, kappa_out, workspace, ws_bytes, stream,
+                           nullptr, &rows, &out);
+}
+
 RZ_API int32_t rz_num_launches_loss(int64_t n_tok) {
   if (n_tok < 1) return 0;
-  return static_cast<int32_t>(3 + 6 * ceil_div(n_tok, kChunkTokens));
+  return static_cast<int32_t>(1 + 6 * ceil_div(n_tok, kChunkTokens));
 }
 
 RZ_API rz_status rz_loss_fwd_bwd_timed(const rz_bf16* H, const rz_bf16* W_head, const int32_t* token_ids,
@@ -837,29 +962,75 @@ RZ_API rz_status rz_loss_fwd_bwd_timed(const rz_bf16* H, const rz_bf16* W_head, 
 // so callers that cannot allocate device memory still get the forward.  Every device
 // that loads the library holds these RZ_NOALLOC_SCRATCH_BYTES until the process exits.
 // All calls share it, so calls whose GPU work overlaps (other streams, other threads)
-// race on it; the status word at its start is cleared by every call, and every other
-// byte a call reads has been written earlier in that same call.
+// race on it.  The status word at its start is cleared by every call; every other byte a
+// call reads has been written earlier in that same call, except after a wait that gave
+// up, when the merge writes NaN instead of reading the partials (merge_lse_kernel).
 static __device__ __align__(256) uint8_t g_noalloc_scratch[RZ_NOALLOC_SCRATCH_BYTES];
 
 namespace {
 
+// Identifier of the calling thread's current CUDA context (cuCtxGetId: unique for the life
+// of the process), or 0 when it cannot be read.  Fetched through the runtime's driver entry
+// point query, like the tensor-map encoder, so the library needs no link to libcuda.
+unsigned long long current_context_id() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrent>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(p);
+  });
+  if (get_current == nullptr || get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
 // Device address of g_noalloc_scratch on the current device.  Host code only sees a
-// host-side stand-in under that name, so the address is looked up once per device
-// (with that device current) and cached.
+// host-side stand-in under that name, so the address is looked up with the device
+// current (cudaGetSymbolAddress) and cached per device together with the CUDA context it
+// belongs to: after the device's context is destroyed and recreated (cudaDeviceReset, or
+// a released primary context) the next call sees a new context and looks it up again.
 rz_status noalloc_scratch(void** out) {
   static void* addr[kMaxDevices] = {};
+  static unsigned long long ctx_of[kMaxDevices] = {};
   static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return RZ_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return RZ_ERR_CUDA;
   std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
+  const unsigned long long ctx = current_context_id();
+  if (addr[dev] == nullptr || ctx == 0 || ctx != ctx_of[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return RZ_ERR_CUDA;
     addr[dev] = p;
+    ctx_of[dev] = current_context_id();  // the lookup may have created the context
   }
   *out = addr[dev];
   return RZ_OK;
+}
+
+rz_status noalloc_forward(const rz_bf16* H, const rz_bf16* W_head, const int32_t* token_ids, int64_t n_tok,
+                          int32_t d, int32_t V, float* lp_out, float* lse_out, void* stream, bool inject_timeout) {
+  const rz_status c = check_forward_args(H, W_head, token_ids, n_tok, d, V, lp_out, lse_out);
+  if (c != RZ_OK || n_tok == 0) return c;
+  const Layout L = make_layout(n_tok, 0, 0, V, Path::Forward);
+  if (L.total > static_cast<size_t>(RZ_NOALLOC_SCRATCH_BYTES)) return RZ_ERR_WORKSPACE_TOO_SMALL;
+  void* scratch = nullptr;
+  const rz_status r = noalloc_scratch(&scratch);
+  if (r != RZ_OK) return r;
+  return forward_on_workspace(H, W_head, token_ids, n_tok, d, V, lp_out, lse_out, scratch, L,
+                              static_cast<cudaStream_t>(stream), inject_timeout);
 }
 
 }  // namespace
@@ -869,21 +1040,22 @@ extern "C" {
 RZ_API rz_status rz_token_logprobs_noalloc(const rz_bf16* H, const rz_bf16* W_head, const int32_t* token_ids,
                                            int64_t n_tok, int32_t d, int32_t V, float* lp_out, float* lse_out,
                                            void* stream) {
-  if (n_tok < 0 || n_tok >= (int64_t{1} << 31)) return RZ_ERR_INVALID_ARG;
-  if (!shape_ok(d, V)) return RZ_ERR_UNSUPPORTED_SHAPE;
-  if (n_tok == 0) return RZ_OK;
-  if (!H || !W_head || !token_ids || !lp_out) return RZ_ERR_INVALID_ARG;
-  if (!aligned(H, 16) || !aligned(W_head, 16) || !aligned(token_ids, 4) || !aligned(lp_out, 4) ||
-      (lse_out && !aligned(lse_out, 4)))
-    return RZ_ERR_INVALID_ARG;
+  return noalloc_forward(H, W_head, token_ids, n_tok, d, V, lp_out, lse_out, stream, false);
+}
+
+RZ_API rz_status rz_selftest_forward_after_timeout(int32_t use_noalloc_scratch, const rz_bf16* H,
+                                                   const rz_bf16* W_head, const int32_t* token_ids, int64_t n_tok,
+                                                   int32_t d, int32_t V, float* lp_out, float* lse_out,
+                                                   void* workspace, size_t ws_bytes, void* stream) {
+  if (use_noalloc_scratch)
+    return noalloc_forward(H, W_head, token_ids, n_tok, d, V, lp_out, lse_out, stream, true);
+  const rz_status c = check_forward_args(H, W_head, token_ids, n_tok, d, V, lp_out, lse_out);
+  if (c != RZ_OK || n_tok == 0) return c;
+  if (!workspace || !aligned(workspace, kAlign)) return RZ_ERR_INVALID_ARG;
   const Layout L = make_layout(n_tok, 0, 0, V, Path::Forward);
-  if (L.total > static_cast<size_t>(RZ_NOALLOC_SCRATCH_BYTES)) return RZ_ERR_WORKSPACE_TOO_SMALL;
-  void* scratch = nullptr;
-  const rz_status r = noalloc_scratch(&scratch);
-  if (r != RZ_OK) return r;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(at<int>(scratch, L.status), 0, 16, st) != cudaSuccess) return RZ_ERR_CUDA;
-  return run_forward(H, W_head, token_ids, 0, n_tok, d, V, lp_out, lse_out, scratch, L, false, st, nullptr);
+  if (ws_bytes < L.total) return RZ_ERR_WORKSPACE_TOO_SMALL;
+  return forward_on_workspace(H, W_head, token_ids, n_tok, d, V, lp_out, lse_out, workspace, L,
+                              static_cast<cudaStream_t>(stream), true);
 }
 
 namespace {

@@ -1,10 +1,10 @@
 // rz_simt.cuh -- the SIMT kernels around the tensor-core contractions:
 //
 //   merge_lse_kernel        fixed-order merge of the per-segment (max, sum) pairs -> lse, lp
-//   coef_*_kernel           group means, coef_i = -A_i / (N L_i)
-//   block_first_kernel      first response of each 4096-token block
-//   token_kappa_kernel      unclipped ratio and kappa per token, per-block loss partials
-//   loss_final_kernel       fixed-order sum of the partials
+//   loss_setup_kernel       device checks, group means, coef_i = -A_i / (N L_i), the first
+//                           response of each 4096-token block
+//   token_kappa_kernel      unclipped ratio and kappa per token, per-block loss partials, and
+//                           (its last block) their fixed-order sum, the loss
 //   dz_from_p_kernel        dZ = kappa (onehot - softmax) from the forward's exponentials
 //   masked_count_kernel, gate_kernel
 //                           loss-stage options: counted tokens per response under a token
@@ -34,12 +34,21 @@ namespace rz {
 
 // lse = M + log(sum_s s_s 2^{(m_s - M) log2 e}), segments merged in order s = 0..S-1.
 // Pointers are launch-relative; the partials have row stride part_ld.
+//
+// If a wait of an earlier kernel of the same call gave up (the timeout bit of the status
+// word is set), some partials were never written and may hold an earlier call's values:
+// every lp and lse of the launch is then NaN instead of a plausible wrong number.
 __global__ void merge_lse_kernel(const float* __restrict__ part_m, const float* __restrict__ part_s,
                                  int64_t part_ld, const float* __restrict__ zy, const int32_t* __restrict__ ids,
                                  int64_t n, int V, int S, float* __restrict__ lp, float* __restrict__ lse_out,
                                  int* status) {
   const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (t >= n) return;
+  if (*reinterpret_cast<volatile const int*>(status) & kDevWaitTimeout) {
+    lp[t] = __int_as_float(0x7fc00000);
+    if (lse_out != nullptr) lse_out[t] = __int_as_float(0x7fc00000);
+    return;
+  }
   float M = -INFINITY;
   for (int s = 0; s < S; ++s) M = fmaxf(M, part_m[static_cast<int64_t>(s) * part_ld + t]);
   float sum = 0.0f;
@@ -59,77 +68,9 @@ __global__ void merge_lse_kernel(const float* __restrict__ part_m, const float* 
 
 // ------------------------------------------------------------------------ loss stage
 
-// Group means and the per-response coefficient coef_i = -A_i / (N L_i), in three short
-// launches over responses and groups:
-//   coef_runs_kernel   checks segments and group ids, flags group ids that are not
-//                      non-decreasing, and lets the first response of each run of equal
-//                      ids sum the run's rewards (the whole group when ids are sorted)
-//   coef_groups_kernel only when ids are not sorted: each group scans all responses
-//   coef_kernel        A_i = r_i - gsum/gcnt, coef_i
-// Both ways add a group's rewards in response-index order (fp64), so both give the same
-// bits.  flags[0] is the unsorted flag (cleared with the status word).
-constexpr int kCoefThreads = 256;
-
-__global__ void __launch_bounds__(kCoefThreads)
-    coef_runs_kernel(const float* __restrict__ rewards, const int64_t* __restrict__ off,
-                     const int32_t* __restrict__ gid, int R, int G, int64_t n, double* __restrict__ gsum,
-                     int* __restrict__ gcnt, int* flags, int* status) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= R) return;
-  int bad = 0;
-  if (i == 0 && (off[0] != 0 || off[R] != n)) bad |= kDevBadSegments;
-  if (off[i + 1] <= off[i]) bad |= kDevBadSegments;
-  const int g = gid[i];
-  if (g < 0 || g >= G) bad |= kDevBadGroupId;
-  if (bad) atomicOr(status, bad);
-  if (i + 1 < R && gid[i + 1] < g) atomicOr(flags, 1);
-  if ((i > 0 && gid[i - 1] == g) || g < 0 || g >= G) return;  // not the start of a valid run
-  double sum = 0.0;
-  int c = 0;
-  for (int j = i; j < R && gid[j] == g; ++j) {
-    sum += static_cast<double>(rewards[j]);
-    ++c;
-  }
-  gsum[g] = sum;  // with sorted ids every group is one run, so one writer per group
-  gcnt[g] = c;
-}
-
-__global__ void __launch_bounds__(kCoefThreads)
-    coef_groups_kernel(const float* __restrict__ rewards, const int32_t* __restrict__ gid, int R, int G,
-                       double* __restrict__ gsum, int* __restrict__ gcnt, const int* flags) {
-  const int g = blockIdx.x * blockDim.x + threadIdx.x;
-  if (g >= G || *flags == 0) return;
-  double sum = 0.0;
-  int c = 0;
-  for (int i = 0; i < R; ++i) {
-    if (__ldg(gid + i) == g) {
-      sum += static_cast<double>(__ldg(rewards + i));
-      ++c;
-    }
-  }
-  gsum[g] = sum;
-  gcnt[g] = c;
-}
-
-__global__ void __launch_bounds__(kCoefThreads)
-    coef_kernel(const float* __restrict__ rewards, const int64_t* __restrict__ off, const int32_t* __restrict__ gid,
-                int R, int G, double N, const int* __restrict__ counted, const double* __restrict__ gsum,
-                const int* __restrict__ gcnt, float* __restrict__ coef) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= R) return;
-  const int g = gid[i];
-  const int64_t L = counted != nullptr ? counted[i] : off[i + 1] - off[i];
-  if (g < 0 || g >= G || off[i + 1] <= off[i] || gcnt[g] <= 0) {
-    coef[i] = __int_as_float(0x7fc00000);
-    return;
-  }
-  if (L <= 0) {  // every token of the response is masked out: it contributes nothing
-    coef[i] = 0.0f;
-    return;
-  }
-  const double A = static_cast<double>(rewards[i]) - gsum[g] / static_cast<double>(gcnt[g]);
-  coef[i] = static_cast<float>(-A / (N * static_cast<double>(L)));
-}
+// Group means and the per-response coefficient coef_i = -A_i / (N L_i): loss_setup_kernel
+// below.  flags[0] is the unsorted-ids flag; flags[1] and flags[2] are the tickets of the
+// setup kernel and of the ratio / kappa kernel (all cleared with the status word).
 
 // Per response (one warp each): the number of tokens whose mask byte is non-zero.
 __global__ void __launch_bounds__(256)
@@ -187,12 +128,86 @@ __device__ __forceinline__ int find_response(const int64_t* __restrict__ off, in
   return lo;
 }
 
-// First response of every 4096-token block of the loss stage (one thread per block).
-__global__ void block_first_kernel(const int64_t* __restrict__ off, int R, int64_t n, int nblocks,
-                                   int* __restrict__ first) {
-  const int b = blockIdx.x * blockDim.x + threadIdx.x;
-  if (b >= nblocks) return;
-  first[b] = find_response(off, R, min(n - 1, static_cast<int64_t>(b) * kKappaBlockTokens));
+// The loss stage's setup in one launch:
+//  - thread i < R checks response i (segments, group id) and flags ids that are not
+//    non-decreasing; a thread that starts a run of equal valid ids sums the run's rewards
+//    (fp64, response order) and, since with non-decreasing ids a run is the whole group,
+//    writes coef_j = -A_j / (N L_j) for every response of the run;
+//  - thread b < nblocks writes the first response of 4096-token block b;
+//  - the last block to finish (a ticket on `ticket`, cleared with the status word) redoes
+//    the group sums by scanning the responses in index order and rewrites every coef when
+//    the ids were not sorted.  Either way a group's rewards are added in response order,
+//    so both give the same bits.
+// counted (nullable): tokens per response under a token mask (masked_count_kernel).
+constexpr int kSetupThreads = 256;
+
+__device__ __forceinline__ float response_coef(const float* __restrict__ rewards, const int64_t* __restrict__ off,
+                                               const int32_t* __restrict__ gid, int G, double N,
+                                               const int* __restrict__ counted, double gsum_g, int gcnt_g, int i) {
+  const int g = gid[i];
+  const int64_t L = counted != nullptr ? counted[i] : off[i + 1] - off[i];
+  if (g < 0 || g >= G || off[i + 1] <= off[i] || gcnt_g <= 0) return __int_as_float(0x7fc00000);
+  if (L <= 0) return 0.0f;  // every token of the response is masked out: it contributes nothing
+  const double A = static_cast<double>(rewards[i]) - gsum_g / static_cast<double>(gcnt_g);
+  return static_cast<float>(-A / (N * static_cast<double>(L)));
+}
+
+__global__ void __launch_bounds__(kSetupThreads)
+    loss_setup_kernel(const float* __restrict__ rewards, const int64_t* __restrict__ off,
+                      const int32_t* __restrict__ gid, int R, int G, int64_t n, double N,
+                      const int* __restrict__ counted, double* __restrict__ gsum, int* __restrict__ gcnt,
+                      float* __restrict__ coef, int nblocks, int* __restrict__ bfirst, int* flags, int* ticket,
+                      int* status) {
+  __shared__ bool s_last;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < R) {
+    int bad = 0;
+    if (i == 0 && (off[0] != 0 || off[R] != n)) bad |= kDevBadSegments;
+    if (off[i + 1] <= off[i]) bad |= kDevBadSegments;
+    const int g = gid[i];
+    if (g < 0 || g >= G) bad |= kDevBadGroupId;
+    if (bad) atomicOr(status, bad);
+    if (i + 1 < R && gid[i + 1] < g) atomicOr(flags, 1);
+    if (g < 0 || g >= G) {
+      coef[i] = __int_as_float(0x7fc00000);
+    } else if (i == 0 || gid[i - 1] != g) {  // the start of a run of equal ids
+      double sum = 0.0;
+      int c = 0;
+      for (int j = i; j < R && gid[j] == g; ++j) {
+        sum += static_cast<double>(rewards[j]);
+        ++c;
+      }
+      gsum[g] = sum;  // with sorted ids every group is one run, so one writer per group
+      gcnt[g] = c;
+      for (int j = i; j < i + c; ++j) coef[j] = response_coef(rewards, off, gid, G, N, counted, sum, c, j);
+    }
+  }
+  if (i < nblocks) bfirst[i] = find_response(off, R, min(n - 1, static_cast<int64_t>(i) * kKappaBlockTokens));
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(ticket, 1) == static_cast<int>(gridDim.x) - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  if (*reinterpret_cast<volatile const int*>(flags) == 0) return;  // sorted: every coef is written
+  for (int g = threadIdx.x; g < G; g += blockDim.x) {
+    double sum = 0.0;
+    int c = 0;
+    for (int j = 0; j < R; ++j) {
+      if (__ldg(gid + j) == g) {
+        sum += static_cast<double>(__ldg(rewards + j));
+        ++c;
+      }
+    }
+    gsum[g] = sum;
+    gcnt[g] = c;
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < R; j += blockDim.x) {
+    const int g = gid[j];
+    const bool valid = g >= 0 && g < G;
+    coef[j] = response_coef(rewards, off, gid, G, N, counted, valid ? gsum[g] : 0.0, valid ? gcnt[g] : 0, j);
+  }
 }
 
 // kappa_t = coef_i * w_t with the unclipped ratio w_t = exp(lp_t - lp_rollout_t), for the
@@ -211,11 +226,14 @@ __global__ void __launch_bounds__(kKappaThreads, 5)
                        const int64_t* __restrict__ off, int R, const float* __restrict__ coef,
                        const int* __restrict__ block_first, int64_t n, int block0, int vec_ok,
                        const uint8_t* __restrict__ mask, float clip_max, float* __restrict__ kappa,
-                       float* __restrict__ w_out, double* __restrict__ block_sums) {
+                       float* __restrict__ w_out, double* __restrict__ block_sums, int total_blocks,
+                       int* __restrict__ ticket, float* __restrict__ loss) {
   constexpr int kFar = 1 << 30;  // a relative start beyond the block
   __shared__ int s_rel[kKappaStagedOffsets + 1];  // start of staged response k, relative to the block
   __shared__ float s_coef[kKappaStagedOffsets];
   __shared__ double warp_sums[kKappaThreads / 32];
+  __shared__ double s_tree[kKappaThreads];
+  __shared__ bool s_last;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int blk = block0 + blockIdx.x;
@@ -311,21 +329,24 @@ __global__ void __launch_bounds__(kKappaThreads, 5)
     double sum = 0.0;
     for (int w = 0; w < kKappaThreads / 32; ++w) sum += warp_sums[w];
     block_sums[blk] = sum;
+    __threadfence();
+    // the last of all total_blocks blocks (over every launch of the call; the ticket is
+    // cleared with the status word) forms the loss
+    s_last = atomicAdd(ticket, 1) == total_blocks - 1;
   }
-}
-
-// loss = sum of the block partials (fixed strided order, then a fixed tree).
-__global__ void loss_final_kernel(const double* __restrict__ block_sums, int nb, float* __restrict__ loss) {
-  __shared__ double sh[1024];
-  double s = 0.0;
-  for (int b = threadIdx.x; b < nb; b += blockDim.x) s += block_sums[b];
-  sh[threadIdx.x] = s;
   __syncthreads();
-  for (int w = blockDim.x >> 1; w > 0; w >>= 1) {
-    if (threadIdx.x < w) sh[threadIdx.x] += sh[threadIdx.x + w];
+  if (!s_last) return;
+  __threadfence();
+  // loss = sum of the block partials in a fixed order: strided per thread, then a fixed tree
+  double acc = 0.0;
+  for (int b = threadIdx.x; b < total_blocks; b += kKappaThreads) acc += __ldcg(block_sums + b);
+  s_tree[threadIdx.x] = acc;
+  __syncthreads();
+  for (int w = kKappaThreads >> 1; w > 0; w >>= 1) {
+    if (threadIdx.x < w) s_tree[threadIdx.x] += s_tree[threadIdx.x + w];
     __syncthreads();
   }
-  if (threadIdx.x == 0) *loss = static_cast<float>(sh[0]);
+  if (threadIdx.x == 0) *loss = static_cast<float>(s_tree[0]);
 }
 
 // ------------------------------------------------------------------------ backward

@@ -99,16 +99,21 @@ def shard_groups(seg_offsets, group_ids, world: int):
 
 
 def dp_loss_fwd_bwd(H, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids, n_groups, group=None,
-                    options=None, sum_shards=None):
+                    options=None, sum_shards=None, workspace=None, n_resp_total=None):
     """One data-parallel step: this rank's shard (whole groups, e.g. from shard_groups) through
     rz_loss_fwd_bwd_ex with N = the global response count, then dW and the loss summed
     deterministically.  dH stays local (its rows are this rank's tokens).  Returns the
-    rz_loss_fwd_bwd dict with the global loss and dW.  `sum_shards` is for testing the
-    orchestration on CPU ranks only (see deterministic_all_reduce)."""
-    n_total = global_response_count(rewards.shape[0], rewards.device, group)
+    rz_loss_fwd_bwd dict with the global loss and dW.  `workspace` (uint8 CUDA tensor of at
+    least rz_workspace_bytes_loss for the shard) is reused when given; `n_resp_total`, when
+    the caller already knows it, saves the collective that counts the responses.
+    `sum_shards` is for testing the orchestration on CPU ranks only (see
+    deterministic_all_reduce)."""
+    n_total = (global_response_count(rewards.shape[0], rewards.device, group) if n_resp_total is None
+               else int(n_resp_total))
     opts = options if options is not None else loss_options()
     opts.n_resp_total = n_total
-    out = rz_loss_fwd_bwd_ex(H, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids, n_groups, opts)
+    out = rz_loss_fwd_bwd_ex(H, W_head, token_ids, lp_rollout, rewards, seg_offsets, group_ids, n_groups, opts,
+                             workspace=workspace)
     out["dW"] = deterministic_all_reduce(out["dW"], group, sum_shards)
     out["loss"] = deterministic_all_reduce(out["loss"], group, sum_shards)
     return out

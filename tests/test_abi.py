@@ -141,6 +141,17 @@ def test_host_argument_checks_streamed(rz):
     assert call(d=96) == 2
     assert call(wsb=100) == 3
 
+    def host_io(**kw):
+        a = dict(Hh=128, Hd=256, W=512, ids=1024, lr=2048, r=3072, off=4096, gid=5120, n=100, R=4, G=2, d=256,
+                 V=4096, loss=6144, dH=7168, dW=8192, dHh=9216, dWh=10240, ws=1 << 20, wsb=1 << 40)
+        a.update(kw)
+        return lib.rz_loss_fwd_bwd_host_io(a["Hh"], a["Hd"], a["W"], a["ids"], a["lr"], a["r"], a["off"], a["gid"],
+                                           a["n"], a["R"], a["G"], a["d"], a["V"], None, a["loss"], a["dH"],
+                                           a["dW"], None, None, a["dHh"], a["dWh"], a["ws"], a["wsb"], None)
+
+    assert host_io(Hh=None) == 1 and host_io(Hd=None) == 1 and host_io(d=96) == 2 and host_io(wsb=100) == 3
+    assert host_io(n=0) == 1
+
 
 def _opts(rz, **kw):
     o = rz.rz_loss_options()
@@ -261,6 +272,18 @@ def test_host_checks_of_the_shard_sum_selftest_noalloc_and_timed(rz):
     # beyond the fixed 32 MiB scratch: 4 n (2 ceil(V / 2048) + 1) bytes plus the status word
     assert noalloc(n=1 << 20, V=151936) == 3
 
+    def after_timeout(**kw):
+        a = dict(use=0, H=256, W=512, ids=1024, n=100, d=256, V=4096, lp=2048, lse=None, ws=1 << 20, wsb=1 << 40)
+        a.update(kw)
+        return lib.rz_selftest_forward_after_timeout(a["use"], a["H"], a["W"], a["ids"], a["n"], a["d"], a["V"],
+                                                     a["lp"], a["lse"], a["ws"], a["wsb"], None)
+
+    # the same host checks as the call each variant runs
+    assert after_timeout(n=-1) == 1 and after_timeout(d=96) == 2 and after_timeout(H=None) == 1
+    assert after_timeout(ws=None) == 1 and after_timeout(ws=(1 << 20) + 16) == 1 and after_timeout(wsb=100) == 3
+    assert after_timeout(use=1, ws=None, wsb=0, n=1 << 20, V=151936) == 3
+    assert after_timeout(n=0, H=None, W=None, ids=None, lp=None, ws=None) == 0
+
     count = ctypes.c_int32(-5)
     kinds = (ctypes.c_int32 * 4)()
     events = (ctypes.c_void_p * 8)()
@@ -273,6 +296,6 @@ def test_host_checks_of_the_shard_sum_selftest_noalloc_and_timed(rz):
     assert timed(ev=None) == 1 and timed(cap=-1) == 1
     assert timed(n=0) == 1 and count.value == 0   # nothing recorded on an argument error
     assert lib.rz_num_launches_loss(0) == 0
-    # 3 loss-stage launches, 6 per 16384-token chunk
-    assert [lib.rz_num_launches_loss(n) for n in (1, 16384, 16385)] == [9, 9, 15]
+    # the loss setup, then 6 per 16384-token chunk
+    assert [lib.rz_num_launches_loss(n) for n in (1, 16384, 16385)] == [7, 7, 13]
     assert lib.rz_read_device_status(None, None, None) == 1

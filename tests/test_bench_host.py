@@ -117,3 +117,58 @@ def test_batch_invariance_check_counts_rows_of_a_batch_variant_forward():
     assert inv["rows_differing"]["alone"] == 20
     assert inv["rows_differing"]["chunks_64"] == 0 and inv["rows_differing"]["permuted"] == 0
     assert inv["diff"] == 20
+
+
+@pytest.mark.parametrize("world", [1, 2, 4, 8])
+def test_data_parallel_shards_cover_the_batch_in_whole_groups(world):
+    import numpy as np
+    import workloads as wl
+    seg = wl.draw_segments("qwen3_4b")
+    lo, resp = 0, 0
+    for rank in range(world):
+        sh, rewards, n_total = bench.dp_shard(seg, world, rank)
+        assert n_total == seg.n_resp  # every rank's N is the whole batch's response count
+        assert sh["tok_lo"] == lo and sh["resp_lo"] == resp
+        assert np.array_equal(rewards, seg.rewards[sh["resp_lo"]:sh["resp_hi"]])
+        gid = seg.group_ids[sh["resp_lo"]:sh["resp_hi"]]
+        # whole groups: no group is split between two ranks
+        assert sh["resp_lo"] == 0 or seg.group_ids[sh["resp_lo"] - 1] != gid[0]
+        assert sh["resp_hi"] == seg.n_resp or seg.group_ids[sh["resp_hi"]] != gid[-1]
+        assert sh["seg_offsets"][0] == 0 and sh["seg_offsets"][-1] == sh["tok_hi"] - sh["tok_lo"]
+        lo, resp = sh["tok_hi"], sh["resp_hi"]
+    assert lo == seg.n_tok and resp == seg.n_resp
+
+
+def _fake_result():
+    kern = {"lmhead_lse": {"launches": 23, "ms_per_step": 261.123456, "share": 0.34, "tflops": 1075.0,
+                           "frac_of_peak": 0.7691234}}
+    ls = {"frac": 0.72, "variant_clip_mask": {"frac": 0.67}, "ratio_stats": {"frac": 0.62}, "sm_mhz": 1252.0}
+    return dict(cfg={"lengths": ("loguniform", 128, 2048)}, peak=1400.0, achieved=1075.0, d=2560, V=151936,
+                n_tok=360896, G=64, R=512, value=468908.2, ms_per_step=769.6, dominant="lmhead_lse",
+                traffic=None, peak_src="fallback", clocks={"sm_mhz": 1155.0}, launches=2820,
+                e2e={"value": 4.4e5}, kernels=kern, invariance={"diff": 0}, loss_stage=ls, fwd_tok_s=1.5e6,
+                fwd_ms=240.0, fwd8_ms=160.0, workloads={"lag64_1437610_tok": {"fwd_bwd_tok_s": 4.6e5}})
+
+
+def test_line_puts_the_contract_keys_first_and_the_compact_figures_last():
+    import argparse
+    args = argparse.Namespace(steps=5, warmup=3, workload="qwen3_4b")
+    line = bench.make_line(args, 1, _fake_result(), {"value": 8.5})
+    keys = list(line)
+    assert keys[:13] == ["metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                         "scaling", "vs_baseline", "dtype", "data", "config"]
+    assert keys[-5:] == ["tensor_frac_6dV", "fwd_only", "fwd_only_fp8", "loss_stage_frac", "workloads"]
+    assert line["roofline"]["frac"] == pytest.approx(1075.0 / 1400.0)
+    assert line["kernels"]["lmhead_lse"]["frac_of_peak"] == 0.7691  # rounded to 4 significant digits
+    # the compact tail fits in the part of the output a log tail keeps
+    tail = json.dumps({k: line[k] for k in keys[-5:]})
+    assert len(tail) < 1500
+
+
+def test_dp_line_reports_strong_scaling():
+    import argparse
+    args = argparse.Namespace(steps=3, warmup=3, workload="qwen3_4b")
+    r = dict(value=3.6e6, ms_per_step=100.0, n_tok=360896, shard_tokens=45000, d=2560, V=151936, status_ok=True,
+             dW_same_bits_on_all_ranks=True, clocks=None, launches=60, n_resp=512, n_groups=64)
+    line = bench.make_dp_line(args, 8, r)
+    assert line["scaling"] == "strong" and line["n_gpus"] == 8 and line["dW_same_bits_on_all_ranks"]

@@ -77,6 +77,11 @@ def _calls():
             rz.rz_loss_fwd_bwd_streamed, lambda x: [torch.zeros((n, d), dtype=torch.bfloat16)] + loss_pos(x),
             lambda x: dict(out=dict(loss=torch.zeros(1), dH=torch.zeros((n, d), dtype=torch.bfloat16),
                                     dW=torch.zeros((V, d)), lp=torch.zeros(n), kappa=torch.zeros(n)))),
+        "rz_loss_fwd_bwd_host_io": (
+            rz.rz_loss_fwd_bwd_host_io, lambda x: [torch.zeros((n, d), dtype=torch.bfloat16)] + loss_pos(x),
+            lambda x: dict(dH_host=torch.zeros((n, d), dtype=torch.bfloat16), dW_host=torch.zeros((V, d)),
+                           out=dict(loss=torch.zeros(1), dH=torch.zeros((n, d), dtype=torch.bfloat16),
+                                    dW=torch.zeros((V, d)), lp=torch.zeros(n), kappa=torch.zeros(n)))),
         "rz_segment_loss": (rz.rz_segment_loss, seg_pos,
                             lambda x: dict(loss=torch.zeros(1), kappa_out=torch.zeros(n), w_out=torch.zeros(n))),
         "rz_segment_loss_ex": (rz.rz_segment_loss_ex, lambda x: seg_pos(x) + [None], lambda x: {}),

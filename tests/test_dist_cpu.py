@@ -119,7 +119,7 @@ def _dp_worker(rank, world, port, out):
         s = dp.shard_groups(p.seg.seg_offsets, p.seg.group_ids, world)[rank]
         t0, t1, r0, r1 = s["tok_lo"], s["tok_hi"], s["resp_lo"], s["resp_hi"]
 
-        def shard_step(H, W, ids, lp_rollout, rewards, seg_offsets, group_ids, n_groups, opts):
+        def shard_step(H, W, ids, lp_rollout, rewards, seg_offsets, group_ids, n_groups, opts, workspace=None):
             # the oracle in place of the GPU call (CPU ranks have no GPU); same N as the kernels get
             lp, lse = oracle.token_logprobs(H, W, ids)
             loss, _, kappa = oracle.loss_from_lp_ex(lp, lp_rollout, rewards.numpy(), seg_offsets, group_ids, n_groups,

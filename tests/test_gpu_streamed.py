@@ -109,3 +109,52 @@ def test_streamed_rejects_null_host_pointer(rz, prob):
                                         dev["rewards"].shape[0], prob.seg.n_groups, d, dev["W"].shape[0], None,
                                         None, None, None, None, None, None, 0, None)
     assert code == 1  # RZ_ERR_INVALID_ARG, nothing enqueued
+
+
+@pytest.mark.parametrize("pinned", [True, False])
+def test_host_io_delivers_the_gradients_to_host_memory(rz, prob, pinned):
+    """rz_loss_fwd_bwd_host_io: dH chunk by chunk and dW at the end copied to host buffers
+    that start as garbage; they must equal the device-resident call bit for bit."""
+    dev = _inputs(prob)
+    ref = _call_device(rz, dev, prob, None)
+    n, d = dev["H"].shape
+    V = dev["W"].shape[0]
+    H_host = dev["H"].cpu()
+    dH_host = torch.full((n, d), 7.0, dtype=torch.bfloat16)
+    dW_host = torch.full((V, d), 7.0)
+    if pinned:
+        H_host, dH_host, dW_host = H_host.pin_memory(), dH_host.pin_memory(), dW_host.pin_memory()
+    H_dev = _garbage_like(dev["H"])
+    out = rz.rz_loss_fwd_bwd_host_io(H_host, H_dev, dev["W"], dev["ids"], dev["lp_roll"], dev["rewards"],
+                                     dev["seg_offsets"], dev["group_ids"], prob.seg.n_groups, dH_host=dH_host,
+                                     dW_host=dW_host)
+    torch.cuda.current_stream().synchronize()  # the stream's work includes the copies
+    assert rz.rz_read_device_status(out["workspace"]) == (0, 0)
+    _same(out, ref)
+    assert torch.equal(dH_host.view(torch.int16), ref["dH"].cpu().view(torch.int16))
+    assert torch.equal(dW_host.view(torch.int32), ref["dW"].cpu().view(torch.int32))
+
+
+def test_host_io_back_to_back_and_without_host_outputs(rz, prob):
+    """Two calls in a row into the same host buffers: the second call's dH must not be
+    copied out before its own contraction; and both host outputs may be omitted."""
+    dev = _inputs(prob)
+    H2 = _garbage_like(dev["H"]).mul_(1e-3)
+    ref2 = _call_device(rz, dict(dev, H=H2), prob, None)
+    n, d = dev["H"].shape
+    V = dev["W"].shape[0]
+    dH_host = torch.empty((n, d), dtype=torch.bfloat16).pin_memory()
+    dW_host = torch.empty((V, d)).pin_memory()
+    H_dev = torch.empty_like(dev["H"])
+    for H in (dev["H"], H2):
+        out = rz.rz_loss_fwd_bwd_host_io(H.cpu().pin_memory(), H_dev, dev["W"], dev["ids"], dev["lp_roll"],
+                                         dev["rewards"], dev["seg_offsets"], dev["group_ids"], prob.seg.n_groups,
+                                         dH_host=dH_host, dW_host=dW_host)
+    torch.cuda.synchronize()
+    _same(out, ref2)
+    assert torch.equal(dH_host.view(torch.int16), ref2["dH"].cpu().view(torch.int16))
+    assert torch.equal(dW_host.view(torch.int32), ref2["dW"].cpu().view(torch.int32))
+    plain = rz.rz_loss_fwd_bwd_host_io(H2.cpu(), H_dev, dev["W"], dev["ids"], dev["lp_roll"], dev["rewards"],
+                                       dev["seg_offsets"], dev["group_ids"], prob.seg.n_groups)
+    torch.cuda.synchronize()
+    _same(plain, ref2)

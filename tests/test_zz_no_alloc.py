@@ -84,3 +84,53 @@ def test_noalloc_rejects_calls_beyond_its_scratch(rz):
     assert _noalloc(rz, H, W, ids, lp, None) == 3  # RZ_ERR_WORKSPACE_TOO_SMALL
     torch.cuda.synchronize()
     assert torch.all(lp == 7.0)  # nothing was enqueued
+
+
+def test_noalloc_out_of_range_ids_give_nan_rows_only(rz):
+    # the bad-id path sets its status bit in the shared scratch (internal here): the rows
+    # with an id outside [0, V) are NaN, every other row is bit-equal to the workspace call
+    n, d, V = 400, 512, 9000
+    H, W, ids = _problem(n, d, V, 4)
+    bad = torch.tensor([7, 200], device="cuda")
+    ids[bad[0]] = V
+    ids[bad[1]] = -1
+    lp = torch.empty(n, device="cuda")
+    lse = torch.empty(n, device="cuda")
+    assert _noalloc(rz, H, W, ids, lp, lse) == 0
+    ref_lp, ref_lse = rz.rz_token_logprobs(H, W, ids)
+    torch.cuda.synchronize()
+    good = torch.ones(n, dtype=torch.bool, device="cuda")
+    good[bad] = False
+    assert torch.isnan(lp[bad]).all()
+    assert torch.equal(lp[good].view(torch.int32), ref_lp[good].view(torch.int32))
+    assert torch.equal(lse.view(torch.int32), ref_lse.view(torch.int32))
+    # and the next call, with valid ids, is clean again
+    ids[bad] = 3
+    assert _noalloc(rz, H, W, ids, lp, lse) == 0
+    ref_lp, _ = rz.rz_token_logprobs(H, W, ids)
+    torch.cuda.synchronize()
+    assert torch.equal(lp.view(torch.int32), ref_lp.view(torch.int32))
+
+
+@pytest.mark.parametrize("use_scratch", [True, False])
+def test_wait_that_gave_up_gives_nan_not_stale_values(rz, use_scratch):
+    # a wait that gives up leaves partials unwritten; the scratch then still holds the
+    # previous call's partials of the same rows.  The merge must not turn those into
+    # plausible logprobs: every lp and lse of the call comes out NaN.
+    n, d, V = 300, 256, 5000
+    H, W, ids = _problem(n, d, V, 5)
+    lp = torch.empty(n, device="cuda")
+    lse = torch.empty(n, device="cuda")
+    assert _noalloc(rz, H, W, ids, lp, lse) == 0  # leaves this shape's partials in the scratch
+    torch.cuda.synchronize()
+    assert torch.isfinite(lp).all()
+    lp_t, lse_t, code, bits = rz.rz_selftest_forward_after_timeout(H, W, ids, use_noalloc_scratch=use_scratch)
+    torch.cuda.synchronize()
+    assert torch.isnan(lp_t).all() and torch.isnan(lse_t).all()
+    if not use_scratch:
+        assert code == 6 and bits & 8  # RZ_ERR_DEVICE_TIMEOUT, RZ_DEV_WAIT_TIMEOUT
+    # the next ordinary call is correct again
+    lp2 = torch.empty(n, device="cuda")
+    assert _noalloc(rz, H, W, ids, lp2, None) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(lp2.view(torch.int32), lp.view(torch.int32))
