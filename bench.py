@@ -348,6 +348,22 @@ def run_rz(args, rank, world, local_rank):
         fwd8_ms = max_over_ranks(fwd8_ms, dev)
     del H8, W8
 
+    # forward from MXFP4 operands (quantised once, outside the timed region)
+    H4, hs4 = rz.rz_quantize_rows_mxfp4(H)
+    W4, ws4 = rz.rz_quantize_rows_mxfp4(W)
+    lp4 = torch.empty(n, dtype=torch.float32, device=dev)
+    for _ in range(2):
+        rz.rz_token_logprobs_mxfp4(H4, hs4, W4, ws4, ids, lp_out=lp4, workspace=wsf, stream=stream, want_lse=False)
+    f0.record(stream)
+    for _ in range(fsteps):
+        rz.rz_token_logprobs_mxfp4(H4, hs4, W4, ws4, ids, lp_out=lp4, workspace=wsf, stream=stream, want_lse=False)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    fwd4_ms = f0.elapsed_time(f1) / fsteps
+    if dist:
+        fwd4_ms = max_over_ranks(fwd4_ms, dev)
+    del H4, W4, hs4, ws4
+
     invariance = run_batch_invariance(rz, torch, dev, stream, H, W, ids, lp, wsf, prob.seed)
     if dist:
         invariance["diff"] = int(max_over_ranks(float(invariance["diff"]), dev))
@@ -388,7 +404,7 @@ def run_rz(args, rank, world, local_rank):
         dominant=dom, achieved=ach, peak=peak_tflops, peak_src=peak_src,
         traffic=traffic_for(dom, tens[dom]["rows"] / tens[dom]["launches"]),
         fwd_ms=fwd_ms, fwd_tok_s=world * n / (fwd_ms * 1e-3), launches=launches_total, e2e=e2e, cfg=cfg,
-        loss_stage=loss_stage, fwd8_ms=fwd8_ms, invariance=invariance, workloads=other,
+        loss_stage=loss_stage, fwd8_ms=fwd8_ms, fwd4_ms=fwd4_ms, invariance=invariance, workloads=other,
     )
 
 
@@ -907,6 +923,9 @@ def make_line(args, world, res, cpu):
         "fwd_only_fp8": _round({"tokens_per_s": n * world / (res["fwd8_ms"] * 1e-3), "ms_per_step": res["fwd8_ms"],
                                 "tensor_frac_2dV": n * 2 * d * V / (res["fwd8_ms"] * 1e-3) / (2 * peak * 1e12),
                                 "peak": "2 x sustained bf16 (nominal e4m3 ratio)"}),
+        "fwd_only_mxfp4": _round({"tokens_per_s": n * world / (res["fwd4_ms"] * 1e-3), "ms_per_step": res["fwd4_ms"],
+                                  "tensor_frac_2dV": n * 2 * d * V / (res["fwd4_ms"] * 1e-3) / (4 * peak * 1e12),
+                                  "peak": "4 x sustained bf16 (nominal dense fp4 ratio)"}),
     }
     ls = res["loss_stage"]
     if ls is not None:

@@ -293,6 +293,36 @@ rz_status rz_token_logprobs_fp8(const uint8_t* H8, const float* h_scale, const u
                                 float* lse_out, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * MXFP4 forward: token logprobs from OCP Microscaling MXFP4 operands (the FP4 weights with
+ * block scales of "vLLM says aligned kernels…", section "Zero mismatch expands to newer
+ * models"), the block-scaled products on the tensor cores, under the same batch-invariance
+ * contract as rz_token_logprobs (same vocabulary segments and per-row log-sum-exp).
+ *
+ *   Format: each row is cut into 32-element blocks along d; a block's scale is 2^X stored as
+ *   the byte X + 127 (UE8M0), X = floor(log2 max|x|) - 2 clamped to [-127, 127] (-127 for an
+ *   all-zero block); each element is the E2M1 value (0, 0.5, 1, 1.5, 2, 3, 4, 6 with a sign)
+ *   nearest to x / 2^X, ties to the even code, saturating at 6.
+ *   codes  [rows, d/2] bytes: element 2j in the low nibble of byte j, element 2j+1 in the high one.
+ *   scales rz_mxfp4_scale_bytes(rows, d) bytes, tiled: the scale of row r, block k (columns
+ *          32k .. 32k+31) is byte ((r/128)*(d/128) + k/4)*512 + (r%32)*16 + ((r%128)/32)*4 + k%4;
+ *          rows are padded with zero bytes to a multiple of 256.
+ *   d must be a multiple of 256 (256 <= d <= 32768).
+ *
+ *   rz_mxfp4_scale_bytes: size of the tiled scale array of `rows` rows (0 for an unsupported d).
+ *   rz_quantize_rows_mxfp4: X [rows, d] bf16 -> codes X4 and tiled scales (16-byte aligned X, X4).
+ *   rz_token_logprobs_mxfp4: z[t,v] = sum_k decode(H4)[t,k] decode(W4)[v,k] (exact products,
+ *     fp32 accumulation on the tensor cores), lp and lse as rz_token_logprobs; scale arrays
+ *     16-byte aligned; workspace size = rz_workspace_bytes_logprobs(n_tok, d, V).
+ */
+size_t rz_mxfp4_scale_bytes(int64_t rows, int32_t d);
+rz_status rz_quantize_rows_mxfp4(const rz_bf16* X, int64_t rows, int32_t d, uint8_t* X4, uint8_t* scales,
+                                 void* stream);
+rz_status rz_token_logprobs_mxfp4(const uint8_t* H4, const uint8_t* h_scales, const uint8_t* W4,
+                                  const uint8_t* w_scales, const int32_t* token_ids, int64_t n_tok, int32_t d,
+                                  int32_t V, float* lp_out, float* lse_out, void* workspace, size_t ws_bytes,
+                                  void* stream);
+
+/*
  * Cross-GPU consistency ("vLLM Train-Inference Consistency Release Notes", section
  * "Achieving Bitwise Consistency": communication reductions that do not vary with timing
  * or scheduling).  The reduction step of a data-parallel all-reduce of dW:

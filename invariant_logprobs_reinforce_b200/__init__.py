@@ -19,6 +19,7 @@ __all__ = [
     "rz_read_device_status", "rz_num_launches_loss", "rz_loss_fwd_bwd_timed", "rz_loss_fwd_bwd_ex",
     "rz_loss_fwd_bwd_streamed", "rz_loss_fwd_bwd_host_io", "rz_segment_loss_ex", "rz_ratio_stats", "rz_grad_norms", "rz_quantize_rows_e4m3",
     "rz_token_logprobs_fp8", "rz_sum_shards_f32", "rz_selftest_wait_timeout", "rz_token_logprobs_noalloc",
+    "rz_mxfp4_scale_bytes", "rz_quantize_rows_mxfp4", "rz_token_logprobs_mxfp4",
     "rz_workspace_bytes_ratio_stats", "rz_workspace_bytes_grad_norms", "rz_selftest_forward_after_timeout",
     "rz_loss_options", "loss_options",
     "EXPORTED_SYMBOLS", "STAT_NAMES", "KERNEL_KINDS",
@@ -37,7 +38,7 @@ EXPORTED_SYMBOLS = (
     "rz_segment_loss_ex",
     "rz_workspace_bytes_ratio_stats", "rz_ratio_stats", "rz_workspace_bytes_grad_norms", "rz_grad_norms",
     "rz_quantize_rows_e4m3", "rz_token_logprobs_fp8", "rz_sum_shards_f32", "rz_selftest_wait_timeout",
-    "rz_selftest_forward_after_timeout",
+    "rz_selftest_forward_after_timeout", "rz_mxfp4_scale_bytes", "rz_quantize_rows_mxfp4", "rz_token_logprobs_mxfp4",
 )
 RZ_LOSS_CLIP_IS, RZ_LOSS_SEQ_GATE, RZ_LOSS_TOKEN_MASK = 1, 2, 4
 STAT_NAMES = ("k1", "k2", "k3", "w_min", "w_max", "dev_max", "dev_median", "dev_peak_over_median", "count")
@@ -135,6 +136,12 @@ def lib() -> ctypes.CDLL:
         L.rz_quantize_rows_e4m3.restype = ctypes.c_int
         L.rz_token_logprobs_fp8.argtypes = [P, P, P, P, P, i64, i32, i32, P, P, P, sz, P]
         L.rz_token_logprobs_fp8.restype = ctypes.c_int
+        L.rz_mxfp4_scale_bytes.argtypes = [i64, i32]
+        L.rz_mxfp4_scale_bytes.restype = sz
+        L.rz_quantize_rows_mxfp4.argtypes = [P, i64, i32, P, P, P]
+        L.rz_quantize_rows_mxfp4.restype = ctypes.c_int
+        L.rz_token_logprobs_mxfp4.argtypes = [P, P, P, P, P, i64, i32, i32, P, P, P, sz, P]
+        L.rz_token_logprobs_mxfp4.restype = ctypes.c_int
         L.rz_sum_shards_f32.argtypes = [P, i32, i64, P, P]
         L.rz_sum_shards_f32.restype = ctypes.c_int
         L.rz_selftest_wait_timeout.argtypes = [ctypes.c_uint64, P, sz, ctypes.POINTER(ctypes.c_uint64), P]
@@ -637,6 +644,54 @@ def rz_token_logprobs_fp8(H8, h_scale, W8, w_scale, token_ids, lp_out=None, lse_
     code = lib().rz_token_logprobs_fp8(_ptr(H8), _ptr(h_scale), _ptr(W8), _ptr(w_scale), _ptr(token_ids), n, d, V,
                                        _ptr(lp), _ptr(lse), _ptr(ws), ws.numel(), _stream_handle(stream))
     _check(code, "rz_token_logprobs_fp8")
+    return lp, lse
+
+
+def rz_mxfp4_scale_bytes(rows: int, d: int) -> int:
+    return int(lib().rz_mxfp4_scale_bytes(rows, d))
+
+
+@_on_tensor_device
+def rz_quantize_rows_mxfp4(X, stream=None):
+    """bf16 [rows, d] -> (packed E2M1 codes uint8 [rows, d/2], tiled UE8M0 scales uint8
+    [rz_mxfp4_scale_bytes(rows, d)]); the layouts are those of include/rz.h."""
+    torch = _torch()
+    rows, d = _matrix(X, torch.bfloat16, "X")
+    nbytes = rz_mxfp4_scale_bytes(rows, d)
+    if nbytes == 0 and rows > 0:
+        raise ValueError(f"d = {d} is not supported (a multiple of 256 up to 32768)")
+    q = torch.empty((rows, d // 2), dtype=torch.uint8, device=X.device)
+    sc = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=X.device)
+    _check(lib().rz_quantize_rows_mxfp4(_ptr(X), rows, d, _ptr(q), _ptr(sc), _stream_handle(stream)),
+           "rz_quantize_rows_mxfp4")
+    return q, sc
+
+
+@_on_tensor_device
+def rz_token_logprobs_mxfp4(H4, h_scales, W4, w_scales, token_ids, lp_out=None, lse_out=None, workspace=None,
+                            stream=None, want_lse=True):
+    """Token logprobs from MXFP4 operands (codes [rows, d/2] and tiled scales from
+    rz_quantize_rows_mxfp4).  Returns (lp, lse)."""
+    torch = _torch()
+    n, half = _matrix(H4, torch.uint8, "H4")
+    dev = H4.device
+    V, half_w = _matrix(W4, torch.uint8, "W4", dev)
+    if half_w != half:
+        raise ValueError(f"W4 has {half_w} bytes per row, H4 has {half}")
+    d = 2 * half
+    for name, t, rows in (("h_scales", h_scales, n), ("w_scales", w_scales, V)):
+        _need(t, torch.uint8, name, dev)
+        if t.dim() != 1 or t.numel() < rz_mxfp4_scale_bytes(rows, d):
+            raise ValueError(f"{name} must be 1-D with at least rz_mxfp4_scale_bytes({rows}, {d}) bytes")
+    _need_shaped(token_ids, torch.int32, "token_ids", dev, (n,))
+    _need_shaped(lp_out, torch.float32, "lp_out", dev, (n,))
+    _need_shaped(lse_out, torch.float32, "lse_out", dev, (n,))
+    lp = lp_out if lp_out is not None else torch.empty(n, dtype=torch.float32, device=dev)
+    lse = lse_out if lse_out is not None else (torch.empty(n, dtype=torch.float32, device=dev) if want_lse else None)
+    ws = _workspace(rz_workspace_bytes_logprobs(n, d, V), workspace, dev)
+    code = lib().rz_token_logprobs_mxfp4(_ptr(H4), _ptr(h_scales), _ptr(W4), _ptr(w_scales), _ptr(token_ids), n, d,
+                                         V, _ptr(lp), _ptr(lse), _ptr(ws), ws.numel(), _stream_handle(stream))
+    _check(code, "rz_token_logprobs_mxfp4")
     return lp, lse
 
 

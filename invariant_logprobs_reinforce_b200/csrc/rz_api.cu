@@ -24,7 +24,7 @@
 #include <mutex>
 
 #include "../../include/rz.h"
-#include "rz_simt.cuh"
+#include "rz_mxf4.cuh"
 
 namespace rz {
 namespace {
@@ -376,6 +376,56 @@ rz_status run_forward_fp8(const uint8_t* H8, const float* hs, const uint8_t* W8,
     return RZ_ERR_CUDA;
   merge_lse_kernel<<<static_cast<unsigned>(ceil_div(n, 256)), 256, 0, stream>>>(
       e.part_m, e.part_s, L.part_ld, e.zy, ids, n, V, num_segments(V), lp, lse, status);
+  return cudaGetLastError() == cudaSuccess ? RZ_OK : RZ_ERR_CUDA;
+}
+
+// Forward from MXFP4 operands (kind::mxf4, block scales applied by the tensor cores): the
+// same vocabulary segments, per-row log-sum-exp arithmetic and merge as run_forward.
+rz_status run_forward_mxfp4(const uint8_t* H4, const uint8_t* hs, const uint8_t* W4, const uint8_t* wsc,
+                            const int32_t* ids, int64_t n, int32_t d, int32_t V, float* lp, float* lse, void* ws,
+                            const Layout& L, cudaStream_t stream) {
+  int* status = at<int>(ws, L.status);
+  CUtensorMap mH, mW;
+  // packed codes: d / 2 bytes per row, boxes of 128 bytes (256 elements) x rows
+  if (!make_map(&mH, CU_TENSOR_MAP_DATA_TYPE_UINT8, H4, d / 2, n, static_cast<uint64_t>(d / 2), 128, BM,
+                CU_TENSOR_MAP_SWIZZLE_128B))
+    return RZ_ERR_CUDA;
+  if (!make_map(&mW, CU_TENSOR_MAP_DATA_TYPE_UINT8, W4, d / 2, V, static_cast<uint64_t>(d / 2), 128, BN,
+                CU_TENSOR_MAP_SWIZZLE_128B))
+    return RZ_ERR_CUDA;
+  GemmSched s = make_sched(n, V, kSegTiles, forward_group_m(d / 2, 1), d);
+  s.num_kb = static_cast<int>(ceil_div(d, kMxKTile));
+  s.l2_pol_a = keep_if_fits(static_cast<uint64_t>(std::min<int64_t>(s.group_m * BM, n)) * (d / 2));
+  s.l2_pol_b = kL2EvictFirst;
+  MxfArgs a;
+  a.sfa = hs;
+  a.sfb = wsc;
+  a.d = d;
+  a.ids = ids;
+  a.rows = n;
+  a.V = V;
+  a.n_tiles = num_vocab_tiles(V);
+  a.part_m = at<float>(ws, L.part_m);
+  a.part_s = at<float>(ws, L.part_s);
+  a.part_ld = L.part_ld;
+  a.zy = at<float>(ws, L.zy);
+  static std::atomic<uint64_t> attr_done{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return RZ_ERR_CUDA;
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+  if (bit == 0 || !(attr_done.load(std::memory_order_acquire) & bit)) {
+    if (cudaFuncSetAttribute(lmhead_mxf4_lse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMxSmemBytes) !=
+        cudaSuccess)
+      return RZ_ERR_CUDA;
+    if (bit != 0) attr_done.fetch_or(bit, std::memory_order_acq_rel);
+  }
+  const int sms = sm_count();
+  if (sms <= 0) return RZ_ERR_CUDA;
+  lmhead_mxf4_lse_kernel<<<std::max(1, std::min(s.num_units, sms)), kGemmThreads, kMxSmemBytes, stream>>>(mH, mW, s,
+                                                                                                        a, status);
+  if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
+  merge_lse_kernel<<<static_cast<unsigned>(ceil_div(n, 256)), 256, 0, stream>>>(
+      a.part_m, a.part_s, L.part_ld, a.zy, ids, n, V, num_segments(V), lp, lse, status);
   return cudaGetLastError() == cudaSuccess ? RZ_OK : RZ_ERR_CUDA;
 }
 
@@ -1156,6 +1206,44 @@ RZ_API rz_status rz_token_logprobs_fp8(const uint8_t* H8, const float* h_scale, 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(at<int>(workspace, L.status), 0, 16, st) != cudaSuccess) return RZ_ERR_CUDA;
   return run_forward_fp8(H8, h_scale, W8, w_scale, token_ids, n_tok, d, V, lp_out, lse_out, workspace, L, st);
+}
+
+RZ_API size_t rz_mxfp4_scale_bytes(int64_t rows, int32_t d) {
+  if (rows < 0 || rows >= (int64_t{1} << 31) || d < 256 || d > 32768 || d % 256 != 0) return 0;
+  return static_cast<size_t>(mxfp4_scale_bytes(rows, d));
+}
+
+RZ_API rz_status rz_quantize_rows_mxfp4(const rz_bf16* X, int64_t rows, int32_t d, uint8_t* X4, uint8_t* scales,
+                                        void* stream) {
+  if (rows < 0 || rows >= (int64_t{1} << 31)) return RZ_ERR_INVALID_ARG;
+  if (d < 256 || d > 32768 || d % 256 != 0) return RZ_ERR_UNSUPPORTED_SHAPE;
+  if (rows == 0) return RZ_OK;
+  if (!X || !X4 || !scales || !aligned(X, 16) || !aligned(X4, 16)) return RZ_ERR_INVALID_ARG;
+  const int64_t padded = (rows + 255) / 256 * 256;
+  const int64_t threads = padded * (d / kMxBlock);
+  quantize_rows_mxfp4_kernel<<<static_cast<unsigned>(ceil_div(threads, 256)), 256, 0,
+                               static_cast<cudaStream_t>(stream)>>>(reinterpret_cast<const __nv_bfloat16*>(X), rows,
+                                                                    d, padded, X4, scales);
+  return cudaGetLastError() == cudaSuccess ? RZ_OK : RZ_ERR_CUDA;
+}
+
+RZ_API rz_status rz_token_logprobs_mxfp4(const uint8_t* H4, const uint8_t* h_scales, const uint8_t* W4,
+                                         const uint8_t* w_scales, const int32_t* token_ids, int64_t n_tok, int32_t d,
+                                         int32_t V, float* lp_out, float* lse_out, void* workspace, size_t ws_bytes,
+                                         void* stream) {
+  if (n_tok < 0 || n_tok >= (int64_t{1} << 31)) return RZ_ERR_INVALID_ARG;
+  if (!shape_ok(d, V) || d < 256 || d % 256 != 0) return RZ_ERR_UNSUPPORTED_SHAPE;
+  if (n_tok == 0) return RZ_OK;
+  if (!H4 || !h_scales || !W4 || !w_scales || !token_ids || !lp_out || !workspace) return RZ_ERR_INVALID_ARG;
+  if (!aligned(H4, 16) || !aligned(W4, 16) || !aligned(h_scales, 16) || !aligned(w_scales, 16) ||
+      !aligned(token_ids, 4) || !aligned(lp_out, 4) || (lse_out && !aligned(lse_out, 4)) ||
+      !aligned(workspace, kAlign))
+    return RZ_ERR_INVALID_ARG;
+  const Layout L = make_layout(n_tok, 0, 0, V, Path::Forward);
+  if (ws_bytes < L.total) return RZ_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(at<int>(workspace, L.status), 0, 16, st) != cudaSuccess) return RZ_ERR_CUDA;
+  return run_forward_mxfp4(H4, h_scales, W4, w_scales, token_ids, n_tok, d, V, lp_out, lse_out, workspace, L, st);
 }
 
 RZ_API rz_status rz_sum_shards_f32(const float* stacked, int32_t nshards, int64_t count, float* out, void* stream) {

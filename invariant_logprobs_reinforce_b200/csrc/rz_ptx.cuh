@@ -196,6 +196,38 @@ __device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
+// D[tmem] (+)= (A * sfa) * (B * sfb) with packed E2M1 (fp4) A and B, one UE8M0 scale per 32
+// elements along K (kind::mxf4, K = 64 per instruction), fp32 accumulate.  sfa_tmem / sfb_tmem
+// address the scale factors in TMEM (byte index within the 32-bit column in bits 30-31; the
+// instruction descriptor repeats it).
+__device__ __forceinline__ void umma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Copy a 32-row x 128-bit shared-memory matrix (described by `sdesc`) into TMEM at `taddr`,
+// replicated into the lanes of all four sub-partitions (lanes l, 32 + l, 64 + l, 96 + l get row
+// l); four 32-bit columns.  Executes in issue order with the tcgen05.mma of the same thread.
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// 1D bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned) from global to
+// shared memory, completing on `bar` (transaction bytes); no multicast.
+__device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                             uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+      : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05 op issued so far by this thread has completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -303,6 +335,27 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
 // accumulator; both operands K-major.
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
   return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Shared-memory descriptor of a plain (unswizzled) K-major matrix of 16-byte rows, 8-row core
+// matrices 128 bytes apart: the source of tcgen05.cp.32x128b (leading byte offset 16, stride
+// byte offset 128, descriptor version 1, layout type 0).
+__device__ __forceinline__ uint64_t smem_desc_rows16(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(16u >> 4) << 16;
+  d |= static_cast<uint64_t>(128u >> 4) << 32;
+  d |= 1ull << 46;
+  return d;
+}
+
+// Instruction descriptor, kind::mxf4 block-scaled: E2M1 A and B (format code 1 in bits [7,10)
+// and [10,13)), both K-major, UE8M0 scales (bit 23), fp32 accumulator, N >> 3 in bits [17,23),
+// M >> 4 in bits [24,29); the scale factors' byte index within their TMEM column in bits
+// [4,6) (B) and [29,31) (A).
+__host__ __device__ constexpr uint32_t idesc_mxf4_f32(int M, int N, uint32_t a_sf_id, uint32_t b_sf_id) {
+  return (b_sf_id << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
+         (static_cast<uint32_t>(M >> 4) << 24) | (a_sf_id << 29);
 }
 
 // ---------------------------------------------------------------- math

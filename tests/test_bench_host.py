@@ -147,7 +147,7 @@ def _fake_result():
                 n_tok=360896, G=64, R=512, value=468908.2, ms_per_step=769.6, dominant="lmhead_lse",
                 traffic=None, peak_src="fallback", clocks={"sm_mhz": 1155.0}, launches=2820,
                 e2e={"value": 4.4e5}, kernels=kern, invariance={"diff": 0}, loss_stage=ls, fwd_tok_s=1.5e6,
-                fwd_ms=240.0, fwd8_ms=160.0, workloads={"lag64_1437610_tok": {"fwd_bwd_tok_s": 4.6e5}})
+                fwd_ms=240.0, fwd8_ms=160.0, fwd4_ms=100.0, workloads={"lag64_1437610_tok": {"fwd_bwd_tok_s": 4.6e5}})
 
 
 def test_line_puts_the_contract_keys_first_and_the_compact_figures_last():
@@ -157,11 +157,12 @@ def test_line_puts_the_contract_keys_first_and_the_compact_figures_last():
     keys = list(line)
     assert keys[:13] == ["metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
                          "scaling", "vs_baseline", "dtype", "data", "config"]
-    assert keys[-5:] == ["tensor_frac_6dV", "fwd_only", "fwd_only_fp8", "loss_stage_frac", "workloads"]
+    assert keys[-6:] == ["tensor_frac_6dV", "fwd_only", "fwd_only_fp8", "fwd_only_mxfp4", "loss_stage_frac",
+                         "workloads"]
     assert line["roofline"]["frac"] == pytest.approx(1075.0 / 1400.0)
     assert line["kernels"]["lmhead_lse"]["frac_of_peak"] == 0.7691  # rounded to 4 significant digits
     # the compact tail fits in the part of the output a log tail keeps
-    tail = json.dumps({k: line[k] for k in keys[-5:]})
+    tail = json.dumps({k: line[k] for k in keys[-6:]})
     assert len(tail) < 1500
 
 

@@ -57,3 +57,22 @@ def test_one_rank_data_parallel_step_equals_the_single_gpu_call(rz):
         assert torch.equal(a["dH"].view(torch.int16), b["dH"].view(torch.int16))
     finally:
         dist.destroy_process_group()
+
+
+def test_bench_data_parallel_mode_at_world_size_one():
+    """bench.py --dp on one GPU: the whole-group shard is the whole (capped) batch, the
+    deterministic all-reduce runs through a one-rank NCCL group, and the line reports a
+    clean status and the same dW bits on every rank."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_PORT")}
+    r = subprocess.run([sys.executable, "bench.py", "--dp", "--steps", "2", "--warmup", "1", "--n-tok-cap", "20000"],
+                       cwd=root, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-3000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["scaling"] == "strong" and line["n_gpus"] == 1
+    assert line["status_ok"] and line["dW_same_bits_on_all_ranks"]
+    assert line["value"] > 0 and line["gpu_launches"] > 0
