@@ -100,14 +100,19 @@ def _operands(rz, n, d, V, seed):
     return H, W, ids, H4, hs, W4, ws
 
 
+def _oracle_operand(X, rows_per_call=4096):
+    """bf16 bits of the oracle's decoded MXFP4 quantisation of X.  The oracle works row by
+    row; it is called on row ranges so that its per-element temporaries stay small."""
+    bits = X.view(torch.int16).cpu().numpy().view(np.uint16)
+    out = np.empty_like(bits)
+    for r0 in range(0, bits.shape[0], rows_per_call):
+        codes, scales = mxfp4.quantize_rows_mxfp4(bits[r0:r0 + rows_per_call])
+        out[r0:r0 + rows_per_call] = _decoded_bits(codes, scales)
+    return out
+
+
 def _oracle_lp(H, W, ids):
-    n, d = H.shape
-    V = W.shape[0]
-    Hb = H.view(torch.int16).cpu().numpy().view(np.uint16)
-    Wb = W.view(torch.int16).cpu().numpy().view(np.uint16)
-    hc, hsc = mxfp4.quantize_rows_mxfp4(Hb)
-    wc, wsc = mxfp4.quantize_rows_mxfp4(Wb)
-    return dense.token_logprobs(_decoded_bits(hc, hsc), _decoded_bits(wc, wsc), ids.cpu().numpy())
+    return dense.token_logprobs(_oracle_operand(H), _oracle_operand(W), ids.cpu().numpy())
 
 
 @pytest.mark.parametrize("n,d,V,seed", [
