@@ -506,10 +506,14 @@ rz_status run_kappa(const float* lp, const float* lp_roll, const int64_t* off, i
   const int vec_ok = aligned(lp, 16) && aligned(lp_roll, 16) && aligned(kappa, 16) &&
                      (w_out == nullptr || aligned(w_out, 16)) && (opt.mask == nullptr || aligned(opt.mask, 4));
   rec_begin(rec, RZ_KERNEL_TOKEN_KAPPA, stream);
-  token_kappa_kernel<<<nblk, kKappaThreads, 0, stream>>>(lp, lp_roll, off, R, at<float>(ws, L.coef),
-                                                         at<int>(ws, L.bfirst), n, blk0, vec_ok, opt.mask,
-                                                         opt.clip_max, kappa, w_out, at<double>(ws, L.bsum),
-                                                         kappa_blocks(n), at<int>(ws, L.status) + 3, loss);
+  // min(w, +inf) = w, so the unclipped variant gives the same bits as a clip at +inf would
+  const bool masked = opt.mask != nullptr, clipped = !std::isinf(opt.clip_max);
+  auto kernel = masked ? (clipped ? token_kappa_kernel<true, true> : token_kappa_kernel<true, false>)
+                       : (clipped ? token_kappa_kernel<false, true> : token_kappa_kernel<false, false>);
+  kernel<<<nblk, kKappaThreads, 0, stream>>>(lp, lp_roll, off, R, at<float>(ws, L.coef), at<int>(ws, L.bfirst), n,
+                                             blk0, vec_ok, opt.mask, opt.clip_max, kappa, w_out,
+                                             at<double>(ws, L.bsum), kappa_blocks(n), at<int>(ws, L.status) + 3,
+                                             loss);
   if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
   rec_end(rec, stream);
   return RZ_OK;

@@ -238,6 +238,9 @@ __global__ void __launch_bounds__(kSetupThreads)
 // finds its first token's response by a short walk and then advances with one compare
 // per token (a boundary can only fall between two consecutive tokens).  Otherwise the
 // block walks the global offsets.
+// MASKED / CLIPPED: compiled variants with and without the token mask and the truncated-IS
+// cap, so the plain call carries neither per-token test (the arithmetic is the same).
+template <bool MASKED, bool CLIPPED>
 __global__ void __launch_bounds__(kKappaThreads, 5)
     token_kappa_kernel(const float* __restrict__ lp, const float* __restrict__ lp_roll,
                        const int64_t* __restrict__ off, int R, const float* __restrict__ coef,
@@ -273,7 +276,7 @@ __global__ void __launch_bounds__(kKappaThreads, 5)
       const int64_t t0 = b0 + wrel + it * 128 + lane * 4;
       la[it] = __ldcs(reinterpret_cast<const float4*>(lp + t0));
       lb[it] = __ldcs(reinterpret_cast<const float4*>(lp_roll + t0));
-      mk[it] = mask != nullptr ? __ldcs(reinterpret_cast<const unsigned int*>(mask + t0)) : 0x01010101u;
+      mk[it] = MASKED ? __ldcs(reinterpret_cast<const unsigned int*>(mask + t0)) : 0x01010101u;
     }
   }
   __syncthreads();
@@ -309,7 +312,8 @@ __global__ void __launch_bounds__(kKappaThreads, 5)
           ck = s_coef[k];
         }
         w[j] = ex2_approx((a4[j] - b4[j]) * kLog2e);
-        kv[j] = ((m4 >> (8 * j)) & 0xffu) ? ck * fminf(w[j], clip_max) : 0.0f;
+        const float g = CLIPPED ? fminf(w[j], clip_max) : w[j];
+        kv[j] = (!MASKED || ((m4 >> (8 * j)) & 0xffu)) ? ck * g : 0.0f;
         part += kv[j];
       }
       const int64_t t0 = b0 + tr;
@@ -328,7 +332,8 @@ __global__ void __launch_bounds__(kKappaThreads, 5)
           const int64_t t = t0 + j;
           while (i + 1 < R && __ldg(off + i + 1) <= t) ++i;
           const float w = ex2_approx((lp[t] - lp_roll[t]) * kLog2e);
-          const float kv = (mask == nullptr || mask[t] != 0) ? __ldg(coef + i) * fminf(w, clip_max) : 0.0f;
+          const float g = CLIPPED ? fminf(w, clip_max) : w;
+          const float kv = (!MASKED || mask[t] != 0) ? __ldg(coef + i) * g : 0.0f;
           kappa[t] = kv;
           if (w_out != nullptr) w_out[t] = w;
           part += kv;
