@@ -583,6 +583,21 @@ def run_e2e(rz, torch, dev, stream, H, W, ids, lp_roll, rewards, off, gid, G, n,
                           "out: dH, dW, lp, loss"}
 
 
+def first_tokens(prob, n, group_size):
+    """The problem cut to its first n tokens: the responses that start before token n, the
+    last one shortened to end at n, in groups of `group_size` consecutive responses (the last
+    possibly partial).  Returns (problem, n_resp)."""
+    import workloads as wl
+    seg = prob.seg
+    R = int(np.searchsorted(seg.seg_offsets, n, side="left"))
+    off = seg.seg_offsets[:R + 1].copy()
+    off[-1] = n
+    gid = (np.arange(R) // group_size).astype(np.int32)
+    G = int(gid[-1]) + 1
+    sub = wl.Segments(off, gid, seg.rewards[:R].copy(), G)
+    return wl.Problem(prob.H[:n], prob.W, prob.ids[:n], sub, prob.d, prob.V, prob.noise, prob.seed), R
+
+
 def _time_calls(torch, stream, fn, reps, warm=1):
     """Mean milliseconds per call of fn() over `reps` calls (CUDA events on `stream`)."""
     for _ in range(warm):
@@ -626,7 +641,9 @@ def run_workloads(rz, torch, dev, stream, peak_tflops):
     del H, W, ids, lp, ws
 
     for name, cap in (("lag64", None), ("moe_head", 1 << 20)):
-        prob = wl.full_config(name, device=str(dev), n_tok_cap=cap)
+        prob = wl.full_config(name, device=str(dev), n_tok_cap=None if cap is None else cap + (1 << 17))
+        if cap is not None:  # exactly `cap` tokens: the responses up to it, the last one cut short
+            prob, _ = first_tokens(prob, cap, wl.CONFIGS[name]["group_size"])
         seg = prob.seg
         n, d, V = prob.n_tok, prob.d, prob.V
         lp0, _ = rz.rz_token_logprobs(prob.H, prob.W, prob.ids, want_lse=False)
@@ -746,7 +763,8 @@ def run_sweep(args, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     stream = torch.cuda.current_stream()
-    prob = wl.full_config(args.workload, device=str(dev), n_tok_cap=args.n_tok_cap or (1 << 20))
+    # a little more than 2^20 tokens in whole groups, so that the 2^20 point exists
+    prob = wl.full_config(args.workload, device=str(dev), n_tok_cap=args.n_tok_cap or ((1 << 20) + (1 << 17)))
     seg = prob.seg
     d, V = prob.d, prob.V
     peaks, src = load_peaks()

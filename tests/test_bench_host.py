@@ -173,3 +173,17 @@ def test_dp_line_reports_strong_scaling():
              dW_same_bits_on_all_ranks=True, clocks=None, launches=60, n_resp=512, n_groups=64)
     line = bench.make_dp_line(args, 8, r)
     assert line["scaling"] == "strong" and line["n_gpus"] == 8 and line["dW_same_bits_on_all_ranks"]
+
+
+def test_first_tokens_cuts_the_batch_at_exactly_n():
+    import numpy as np
+    import workloads as wl
+    seg = wl.draw_segments("moe_head")
+    prob = wl.Problem(np.zeros((seg.n_tok, 1), np.uint16), None, np.zeros(seg.n_tok, np.int32), seg, 1, 1)
+    for n in (4096, 1 << 20, int(seg.seg_offsets[40])):
+        sub, R = bench.first_tokens(prob, n, 16)
+        off = sub.seg.seg_offsets
+        assert sub.n_tok == n and off[0] == 0 and off[-1] == n and np.all(np.diff(off) >= 1)
+        assert np.array_equal(off[:-1], seg.seg_offsets[:R])          # the same response starts
+        assert np.array_equal(sub.seg.group_ids, np.arange(R) // 16)   # groups of 16
+        assert sub.seg.n_groups == (R + 15) // 16
