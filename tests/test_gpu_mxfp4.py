@@ -100,19 +100,33 @@ def _operands(rz, n, d, V, seed):
     return H, W, ids, H4, hs, W4, ws
 
 
-def _oracle_operand(X, rows_per_call=4096):
-    """bf16 bits of the oracle's decoded MXFP4 quantisation of X.  The oracle works row by
-    row; it is called on row ranges so that its per-element temporaries stay small."""
+def oracle_decoded_chunk(bits):
+    """The oracle's MXFP4 quantisation of some rows, decoded, as bf16 bits (a process-pool task)."""
+    codes, scales = mxfp4.quantize_rows_mxfp4(bits)
+    return _decoded_bits(codes, scales)
+
+
+@pytest.fixture(scope="module")
+def pool():
+    """Host processes for the oracle, started with spawn (a forked child of a process that has
+    used CUDA can hang); the oracle is row-wise, so row ranges go to the workers."""
+    import concurrent.futures
+    import multiprocessing
+    import os
+    workers = max(1, min(16, os.cpu_count() or 1))
+    with concurrent.futures.ProcessPoolExecutor(workers, mp_context=multiprocessing.get_context("spawn")) as ex:
+        yield ex
+
+
+def _oracle_operand(X, pool, rows_per_call=2048):
+    """bf16 bits of the oracle's decoded MXFP4 quantisation of X, row range by row range."""
     bits = X.view(torch.int16).cpu().numpy().view(np.uint16)
-    out = np.empty_like(bits)
-    for r0 in range(0, bits.shape[0], rows_per_call):
-        codes, scales = mxfp4.quantize_rows_mxfp4(bits[r0:r0 + rows_per_call])
-        out[r0:r0 + rows_per_call] = _decoded_bits(codes, scales)
-    return out
+    chunks = [bits[r0:r0 + rows_per_call] for r0 in range(0, bits.shape[0], rows_per_call)]
+    return np.concatenate(list(pool.map(oracle_decoded_chunk, chunks)), axis=0)
 
 
-def _oracle_lp(H, W, ids):
-    return dense.token_logprobs(_oracle_operand(H), _oracle_operand(W), ids.cpu().numpy())
+def _oracle_lp(H, W, ids, pool):
+    return dense.token_logprobs(_oracle_operand(H, pool), _oracle_operand(W, pool), ids.cpu().numpy())
 
 
 @pytest.mark.parametrize("n,d,V,seed", [
@@ -122,11 +136,11 @@ def _oracle_lp(H, W, ids):
     (512, 2560, 151936, 14),    # the Qwen3-4B head
     (256, 7168, 129280, 15),    # the MoE head
 ])
-def test_logprobs_match_the_oracle_on_the_decoded_operands(rz, n, d, V, seed):
+def test_logprobs_match_the_oracle_on_the_decoded_operands(rz, pool, n, d, V, seed):
     H, W, ids, H4, hs, W4, ws = _operands(rz, n, d, V, seed)
     lp, lse = rz.rz_token_logprobs_mxfp4(H4, hs, W4, ws, ids)
     torch.cuda.synchronize()
-    lp_o, lse_o = _oracle_lp(H, W, ids)
+    lp_o, lse_o = _oracle_lp(H, W, ids, pool)
     assert np.abs(lp.cpu().numpy() - lp_o).max() <= h.LP_ATOL
     assert np.abs(lse.cpu().numpy() - lse_o).max() <= h.LP_ATOL
 
