@@ -1119,12 +1119,13 @@ size_t stats_parts_off() { return kAlign; }
 size_t stats_hist_off(int64_t n) { return align_up(stats_parts_off() + sizeof(StatPartial) * stat_blocks(n), kAlign); }
 size_t stats_sel_off(int64_t n) { return align_up(stats_hist_off(n) + sizeof(unsigned) * kStatBins, kAlign); }
 size_t stats_acc_off(int64_t n) { return align_up(stats_sel_off(n) + 16, kAlign); }
+size_t stats_k3_off(int64_t n) { return align_up(stats_acc_off(n) + sizeof(StatPartial), kAlign); }
 constexpr int kNormBlocks = 1184;  // 8 per SM on 148 SMs; fixed, so the partial order is fixed
 }  // namespace
 
 RZ_API size_t rz_workspace_bytes_ratio_stats(int64_t n_tok, int32_t n_resp) {
   if (n_tok < 1 || n_tok >= (int64_t{1} << 31) || n_resp < 1) return 0;
-  return align_up(stats_acc_off(n_tok) + sizeof(StatPartial), kAlign);
+  return align_up(stats_k3_off(n_tok) + sizeof(double) * stat_blocks(n_tok), kAlign);
 }
 
 RZ_API rz_status rz_ratio_stats(const float* lp, const float* lp_rollout, const int64_t* seg_offsets, int64_t n_tok,
@@ -1153,13 +1154,14 @@ RZ_API rz_status rz_ratio_stats(const float* lp, const float* lp_rollout, const 
   const int grid = std::min(nb, kStatCtasPerSm * sms);
   ratio_stats_pass0<<<nb, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, vec, nb, parts, hist);
   ratio_stats_reduce<<<1, 1024, 0, st>>>(parts, nb, acc, sel);
-  ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, kStatBins, 11, sel, acc, 0, stats_out);
+  double* k3_parts = at<double>(workspace, stats_k3_off(n_tok));
+  ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, kStatBins, 11, sel, acc, 0, stats_out, k3_parts, nb);
   ratio_stats_pass<<<grid, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, vec, nb, sel, 21, 10, 0x7ffu,
-                                                  hist);
-  ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, kStatBins, 11, sel, acc, 0, stats_out);
+                                                  hist, 0, k3_parts);
+  ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, kStatBins, 11, sel, acc, 0, stats_out, k3_parts, nb);
   ratio_stats_pass<<<grid, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, vec, nb, sel, 10, 0, 0x3ffu,
-                                                  hist);
-  ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, 1024, 10, sel, acc, 1, stats_out);
+                                                  hist, 1, k3_parts);
+  ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, 1024, 10, sel, acc, 1, stats_out, k3_parts, nb);
   if (resp_mean_ratio_out != nullptr)
     response_mean_ratio_kernel<<<static_cast<unsigned>(ceil_div(n_resp, 8)), 256, 0, st>>>(
         lp, lp_rollout, token_mask, seg_offsets, n_resp, resp_mean_ratio_out);

@@ -527,7 +527,7 @@ __device__ __forceinline__ void load_stat_quads(const float* __restrict__ lp, co
 // (one block per CTA when the grid covers them all): each block's fp64 partial is computed
 // the same way whichever CTA takes it, so the statistics do not depend on the grid, and a
 // CTA adds its shared histogram into the global one once, at the end (integer counts).
-__global__ void __launch_bounds__(kStatThreads)
+__global__ void __launch_bounds__(kStatThreads, kStatCtasPerSm)
     ratio_stats_pass0(const float* __restrict__ lp, const float* __restrict__ lp_roll, const uint8_t* __restrict__ mask,
                       int64_t n, bool vec, int nblk, StatPartial* __restrict__ parts, unsigned* __restrict__ hist) {
   __shared__ unsigned s_hist[kStatBins];
@@ -553,7 +553,6 @@ __global__ void __launch_bounds__(kStatThreads)
           const float dev = fabsf(w - 1.0f);
           k1 -= x;
           k2 += 0.5 * x * x;
-          k3 += expm1_minus_x(x);
           wmin = fminf(wmin, w);
           wmax = fmaxf(wmax, w);
           dmax = fmaxf(dmax, dev);
@@ -593,18 +592,27 @@ __global__ void __launch_bounds__(kStatThreads)
     if (s_hist[b]) atomicAdd(&hist[b], s_hist[b]);
 }
 
-// Histogram of the next radix digit among the deviations whose higher bits equal `prefix`.
-__global__ void __launch_bounds__(kStatThreads)
+// Histogram of the next radix digit among the deviations whose higher bits equal `prefix`,
+// and the k3 sum of the 4096-token blocks whose index has parity `k3_parity` (the fp64 series
+// is the heaviest arithmetic of the statistics: split over the two radix passes, which stream
+// at copy speed with issue slots to spare, it keeps every pass near the memory time).  A
+// block's k3 partial is formed the same way whichever CTA takes the block (per-thread sums
+// in token order, warp butterfly, warps in order), so it does not depend on the grid.
+__global__ void __launch_bounds__(kStatThreads, kStatCtasPerSm)
     ratio_stats_pass(const float* __restrict__ lp, const float* __restrict__ lp_roll, const uint8_t* __restrict__ mask,
                      int64_t n, bool vec, int nblk, const unsigned* __restrict__ sel, int shift_hi, int shift,
-                     unsigned digit_mask, unsigned* __restrict__ hist) {
+                     unsigned digit_mask, unsigned* __restrict__ hist, int k3_parity,
+                     double* __restrict__ k3_parts) {
   __shared__ unsigned s_hist[kStatBins];
+  __shared__ double s_k3[kStatThreads / 32];
   for (int b = threadIdx.x; b < kStatBins; b += kStatThreads) s_hist[b] = 0u;
   const unsigned prefix = sel[0];
   __syncthreads();
   for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x) {
     StatQuads q;
     load_stat_quads(lp, lp_roll, mask, n, vec, blk, q);
+    const bool with_k3 = (blk & 1) == k3_parity;  // uniform across the CTA
+    double k3 = 0.0;
 #pragma unroll
     for (int k = 0; k < kStatQuads; ++k) {
 #pragma unroll
@@ -612,8 +620,21 @@ __global__ void __launch_bounds__(kStatThreads)
         if (q.on[k][i]) {
           const unsigned key = __float_as_uint(fabsf(ratio_of(q.a[k][i], q.b[k][i]) - 1.0f));
           if ((key >> shift_hi) == prefix) hist_add(s_hist, (key >> shift) & digit_mask, true);
+          if (with_k3) k3 += expm1_minus_x(static_cast<double>(q.a[k][i]) - static_cast<double>(q.b[k][i]));
         }
       }
+    }
+    if (with_k3) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) k3 += __shfl_xor_sync(0xffffffffu, k3, o);
+      if ((threadIdx.x & 31) == 0) s_k3[threadIdx.x >> 5] = k3;
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        double sum = s_k3[0];
+        for (int w = 1; w < kStatThreads / 32; ++w) sum += s_k3[w];
+        k3_parts[blk] = sum;
+      }
+      __syncthreads();  // s_k3 is rewritten by the next block
     }
   }
   __syncthreads();
@@ -671,8 +692,20 @@ static_assert(2 * kSelectThreads >= kStatBins, "two bins per thread");
 
 __global__ void __launch_bounds__(kSelectThreads)
     ratio_stats_select(unsigned* __restrict__ hist, int nbins, int digit_bits, unsigned* __restrict__ sel,
-                       const StatPartial* __restrict__ acc_in, int last, double* __restrict__ stats) {
+                       const StatPartial* __restrict__ acc_in, int last, double* __restrict__ stats,
+                       const double* __restrict__ k3_parts, int nblk) {
   __shared__ unsigned s_warp[kSelectThreads / 32];
+  __shared__ double s_k3[kSelectThreads];
+  if (last) {  // the k3 sum of all blocks: strided per thread, then a fixed tree
+    double a = 0.0;
+    for (int b = threadIdx.x; b < nblk; b += kSelectThreads) a += k3_parts[b];
+    s_k3[threadIdx.x] = a;
+    __syncthreads();
+    for (int w = kSelectThreads >> 1; w > 0; w >>= 1) {
+      if (threadIdx.x < w) s_k3[threadIdx.x] += s_k3[threadIdx.x + w];
+      __syncthreads();
+    }
+  }
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int b0 = 2 * threadIdx.x;
   const unsigned h0 = b0 < nbins ? hist[b0] : 0u;
@@ -723,7 +756,7 @@ __global__ void __launch_bounds__(kSelectThreads)
   const double med = static_cast<double>(__uint_as_float(med_bits));
   stats[0] = acc.k1 / m;
   stats[1] = acc.k2 / m;
-  stats[2] = acc.k3 / m;
+  stats[2] = s_k3[0] / m;
   stats[3] = acc.w_min;
   stats[4] = acc.w_max;
   stats[5] = acc.dev_max;
