@@ -479,7 +479,7 @@ rz_status run_loss_setup(const float* rewards, const int64_t* off, const int32_t
     if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
   }
   const int nb = kappa_blocks(n);
-  const unsigned grid = static_cast<unsigned>(ceil_div(std::max<int64_t>(R, nb), kSetupThreads));
+  const unsigned grid = static_cast<unsigned>(ceil_div(R, kSetupThreads));
   loss_setup_kernel<<<grid, kSetupThreads, 0, stream>>>(rewards, off, gid, R, G, n, opt.N, counted,
                                                         at<double>(ws, L.gsum), at<int>(ws, L.gcnt),
                                                         at<float>(ws, L.coef), nb, at<int>(ws, L.bfirst), flags,

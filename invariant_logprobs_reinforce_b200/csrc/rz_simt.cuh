@@ -133,7 +133,9 @@ __device__ __forceinline__ int find_response(const int64_t* __restrict__ off, in
 //    non-decreasing; a thread that starts a run of equal valid ids sums the run's rewards
 //    (fp64, response order) and, since with non-decreasing ids a run is the whole group,
 //    writes coef_j = -A_j / (N L_j) for every response of the run;
-//  - thread b < nblocks writes the first response of 4096-token block b;
+//  - thread i < R writes i as the first response of every 4096-token block that starts
+//    inside response i (after a failed segment check some blocks may keep stale entries;
+//    the ratio / kappa kernel clamps what it reads, and the outputs carry no meaning then);
 //  - the last block to finish (a ticket on `ticket`, cleared with the status word) redoes
 //    the group sums by scanning the responses in index order and rewrites every coef when
 //    the ids were not sorted.  Either way a group's rewards are added in response order,
@@ -199,7 +201,15 @@ __global__ void __launch_bounds__(kSetupThreads)
       for (int j = i; j < i + c; ++j) coef[j] = response_coef(rewards, off, gid, G, N, counted, sum, c, j);
     }
   }
-  if (i < nblocks) bfirst[i] = find_response(off, R, min(n - 1, static_cast<int64_t>(i) * kKappaBlockTokens));
+  // first responses of the 4096-token blocks: block b starts at token b * 4096, which lies in
+  // the response i with off[i] <= b * 4096 < off[i + 1], i.e. b in [ceil(off[i] / 4096),
+  // ceil(off[i + 1] / 4096)); with valid offsets every block is written once, by that response
+  if (i < R) {
+    const int64_t o0 = off[i], o1 = off[i + 1];
+    const int64_t b_hi = min(static_cast<int64_t>(nblocks), (o1 + kKappaBlockTokens - 1) / kKappaBlockTokens);
+    for (int64_t b = max(static_cast<int64_t>(0), (o0 + kKappaBlockTokens - 1) / kKappaBlockTokens); b < b_hi; ++b)
+      bfirst[b] = i;
+  }
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) s_last = atomicAdd(ticket, 1) == static_cast<int>(gridDim.x) - 1;
