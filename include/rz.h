@@ -95,7 +95,10 @@ size_t rz_workspace_bytes_segment_loss(int64_t n_tok, int32_t n_resp, int32_t n_
  *
  * Logits are never written to memory: a fused tensor-core kernel computes H W^T tile by
  * tile and keeps an online log-sum-exp per row over fixed vocabulary segments, then a
- * second kernel merges the segments in fixed order.  n_tok == 0 is a no-op.
+ * second kernel merges the segments in fixed order.  A call of few rows (too few row blocks
+ * to occupy the GPU with one unit per segment) runs one unit per 256-column tile and the
+ * merge replays the same per-tile folds: the bits are the same either way.  n_tok == 0 is
+ * a no-op.
  */
 rz_status rz_token_logprobs(const rz_bf16* H, const rz_bf16* W_head, const int32_t* token_ids, int64_t n_tok,
                             int32_t d, int32_t V, float* lp_out, float* lse_out, void* workspace,
@@ -394,8 +397,9 @@ rz_status rz_loss_fwd_bwd_timed(const rz_bf16* H, const rz_bf16* W_head, const i
  * Arguments and results are those of rz_token_logprobs (same kernels, same bits), minus
  * the workspace.  The scratch is a fixed array of RZ_NOALLOC_SCRATCH_BYTES inside the
  * library, held by every GPU that loads the library until the process exits.  A call
- * needs 256 + 4*n_tok*(2*ceil(V/2048) + 1) bytes of it (rounded up to 256-byte pieces):
- * at V = 151936 that is about 55,000 tokens per call.  Larger calls return
+ * needs 256 + 4*n_tok*(2*C + 1) bytes of it (rounded up to 256-byte pieces), C =
+ * ceil(V/2048), or C = ceil(V/256) for a call of few rows (ceil(n_tok/128)*ceil(V/2048) <
+ * 296): at V = 151936 that is about 55,000 tokens per call.  Larger calls return
  * RZ_ERR_WORKSPACE_TOO_SMALL and enqueue nothing; split them into several calls.
  *
  * The first call on each device looks up the scratch address (cudaGetSymbolAddress)

@@ -42,6 +42,14 @@ bool shape_ok(int32_t d, int32_t V) { return d >= 64 && d <= 32768 && d % 64 == 
 int num_segments(int32_t V) { return static_cast<int>(ceil_div(V, kSegWidth)); }
 int num_vocab_tiles(int32_t V) { return static_cast<int>(ceil_div(V, BN)); }
 
+// A forward-only call whose (row block, segment) units would leave most SMs idle (a decode
+// step of a few rows) runs one unit per 256-column tile instead and the merge folds each
+// segment's tiles in order (merge_lse_kernel): the same bits, with up to eight times the
+// units.  The threshold is a constant (two units per SM of a 148-SM B200), not a query of
+// the device, so workspace sizes do not depend on the device.
+constexpr int64_t kTileUnitsBelow = 296;
+bool tile_units(int64_t rows, int32_t V) { return ceil_div(rows, BM) * num_segments(V) < kTileUnitsBelow; }
+
 int64_t padded_vocab(int32_t V) { return align_up(static_cast<size_t>(V), 8); }
 
 int kappa_blocks(int64_t n) { return static_cast<int>(ceil_div(n, static_cast<int64_t>(kKappaBlockTokens))); }
@@ -77,7 +85,8 @@ Layout make_layout(int64_t n, int32_t R, int32_t G, int32_t V, Path path) {
   };
   L.status = take(16);
   if (path != Path::LossStage) {
-    const int S = num_segments(V);
+    // partial columns: one per segment, or one per tile for a forward call of few row blocks
+    const int S = (path == Path::Forward && tile_units(n, V)) ? num_vocab_tiles(V) : num_segments(V);
     L.part_ld = path == Path::Forward ? n : chunk_capacity(n);
     L.part_m = take(sizeof(float) * static_cast<size_t>(S) * L.part_ld);
     L.part_s = take(sizeof(float) * static_cast<size_t>(S) * L.part_ld);
@@ -281,13 +290,14 @@ GemmSched make_sched(int64_t m_rows, int64_t n_cols, int tiles_per_unit, int gro
 // exponentials e = exp(z - tile_max) and the tile maxima for the backward.
 rz_status run_forward(const rz_bf16* H, const rz_bf16* W, const int32_t* ids, int64_t r0, int64_t rows, int32_t d,
                       int32_t V, float* lp, float* lse, void* ws, const Layout& L, bool store_p, cudaStream_t stream,
-                      Recorder* rec) {
+                      Recorder* rec, bool allow_tile_units = false) {
   int* status = at<int>(ws, L.status);
   CUtensorMap mH, mW;
   // rows past the range read as zeros, so no other rows' data enters the launch
   if (!make_operand_map(&mH, H, d, r0 + rows, static_cast<uint64_t>(d) * 2, BM)) return RZ_ERR_CUDA;
   if (!make_operand_map(&mW, W, d, V, static_cast<uint64_t>(d) * 2, BN)) return RZ_ERR_CUDA;
-  GemmSched s = make_sched(rows, V, kSegTiles, forward_group_m(d, 2), d);
+  const bool per_tile = allow_tile_units && !store_p && tile_units(rows, V);
+  GemmSched s = make_sched(rows, V, per_tile ? 1 : kSegTiles, forward_group_m(d, 2), d);
   s.l2_pol_a = keep_if_fits(static_cast<uint64_t>(std::min<int64_t>(s.group_m * BM, rows)) * d * 2);
   s.l2_pol_b = store_p ? kL2Normal : kL2EvictFirst;
   const OperandPos pos{static_cast<int>(r0), 0, 0, 0};
@@ -334,7 +344,8 @@ rz_status run_forward(const rz_bf16* H, const rz_bf16* W, const int32_t* ids, in
   const int threads = 256;
   rec_begin(rec, RZ_KERNEL_MERGE_LSE, stream);
   merge_lse_kernel<<<static_cast<unsigned>(ceil_div(rows, threads)), threads, 0, stream>>>(
-      part_m, part_s, L.part_ld, zy, ids + r0, rows, V, num_segments(V), lp + r0, lse ? lse + r0 : nullptr, status);
+      part_m, part_s, L.part_ld, zy, ids + r0, rows, V, num_segments(V), lp + r0, lse ? lse + r0 : nullptr, status,
+      per_tile ? num_vocab_tiles(V) : 0);
   if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
   rec_end(rec, stream);
   return RZ_OK;
@@ -734,7 +745,7 @@ rz_status forward_on_workspace(const rz_bf16* H, const rz_bf16* W_head, const in
                                                    at<unsigned long long>(ws, L.status + 16));
     if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
   }
-  return run_forward(H, W_head, token_ids, 0, n_tok, d, V, lp_out, lse_out, ws, L, false, st, nullptr);
+  return run_forward(H, W_head, token_ids, 0, n_tok, d, V, lp_out, lse_out, ws, L, false, st, nullptr, true);
 }
 
 }  // namespace

@@ -29,6 +29,17 @@ constexpr int kSegWidth = kSegTiles * BN;  // 2048 vocabulary columns
 // the order in which token contributions reach dW never depends on n_tok).
 constexpr int kChunkTokens = 16384;
 
+// Fold one tile's (maximum, sum of exponentials) pair into a row's running pair, in a fixed
+// rounding order (explicit fp32 operations, no contraction left to the compiler), so that the
+// epilogue and a later merge that replays the same folds give the same bits:
+//   m' = max(m, tmax);  s' = s 2^((m - m') log2 e) + tsum 2^((tmax - m') log2 e)
+// From (m, s) = (-inf, 0) the first fold gives exactly (tmax, tsum).
+__device__ __forceinline__ void lse_fold(float& m, float& s, float tmax, float tsum) {
+  const float m_new = fmaxf(m, tmax);
+  s = __fmaf_rn(s, ex2_approx(__fmul_rn(m - m_new, kLog2e)), __fmul_rn(tsum, ex2_approx(__fmul_rn(tmax - m_new, kLog2e))));
+  m = m_new;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&p);
@@ -183,9 +194,7 @@ struct EpiLse {
       }
     });
     const float tmax = st.rs * ymax;
-    const float m_new = fmaxf(st.m, tmax);
-    st.s = st.s * ex2_approx((st.m - m_new) * kLog2e) + tsum * ex2_approx((tmax - m_new) * kLog2e);
-    st.m = m_new;
+    lse_fold(st.m, st.s, tmax, tsum);
     if constexpr (STORE_P) {
       if (st.row < rows) tile_max[st.row * n_tiles + nt] = tmax;
     }

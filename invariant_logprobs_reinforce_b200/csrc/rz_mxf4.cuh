@@ -381,9 +381,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[acc]);
-        const float m_new = fmaxf(m, ymax);
-        s = s * ex2_approx((m - m_new) * kLog2e) + tsum * ex2_approx((ymax - m_new) * kLog2e);
-        m = m_new;
+        lse_fold(m, s, ymax, tsum);
       }
       if (aborted) break;
       if (row < args.rows) {

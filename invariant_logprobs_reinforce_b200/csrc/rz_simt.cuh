@@ -35,13 +35,18 @@ namespace rz {
 // lse = M + log(sum_s s_s 2^{(m_s - M) log2 e}), segments merged in order s = 0..S-1.
 // Pointers are launch-relative; the partials have row stride part_ld.
 //
+// n_tiles > 0: the partials are per 256-column tile (calls with too few row blocks to fill
+// the GPU with one unit per segment run one unit per tile) and each segment's pair is first
+// rebuilt by folding its tiles' pairs in order with lse_fold, exactly as the epilogue folds
+// them when a unit is a whole segment: the same bits either way.
+//
 // If a wait of an earlier kernel of the same call gave up (the timeout bit of the status
 // word is set), some partials were never written and may hold an earlier call's values:
 // every lp and lse of the launch is then NaN instead of a plausible wrong number.
 __global__ void merge_lse_kernel(const float* __restrict__ part_m, const float* __restrict__ part_s,
                                  int64_t part_ld, const float* __restrict__ zy, const int32_t* __restrict__ ids,
                                  int64_t n, int V, int S, float* __restrict__ lp, float* __restrict__ lse_out,
-                                 int* status) {
+                                 int* status, int n_tiles = 0) {
   const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (t >= n) return;
   if (*reinterpret_cast<volatile const int*>(status) & kDevWaitTimeout) {
@@ -49,12 +54,30 @@ __global__ void merge_lse_kernel(const float* __restrict__ part_m, const float* 
     if (lse_out != nullptr) lse_out[t] = __int_as_float(0x7fc00000);
     return;
   }
+  // pair of segment s: stored, or folded from its tiles
+  auto segment = [&](int s, float& m, float& sm) {
+    if (n_tiles == 0) {
+      m = part_m[static_cast<int64_t>(s) * part_ld + t];
+      sm = part_s[static_cast<int64_t>(s) * part_ld + t];
+      return;
+    }
+    m = -INFINITY;
+    sm = 0.0f;
+    for (int k = s * kSegTiles; k < min(n_tiles, (s + 1) * kSegTiles); ++k)
+      lse_fold(m, sm, part_m[static_cast<int64_t>(k) * part_ld + t], part_s[static_cast<int64_t>(k) * part_ld + t]);
+  };
   float M = -INFINITY;
-  for (int s = 0; s < S; ++s) M = fmaxf(M, part_m[static_cast<int64_t>(s) * part_ld + t]);
+  for (int s = 0; s < S; ++s) {
+    float m, sm;
+    segment(s, m, sm);
+    M = fmaxf(M, m);
+  }
   float sum = 0.0f;
-  for (int s = 0; s < S; ++s)
-    sum += part_s[static_cast<int64_t>(s) * part_ld + t] *
-           ex2_approx((part_m[static_cast<int64_t>(s) * part_ld + t] - M) * kLog2e);
+  for (int s = 0; s < S; ++s) {
+    float m, sm;
+    segment(s, m, sm);
+    sum += sm * ex2_approx((m - M) * kLog2e);
+  }
   const float l = M + logf(sum);
   const int y = ids[t];
   if (y < 0 || y >= V) {
