@@ -510,10 +510,14 @@ rz_status run_gate(const float* lp, const float* lp_roll, const int64_t* off, in
 }
 
 // Loss stage, part 2: kappa and ratio for the 4096-token blocks [blk0, blk0 + nblk); the
-// block that finishes last of all the call's blocks writes the loss.
+// block that finishes last of all the call's blocks writes the loss.  after_setup: the
+// kernel directly before this one on the stream is the setup kernel, so this one is
+// launched as its programmatic dependent (its lp / lp_rollout loads overlap the setup; it
+// waits for the setup's results before reading them).  Only then: lp may come from the
+// kernel before, which a programmatic launch would not wait for.
 rz_status run_kappa(const float* lp, const float* lp_roll, const int64_t* off, int64_t n, int32_t R, int blk0,
                     int nblk, const LossOpts& opt, float* kappa, float* w_out, float* loss, void* ws, const Layout& L,
-                    cudaStream_t stream, Recorder* rec) {
+                    cudaStream_t stream, Recorder* rec, bool after_setup = false) {
   const int vec_ok = aligned(lp, 16) && aligned(lp_roll, 16) && aligned(kappa, 16) &&
                      (w_out == nullptr || aligned(w_out, 16)) && (opt.mask == nullptr || aligned(opt.mask, 4));
   rec_begin(rec, RZ_KERNEL_TOKEN_KAPPA, stream);
@@ -521,11 +525,21 @@ rz_status run_kappa(const float* lp, const float* lp_roll, const int64_t* off, i
   const bool masked = opt.mask != nullptr, clipped = !std::isinf(opt.clip_max);
   auto kernel = masked ? (clipped ? token_kappa_kernel<true, true> : token_kappa_kernel<true, false>)
                        : (clipped ? token_kappa_kernel<false, true> : token_kappa_kernel<false, false>);
-  kernel<<<nblk, kKappaThreads, 0, stream>>>(lp, lp_roll, off, R, at<float>(ws, L.coef), at<int>(ws, L.bfirst), n,
-                                             blk0, vec_ok, opt.mask, opt.clip_max, kappa, w_out,
-                                             at<double>(ws, L.bsum), kappa_blocks(n), at<int>(ws, L.status) + 3,
-                                             loss);
-  if (cudaGetLastError() != cudaSuccess) return RZ_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(nblk));
+  cfg.blockDim = dim3(kKappaThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = (after_setup && rec == nullptr) ? 1 : 0;  // a recorded event in between would end the overlap
+  const float* coef = at<float>(ws, L.coef);
+  const int* bfirst = at<int>(ws, L.bfirst);
+  const int total = kappa_blocks(n);
+  if (cudaLaunchKernelEx(&cfg, kernel, lp, lp_roll, off, R, coef, bfirst, n, blk0, vec_ok, opt.mask, opt.clip_max,
+                         kappa, w_out, at<double>(ws, L.bsum), total, at<int>(ws, L.status) + 3, loss) != cudaSuccess)
+    return RZ_ERR_CUDA;
   rec_end(rec, stream);
   return RZ_OK;
 }
@@ -540,7 +554,8 @@ rz_status run_segment_loss(const float* lp, const float* lp_roll, const float* r
     r = run_gate(lp, lp_roll, off, R, opt, ws, L, stream);
     if (r != RZ_OK) return r;
   }
-  return run_kappa(lp, lp_roll, off, n, R, 0, kappa_blocks(n), opt, kappa, w_out, loss, ws, L, stream, rec);
+  return run_kappa(lp, lp_roll, off, n, R, 0, kappa_blocks(n), opt, kappa, w_out, loss, ws, L, stream, rec,
+                   /*after_setup=*/!opt.gate);
 }
 
 // A non-blocking stream per device for device-to-host copies of results, created on
@@ -1136,7 +1151,7 @@ constexpr int kNormBlocks = 1184;  // 8 per SM on 148 SMs; fixed, so the partial
 
 RZ_API size_t rz_workspace_bytes_ratio_stats(int64_t n_tok, int32_t n_resp) {
   if (n_tok < 1 || n_tok >= (int64_t{1} << 31) || n_resp < 1) return 0;
-  return align_up(stats_k3_off(n_tok) + sizeof(double) * stat_blocks(n_tok), kAlign);
+  return align_up(stats_k3_off(n_tok) + sizeof(double) * 2 * stat_blocks(n_tok), kAlign);
 }
 
 RZ_API rz_status rz_ratio_stats(const float* lp, const float* lp_rollout, const int64_t* seg_offsets, int64_t n_tok,
@@ -1166,13 +1181,14 @@ RZ_API rz_status rz_ratio_stats(const float* lp, const float* lp_rollout, const 
   ratio_stats_pass0<<<nb, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, vec, nb, parts, hist);
   ratio_stats_reduce<<<1, 1024, 0, st>>>(parts, nb, acc, sel);
   double* k3_parts = at<double>(workspace, stats_k3_off(n_tok));
-  ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, kStatBins, 11, sel, acc, 0, stats_out, k3_parts, nb);
-  ratio_stats_pass<<<grid, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, vec, nb, sel, 21, 10, 0x7ffu,
-                                                  hist, 0, k3_parts);
-  ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, kStatBins, 11, sel, acc, 0, stats_out, k3_parts, nb);
-  ratio_stats_pass<<<grid, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, vec, nb, sel, 10, 0, 0x3ffu,
-                                                  hist, 1, k3_parts);
-  ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, 1024, 10, sel, acc, 1, stats_out, k3_parts, nb);
+  const int nk3 = 2 * nb;  // two k3 half-sums per token block, one from each radix pass
+  ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, kStatBins, 11, sel, acc, 0, stats_out, k3_parts, nk3);
+  ratio_stats_pass<0><<<grid, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, vec, nb, sel, 21, 10, 0x7ffu,
+                                                     hist, k3_parts);
+  ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, kStatBins, 11, sel, acc, 0, stats_out, k3_parts, nk3);
+  ratio_stats_pass<1><<<grid, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, vec, nb, sel, 10, 0, 0x3ffu,
+                                                     hist, k3_parts);
+  ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, 1024, 10, sel, acc, 1, stats_out, k3_parts, nk3);
   if (resp_mean_ratio_out != nullptr)
     response_mean_ratio_kernel<<<static_cast<unsigned>(ceil_div(n_resp, 8)), 256, 0, st>>>(
         lp, lp_rollout, token_mask, seg_offsets, n_resp, resp_mean_ratio_out);

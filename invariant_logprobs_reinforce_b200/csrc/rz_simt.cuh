@@ -153,28 +153,38 @@ __device__ __forceinline__ int find_response(const int64_t* __restrict__ off, in
 
 // The loss stage's setup in one launch:
 //  - thread i < R checks response i (segments, group id) and flags ids that are not
-//    non-decreasing; a thread that starts a run of equal valid ids sums the run's rewards
-//    (fp64, response order) and, since with non-decreasing ids a run is the whole group,
-//    writes coef_j = -A_j / (N L_j) for every response of the run;
+//    non-decreasing;
+//  - coef_i = -A_i / (N L_i) from the sum of the rewards of the run of equal valid ids that
+//    holds response i, added in response order from the run's first response (with
+//    non-decreasing ids a run is the whole group); the run's first response also writes the
+//    group's sum and count.  A warp covers 32 consecutive responses and loads their fields
+//    at once; a run inside the window is summed from registers (shuffles, in order), and
+//    only a run that crosses the window's edge reads the neighbouring responses, 32 at a
+//    time;
 //  - thread i < R writes i as the first response of every 4096-token block that starts
 //    inside response i (after a failed segment check some blocks may keep stale entries;
 //    the ratio / kappa kernel clamps what it reads, and the outputs carry no meaning then);
 //  - the last block to finish (a ticket on `ticket`, cleared with the status word) redoes
 //    the group sums by scanning the responses in index order and rewrites every coef when
-//    the ids were not sorted.  Either way a group's rewards are added in response order,
-//    so both give the same bits.
+//    the ids were not sorted.  Either way a group's rewards are added in response order
+//    from 0, so both give the same bits.
 // counted (nullable): tokens per response under a token mask (masked_count_kernel).
 constexpr int kSetupThreads = 256;
+
+// coef_i from response i's reward, counted length L, validity and its group's (sum, count)
+__device__ __forceinline__ float coef_of(float reward, int64_t L, bool bad, double gsum_g, int gcnt_g, double N) {
+  if (bad || gcnt_g <= 0) return __int_as_float(0x7fc00000);
+  if (L <= 0) return 0.0f;  // every token of the response is masked out: it contributes nothing
+  const double A = static_cast<double>(reward) - gsum_g / static_cast<double>(gcnt_g);
+  return static_cast<float>(-A / (N * static_cast<double>(L)));
+}
 
 __device__ __forceinline__ float response_coef(const float* __restrict__ rewards, const int64_t* __restrict__ off,
                                                const int32_t* __restrict__ gid, int G, double N,
                                                const int* __restrict__ counted, double gsum_g, int gcnt_g, int i) {
   const int g = gid[i];
   const int64_t L = counted != nullptr ? counted[i] : off[i + 1] - off[i];
-  if (g < 0 || g >= G || off[i + 1] <= off[i] || gcnt_g <= 0) return __int_as_float(0x7fc00000);
-  if (L <= 0) return 0.0f;  // every token of the response is masked out: it contributes nothing
-  const double A = static_cast<double>(rewards[i]) - gsum_g / static_cast<double>(gcnt_g);
-  return static_cast<float>(-A / (N * static_cast<double>(L)));
+  return coef_of(rewards[i], L, g < 0 || g >= G || off[i + 1] <= off[i], gsum_g, gcnt_g, N);
 }
 
 __global__ void __launch_bounds__(kSetupThreads)
@@ -184,51 +194,105 @@ __global__ void __launch_bounds__(kSetupThreads)
                       float* __restrict__ coef, int nblocks, int* __restrict__ bfirst, int* flags, int* ticket,
                       int* status) {
   __shared__ bool s_last;
+  // the kappa kernel that follows may start launching now: it waits for this grid to
+  // finish before it reads anything written here
+  grid_dependents_launch();
+  constexpr unsigned kAll = 0xffffffffu;
+  const int lane = threadIdx.x & 31;
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < R) {
+  const int w0 = i - lane;  // the warp's first response
+  const bool in = i < R;
+  // every field of response i, loaded at once
+  const int g = in ? gid[i] : 0;
+  const bool has_next = in && i + 1 < R;
+  const int g_next = has_next ? gid[i + 1] : 0;
+  const int g_prev = (lane == 0 && in && i > 0) ? gid[i - 1] : 0;
+  const float r = in ? rewards[i] : 0.0f;
+  const int64_t o0 = in ? off[i] : 0, o1 = in ? off[i + 1] : 0;
+  const int64_t L = (in && counted != nullptr) ? counted[i] : o1 - o0;
+  const bool gvalid = in && g >= 0 && g < G;
+  if (in) {
     int bad = 0;
-    if (i == 0 && (off[0] != 0 || off[R] != n)) bad |= kDevBadSegments;
-    if (off[i + 1] <= off[i]) bad |= kDevBadSegments;
-    const int g = gid[i];
-    if (g < 0 || g >= G) bad |= kDevBadGroupId;
+    if (i == 0 && (o0 != 0 || off[R] != n)) bad |= kDevBadSegments;
+    if (o1 <= o0) bad |= kDevBadSegments;
+    if (!gvalid) bad |= kDevBadGroupId;
     if (bad) atomicOr(status, bad);
-    if (i + 1 < R && gid[i + 1] < g) atomicOr(flags, 1);
-    if (g < 0 || g >= G) {
-      coef[i] = __int_as_float(0x7fc00000);
-    } else if (i == 0 || gid[i - 1] != g) {  // the start of a run of equal ids
-      // the run's rewards in response order; ids and rewards are loaded four at a time so
-      // that a run costs a quarter of the dependent round trips
-      double sum = 0.0;
-      int c = 0;
-      bool open = true;
-      for (int j0 = i; open && j0 < R; j0 += 4) {
-        int gj[4];
-        float rj[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          gj[u] = j0 + u < R ? gid[j0 + u] : -1;
-          rj[u] = j0 + u < R ? rewards[j0 + u] : 0.0f;
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          open = open && gj[u] == g;
-          if (open) {
-            sum += static_cast<double>(rj[u]);
-            ++c;
-          }
-        }
+    if (has_next && g_next < g) atomicOr(flags, 1);
+  }
+  // runs of equal valid ids in the window: a lane starts one when its id differs from the
+  // previous response's (lane 0: from response w0 - 1); an invalid or absent response
+  // breaks every run
+  const int g_left = __shfl_up_sync(kAll, g, 1);
+  const bool brk = !gvalid || (lane == 0 ? (i == 0 || g_prev != g) : g_left != g);
+  const unsigned B = __ballot_sync(kAll, brk);
+  const unsigned upto = B & (kAll >> (31 - lane));  // starts at lanes <= lane
+  const unsigned above = B & ~(kAll >> (31 - lane));
+  const int ls = upto ? 31 - __clz(upto) : 0;  // the lane's run, clipped to the window
+  const int le = above ? __ffs(above) - 2 : 31;
+  // the run of lane 0, if it began in an earlier window: its responses before w0, in order
+  double sum = 0.0;
+  int c = 0;
+  if (__shfl_sync(kAll, gvalid && !brk, 0)) {
+    const int g0 = __shfl_sync(kAll, g, 0);
+    int start = w0;
+    for (int base = w0 - 32;; base -= 32) {  // its first response, 32 at a time
+      const int j = base + lane;
+      const unsigned m = __ballot_sync(kAll, !(j >= 0 && gid[j] == g0));
+      if (m) {
+        start = base + 32 - __clz(m);
+        break;
       }
-      gsum[g] = sum;  // with sorted ids every group is one run, so one writer per group
-      gcnt[g] = c;
-#pragma unroll 4
-      for (int j = i; j < i + c; ++j) coef[j] = response_coef(rewards, off, gid, G, N, counted, sum, c, j);
     }
+    double acc = 0.0;
+    for (int base = start; base < w0; base += 32) {
+      const int j = base + lane;
+      const float rj = j < w0 ? rewards[j] : 0.0f;
+      const int nk = min(32, w0 - base);
+      for (int k = 0; k < 32; ++k) {
+        const float v = __shfl_sync(kAll, rj, k);
+        if (k < nk) acc += static_cast<double>(v);
+      }
+    }
+    if (upto == 0) {  // the lanes of that run
+      sum = acc;
+      c = w0 - start;
+    }
+  }
+  // the window's part of the lane's run, in order
+  for (int k = 0; k < 32; ++k) {
+    const float v = __shfl_sync(kAll, r, k);
+    if (k >= ls && k <= le) sum += static_cast<double>(v);
+  }
+  c += le - ls + 1;
+  // the run of lane 31, if it goes on past the window: its responses after, in order
+  if (__shfl_sync(kAll, gvalid && has_next && g_next == g, 31)) {
+    const int g31 = __shfl_sync(kAll, g, 31);
+    const bool last_run = le == 31;
+    for (int base = w0 + 32;; base += 32) {
+      const int j = base + lane;
+      const bool same = j < R && gid[j] == g31;
+      const float rj = j < R ? rewards[j] : 0.0f;
+      const unsigned m = __ballot_sync(kAll, !same);
+      const int nk = m ? __ffs(m) - 1 : 32;
+      for (int k = 0; k < 32; ++k) {
+        const float v = __shfl_sync(kAll, rj, k);
+        if (last_run && k < nk) sum += static_cast<double>(v);
+      }
+      if (last_run) c += nk;
+      if (nk < 32) break;
+    }
+  }
+  if (in) {
+    if (gvalid && brk) {  // the run's first response; with sorted ids one writer per group
+      gsum[g] = sum;
+      gcnt[g] = c;
+    }
+    coef[i] = coef_of(r, L, !gvalid || o1 <= o0, sum, c, N);
   }
   // first responses of the 4096-token blocks: block b starts at token b * 4096, which lies in
   // the response i with off[i] <= b * 4096 < off[i + 1], i.e. b in [ceil(off[i] / 4096),
   // ceil(off[i + 1] / 4096)); with valid offsets every block is written once, by that response
-  if (i < R) {
-    const int64_t o0 = off[i], o1 = off[i + 1];
+  if (in) {
     const int64_t b_hi = min(static_cast<int64_t>(nblocks), (o1 + kKappaBlockTokens - 1) / kKappaBlockTokens);
     for (int64_t b = max(static_cast<int64_t>(0), (o0 + kKappaBlockTokens - 1) / kKappaBlockTokens); b < b_hi; ++b)
       bfirst[b] = i;
@@ -292,13 +356,6 @@ __global__ void __launch_bounds__(kKappaThreads, 5)
   const int blk = block0 + blockIdx.x;
   const int64_t b0 = static_cast<int64_t>(blk) * kKappaBlockTokens;
   const int nb = static_cast<int>(min(n - b0, static_cast<int64_t>(kKappaBlockTokens)));  // tokens in the block
-  const int i0 = min(max(block_first[blk], 0), R - 1);
-  const int cnt = min(kKappaStagedOffsets, R - i0);
-  for (int k = threadIdx.x; k <= cnt; k += kKappaThreads) {
-    const int64_t o = (i0 + k < R) ? off[i0 + k] - b0 : kFar;
-    s_rel[k] = static_cast<int>(max(min(o, static_cast<int64_t>(kFar)), static_cast<int64_t>(-kFar)));
-    if (k < cnt) s_coef[k] = coef[i0 + k];
-  }
   const bool full = vec_ok && nb == kKappaBlockTokens;
   const int wrel = warp * (kKappaBlockTokens / 8);
   float4 la[kKappaIters], lb[kKappaIters];
@@ -311,6 +368,16 @@ __global__ void __launch_bounds__(kKappaThreads, 5)
       lb[it] = __ldcs(reinterpret_cast<const float4*>(lp_roll + t0));
       mk[it] = MASKED ? __ldcs(reinterpret_cast<const unsigned int*>(mask + t0)) : 0x01010101u;
     }
+  }
+  // launched as a programmatic dependent of the setup kernel, the block's token loads above
+  // overlap the setup; everything below reads what the setup wrote
+  grid_dependency_wait();
+  const int i0 = min(max(block_first[blk], 0), R - 1);
+  const int cnt = min(kKappaStagedOffsets, R - i0);
+  for (int k = threadIdx.x; k <= cnt; k += kKappaThreads) {
+    const int64_t o = (i0 + k < R) ? off[i0 + k] - b0 : kFar;
+    s_rel[k] = static_cast<int>(max(min(o, static_cast<int64_t>(kFar)), static_cast<int64_t>(-kFar)));
+    if (k < cnt) s_coef[k] = coef[i0 + k];
   }
   __syncthreads();
   // the staged responses cover the block when the first starts at or before its first
@@ -626,16 +693,17 @@ __global__ void __launch_bounds__(kStatThreads, kStatCtasPerSm)
 }
 
 // Histogram of the next radix digit among the deviations whose higher bits equal `prefix`,
-// and the k3 sum of the 4096-token blocks whose index has parity `k3_parity` (the fp64 series
-// is the heaviest arithmetic of the statistics: split over the two radix passes, which stream
-// at copy speed with issue slots to spare, it keeps every pass near the memory time).  A
-// block's k3 partial is formed the same way whichever CTA takes the block (per-thread sums
-// in token order, warp butterfly, warps in order), so it does not depend on the grid.
+// and half of the k3 sum: in every 4096-token block, each thread's quads k with k % 2 ==
+// K3_HALF (the fp64 series is the heaviest arithmetic of the statistics; split evenly over
+// the two radix passes, which stream at copy speed with issue slots to spare, it costs every
+// SM the same).  The block's half-sum goes to k3_parts[2 blk + K3_HALF], formed the same way
+// whichever CTA takes the block (per-thread sums in token order, warp butterfly, warps in
+// order), so it does not depend on the grid.
+template <int K3_HALF>
 __global__ void __launch_bounds__(kStatThreads, kStatCtasPerSm)
     ratio_stats_pass(const float* __restrict__ lp, const float* __restrict__ lp_roll, const uint8_t* __restrict__ mask,
                      int64_t n, bool vec, int nblk, const unsigned* __restrict__ sel, int shift_hi, int shift,
-                     unsigned digit_mask, unsigned* __restrict__ hist, int k3_parity,
-                     double* __restrict__ k3_parts) {
+                     unsigned digit_mask, unsigned* __restrict__ hist, double* __restrict__ k3_parts) {
   __shared__ unsigned s_hist[kStatBins];
   __shared__ double s_k3[kStatThreads / 32];
   for (int b = threadIdx.x; b < kStatBins; b += kStatThreads) s_hist[b] = 0u;
@@ -644,7 +712,6 @@ __global__ void __launch_bounds__(kStatThreads, kStatCtasPerSm)
   for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x) {
     StatQuads q;
     load_stat_quads(lp, lp_roll, mask, n, vec, blk, q);
-    const bool with_k3 = (blk & 1) == k3_parity;  // uniform across the CTA
     double k3 = 0.0;
 #pragma unroll
     for (int k = 0; k < kStatQuads; ++k) {
@@ -653,24 +720,21 @@ __global__ void __launch_bounds__(kStatThreads, kStatCtasPerSm)
         if (q.on[k][i]) {
           const unsigned key = __float_as_uint(fabsf(ratio_of(q.a[k][i], q.b[k][i]) - 1.0f));
           if ((key >> shift_hi) == prefix) hist_add(s_hist, (key >> shift) & digit_mask, true);
-          if (with_k3) k3 += expm1_minus_x(static_cast<double>(q.a[k][i]) - static_cast<double>(q.b[k][i]));
+          if (k % 2 == K3_HALF) k3 += expm1_minus_x(static_cast<double>(q.a[k][i]) - static_cast<double>(q.b[k][i]));
         }
       }
     }
-    if (with_k3) {
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) k3 += __shfl_xor_sync(0xffffffffu, k3, o);
-      if ((threadIdx.x & 31) == 0) s_k3[threadIdx.x >> 5] = k3;
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        double sum = s_k3[0];
-        for (int w = 1; w < kStatThreads / 32; ++w) sum += s_k3[w];
-        k3_parts[blk] = sum;
-      }
-      __syncthreads();  // s_k3 is rewritten by the next block
+    for (int o = 16; o > 0; o >>= 1) k3 += __shfl_xor_sync(0xffffffffu, k3, o);
+    if ((threadIdx.x & 31) == 0) s_k3[threadIdx.x >> 5] = k3;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      double sum = s_k3[0];
+      for (int w = 1; w < kStatThreads / 32; ++w) sum += s_k3[w];
+      k3_parts[2 * static_cast<int64_t>(blk) + K3_HALF] = sum;
     }
+    __syncthreads();  // s_k3 is rewritten by the next block
   }
-  __syncthreads();
   for (int b = threadIdx.x; b < kStatBins; b += kStatThreads)
     if (s_hist[b]) atomicAdd(&hist[b], s_hist[b]);
 }
@@ -726,12 +790,12 @@ static_assert(2 * kSelectThreads >= kStatBins, "two bins per thread");
 __global__ void __launch_bounds__(kSelectThreads)
     ratio_stats_select(unsigned* __restrict__ hist, int nbins, int digit_bits, unsigned* __restrict__ sel,
                        const StatPartial* __restrict__ acc_in, int last, double* __restrict__ stats,
-                       const double* __restrict__ k3_parts, int nblk) {
+                       const double* __restrict__ k3_parts, int nk3) {
   __shared__ unsigned s_warp[kSelectThreads / 32];
   __shared__ double s_k3[kSelectThreads];
-  if (last) {  // the k3 sum of all blocks: strided per thread, then a fixed tree
+  if (last) {  // the k3 sum of all block halves: strided per thread, then a fixed tree
     double a = 0.0;
-    for (int b = threadIdx.x; b < nblk; b += kSelectThreads) a += k3_parts[b];
+    for (int b = threadIdx.x; b < nk3; b += kSelectThreads) a += k3_parts[b];
     s_k3[threadIdx.x] = a;
     __syncthreads();
     for (int w = kSelectThreads >> 1; w > 0; w >>= 1) {
