@@ -369,7 +369,7 @@ rz_status run_forward_fp8(const uint8_t* H8, const float* hs, const uint8_t* W8,
   s.l2_pol_a = keep_if_fits(static_cast<uint64_t>(std::min<int64_t>(s.group_m * BM, n)) * d);  // e4m3
   s.l2_pol_b = kL2EvictFirst;
   const OperandPos pos{0, 0, 0, 0};
-  EpiLse<false> e;
+  EpiLse<false, true> e;
   std::memset(&e.p_map, 0, sizeof(e.p_map));
   e.ids = ids;
   e.rows = n;
@@ -383,7 +383,7 @@ rz_status run_forward_fp8(const uint8_t* H8, const float* hs, const uint8_t* W8,
   e.row_scale = hs;
   e.col_scale = wsc;
   e.col_scale_vec = aligned(wsc, 16) ? 1 : 0;
-  if (launch_gemm<false, false, EpiLse<false>, true>(mH, mW, s, pos, e, status, stream) != cudaSuccess)
+  if (launch_gemm<false, false, EpiLse<false, true>, true>(mH, mW, s, pos, e, status, stream) != cudaSuccess)
     return RZ_ERR_CUDA;
   merge_lse_kernel<<<static_cast<unsigned>(ceil_div(n, 256)), 256, 0, stream>>>(
       e.part_m, e.part_s, L.part_ld, e.zy, ids, n, V, num_segments(V), lp, lse, status);
@@ -509,6 +509,21 @@ rz_status run_gate(const float* lp, const float* lp_roll, const int64_t* off, in
   return cudaGetLastError() == cudaSuccess ? RZ_OK : RZ_ERR_CUDA;
 }
 
+// The kappa kernels' dynamic shared memory (bulk-copy stages) exceeds the default limit:
+// raised once per device and variant (devices done kept as bits, as for the GEMM kernels).
+cudaError_t ensure_kappa_smem_attr(bool masked, bool clipped, const void* kernel, int smem) {
+  static std::atomic<uint64_t> done[4];
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  std::atomic<uint64_t>& word = done[(masked ? 2 : 0) + (clipped ? 1 : 0)];
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+  if (bit != 0 && (word.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (err == cudaSuccess && bit != 0) word.fetch_or(bit, std::memory_order_acq_rel);
+  return err;
+}
+
 // Loss stage, part 2: kappa and ratio for the 4096-token blocks [blk0, blk0 + nblk); the
 // block that finishes last of all the call's blocks writes the loss.  after_setup: the
 // kernel directly before this one on the stream is the setup kernel, so this one is
@@ -518,16 +533,24 @@ rz_status run_gate(const float* lp, const float* lp_roll, const int64_t* off, in
 rz_status run_kappa(const float* lp, const float* lp_roll, const int64_t* off, int64_t n, int32_t R, int blk0,
                     int nblk, const LossOpts& opt, float* kappa, float* w_out, float* loss, void* ws, const Layout& L,
                     cudaStream_t stream, Recorder* rec, bool after_setup = false) {
+  // whole blocks are bulk-copied into shared memory and kappa / w are stored four at a
+  // time: both need 16-byte aligned arrays (a 4096-token block then starts 16-byte aligned)
   const int vec_ok = aligned(lp, 16) && aligned(lp_roll, 16) && aligned(kappa, 16) &&
-                     (w_out == nullptr || aligned(w_out, 16)) && (opt.mask == nullptr || aligned(opt.mask, 4));
+                     (w_out == nullptr || aligned(w_out, 16)) && (opt.mask == nullptr || aligned(opt.mask, 16));
   rec_begin(rec, RZ_KERNEL_TOKEN_KAPPA, stream);
   // min(w, +inf) = w, so the unclipped variant gives the same bits as a clip at +inf would
   const bool masked = opt.mask != nullptr, clipped = !std::isinf(opt.clip_max);
   auto kernel = masked ? (clipped ? token_kappa_kernel<true, true> : token_kappa_kernel<true, false>)
                        : (clipped ? token_kappa_kernel<false, true> : token_kappa_kernel<false, false>);
+  const int smem = masked ? KappaSmem<true>::kBytes : KappaSmem<false>::kBytes;
+  if (ensure_kappa_smem_attr(masked, clipped, reinterpret_cast<const void*>(kernel), smem) != cudaSuccess)
+    return RZ_ERR_CUDA;
+  const int sms = sm_count();
+  if (sms <= 0) return RZ_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(nblk));
+  cfg.gridDim = dim3(static_cast<unsigned>(std::max(1, std::min(nblk, kKappaCtasPerSm * sms))));
   cfg.blockDim = dim3(kKappaThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -536,9 +559,10 @@ rz_status run_kappa(const float* lp, const float* lp_roll, const int64_t* off, i
   cfg.numAttrs = (after_setup && rec == nullptr) ? 1 : 0;  // a recorded event in between would end the overlap
   const float* coef = at<float>(ws, L.coef);
   const int* bfirst = at<int>(ws, L.bfirst);
-  const int total = kappa_blocks(n);
-  if (cudaLaunchKernelEx(&cfg, kernel, lp, lp_roll, off, R, coef, bfirst, n, blk0, vec_ok, opt.mask, opt.clip_max,
-                         kappa, w_out, at<double>(ws, L.bsum), total, at<int>(ws, L.status) + 3, loss) != cudaSuccess)
+  int* status = at<int>(ws, L.status);
+  if (cudaLaunchKernelEx(&cfg, kernel, lp, lp_roll, off, R, coef, bfirst, n, blk0, nblk, vec_ok, opt.mask,
+                         opt.clip_max, kappa, w_out, at<double>(ws, L.bsum), kappa_blocks(n), status + 3, loss,
+                         status) != cudaSuccess)
     return RZ_ERR_CUDA;
   rec_end(rec, stream);
   return RZ_OK;
@@ -1149,6 +1173,24 @@ size_t stats_k3_off(int64_t n) { return align_up(stats_acc_off(n) + sizeof(StatP
 constexpr int kNormBlocks = 1184;  // 8 per SM on 148 SMs; fixed, so the partial order is fixed
 }  // namespace
 
+// The statistics passes' bulk-copy stages exceed the default shared-memory limit: raised
+// once per device and mask variant.
+cudaError_t ensure_stat_smem_attr(bool masked, const void* p0, const void* p1, const void* p2, int smem) {
+  static std::atomic<uint64_t> done[2];
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  std::atomic<uint64_t>& word = done[masked ? 1 : 0];
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+  if (bit != 0 && (word.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  for (const void* f : {p0, p1, p2}) {
+    err = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
+  }
+  if (bit != 0) word.fetch_or(bit, std::memory_order_acq_rel);
+  return cudaSuccess;
+}
+
 RZ_API size_t rz_workspace_bytes_ratio_stats(int64_t n_tok, int32_t n_resp) {
   if (n_tok < 1 || n_tok >= (int64_t{1} << 31) || n_resp < 1) return 0;
   return align_up(stats_k3_off(n_tok) + sizeof(double) * 2 * stat_blocks(n_tok), kAlign);
@@ -1172,23 +1214,32 @@ RZ_API rz_status rz_ratio_stats(const float* lp, const float* lp_rollout, const 
   if (cudaMemsetAsync(sel, 0, 16, st) != cudaSuccess) return RZ_ERR_CUDA;
   const int nb = stat_blocks(n_tok);
   StatPartial* acc = at<StatPartial>(workspace, stats_acc_off(n_tok));
-  const bool vec = aligned(lp, 16) && aligned(lp_rollout, 16);
-  // pass 0 (arithmetic-heavy, few histogram bins) runs one CTA per token block; the radix
-  // passes run persistent CTAs, a few per SM, that flush their histograms once
+  int* status = at<int>(workspace, 0);
+  // whole blocks are bulk-copied into shared memory: 16-byte aligned arrays only (otherwise
+  // every block is read from global memory)
+  const bool vec = aligned(lp, 16) && aligned(lp_rollout, 16) && (token_mask == nullptr || aligned(token_mask, 16));
   const int sms = sm_count();
   if (sms <= 0) return RZ_ERR_CUDA;
   const int grid = std::min(nb, kStatCtasPerSm * sms);
-  ratio_stats_pass0<<<nb, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, vec, nb, parts, hist);
-  ratio_stats_reduce<<<1, 1024, 0, st>>>(parts, nb, acc, sel);
   double* k3_parts = at<double>(workspace, stats_k3_off(n_tok));
   const int nk3 = 2 * nb;  // two k3 half-sums per token block, one from each radix pass
-  ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, kStatBins, 11, sel, acc, 0, stats_out, k3_parts, nk3);
-  ratio_stats_pass<0><<<grid, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, vec, nb, sel, 21, 10, 0x7ffu,
-                                                     hist, k3_parts);
-  ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, kStatBins, 11, sel, acc, 0, stats_out, k3_parts, nk3);
-  ratio_stats_pass<1><<<grid, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, vec, nb, sel, 10, 0, 0x3ffu,
-                                                     hist, k3_parts);
-  ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, 1024, 10, sel, acc, 1, stats_out, k3_parts, nk3);
+  const bool masked = token_mask != nullptr;
+  auto pass0 = masked ? ratio_stats_pass0<true> : ratio_stats_pass0<false>;
+  auto pass1 = masked ? ratio_stats_pass<true, 0> : ratio_stats_pass<false, 0>;
+  auto pass2 = masked ? ratio_stats_pass<true, 1> : ratio_stats_pass<false, 1>;
+  const int smem = masked ? StatSmem<true>::kBytes : StatSmem<false>::kBytes;
+  if (ensure_stat_smem_attr(masked, reinterpret_cast<const void*>(pass0), reinterpret_cast<const void*>(pass1),
+                            reinterpret_cast<const void*>(pass2), smem) != cudaSuccess)
+    return RZ_ERR_CUDA;
+  pass0<<<grid, kStatThreads, smem, st>>>(lp, lp_rollout, token_mask, n_tok, vec, nb, parts, hist, status);
+  ratio_stats_reduce<<<1, 1024, 0, st>>>(parts, nb, acc, sel);
+  ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, kStatBins, 11, sel, acc, 0, stats_out, k3_parts, nk3, status);
+  pass1<<<grid, kStatThreads, smem, st>>>(lp, lp_rollout, token_mask, n_tok, vec, nb, sel, 21, 10, 0x7ffu, hist,
+                                          k3_parts, status);
+  ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, kStatBins, 11, sel, acc, 0, stats_out, k3_parts, nk3, status);
+  pass2<<<grid, kStatThreads, smem, st>>>(lp, lp_rollout, token_mask, n_tok, vec, nb, sel, 10, 0, 0x3ffu, hist,
+                                          k3_parts, status);
+  ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, 1024, 10, sel, acc, 1, stats_out, k3_parts, nk3, status);
   if (resp_mean_ratio_out != nullptr)
     response_mean_ratio_kernel<<<static_cast<unsigned>(ceil_div(n_resp, 8)), 256, 0, st>>>(
         lp, lp_rollout, token_mask, seg_offsets, n_resp, resp_mean_ratio_out);

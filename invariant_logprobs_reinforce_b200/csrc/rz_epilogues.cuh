@@ -1,7 +1,8 @@
 // rz_epilogues.cuh -- the epilogues that turn the tensor-core engine into the three
 // contractions of the path:
 //
-//   EpiLse<false>  fused LM head + online log-sum-exp + gather (logits stay on chip)
+//   EpiLse<false>  fused LM head + online log-sum-exp + gather (logits stay on chip);
+//                  EpiLse<false, true> the same with split partial sums (the fp8 forward)
 //   EpiLse<true>   the same, also keeping exp(z - tile max) (fp16) for the backward
 //   EpiDh          dH = dZ W tile, TMA-stored as bf16
 //   EpiDw          dW (+)= dZ^T H tile, TMA-stored / TMA-reduce-added in chunk order
@@ -60,7 +61,7 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
 // e_v are also written (fp16, TMA store) together with the tile maximum, so the backward
 // can form softmax probabilities without recomputing the logits; the log-sum-exp
 // arithmetic is the same code either way, so both variants give the same lse bits.
-template <bool STORE_P>
+template <bool STORE_P, bool SPLIT = false>
 struct EpiLse {
   CUtensorMap p_map;  // STORE_P: fp16 [rows, V] (box 32 x 32, 64-byte swizzle)
   const int32_t* ids; // launch-relative
@@ -157,17 +158,36 @@ struct EpiLse {
     // scaled operands only (never with STORE_P, whose staging slots the buffer shares)
     float* cs_buf = reinterpret_cast<float*>(stage.base);
     if (!STORE_P && col_scale != nullptr) stage_col_scales(st, nt, lane, cs_buf);
-    // pass 1: tile maximum of y over the valid columns
+    // pass 1: tile maximum of y over the valid columns.  SPLIT (the fp8 forward, whose MMAs
+    // take half the time of bf16's, so its epilogue is relatively twice as heavy): four
+    // partial maxima, column j into partial j % 4 (a maximum does not depend on the order),
+    // and no per-column test on chunks wholly inside V.
     float ymax = -INFINITY;
+    float ym[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
     tmem_for_chunks(taddr, nch, [&](int c, float (&v)[32]) {
       const int col0 = nt * BN + c * 32;
       scale_columns(cs_buf, c, v);
+      if constexpr (SPLIT) {
+        if (col0 + 32 <= V) {
 #pragma unroll
-      for (int j = 0; j < 32; ++j)
-        if (col0 + j < V) ymax = fmaxf(ymax, v[j]);
+          for (int j = 0; j < 32; ++j) ym[j & 3] = fmaxf(ym[j & 3], v[j]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (col0 + j < V) ym[j & 3] = fmaxf(ym[j & 3], v[j]);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (col0 + j < V) ymax = fmaxf(ymax, v[j]);
+      }
     });
-    // pass 2: exponentials relative to the tile maximum, their sum, the gather
+    if constexpr (SPLIT) ymax = fmaxf(fmaxf(ym[0], ym[1]), fmaxf(ym[2], ym[3]));
+    // pass 2: exponentials relative to the tile maximum, their sum, the gather.  The sum runs
+    // in column order; SPLIT: as four partial sums (column j into partial j % 4) added
+    // pairwise at the end, a fixed order per row with a quarter of the dependent adds.
     float tsum = 0.0f;
+    float ts[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     tmem_for_chunks(taddr, nch, [&](int c, float (&v)[32]) {
       const int col0 = nt * BN + c * 32;
       scale_columns(cs_buf, c, v);
@@ -179,10 +199,22 @@ struct EpiLse {
         zy[st.row] = st.rs * z;
       }
       float e[32];
+      if constexpr (SPLIT) {
+        if (col0 + 32 <= V) {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        e[j] = (col0 + j < V) ? ex2_approx((v[j] - ymax) * c2) : 0.0f;
-        tsum += e[j];
+          for (int j = 0; j < 32; ++j) e[j] = ex2_approx((v[j] - ymax) * c2);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) e[j] = (col0 + j < V) ? ex2_approx((v[j] - ymax) * c2) : 0.0f;
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) ts[j & 3] += e[j];
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          e[j] = (col0 + j < V) ? ex2_approx((v[j] - ymax) * c2) : 0.0f;
+          tsum += e[j];
+        }
       }
       if constexpr (STORE_P) {
         uint4 row[4];
@@ -193,6 +225,7 @@ struct EpiLse {
         stage.store_rows(&p_map, lane, row, col0, mb * BM + (r - lane), rows);
       }
     });
+    if constexpr (SPLIT) tsum = (ts[0] + ts[1]) + (ts[2] + ts[3]);
     const float tmax = st.rs * ymax;
     lse_fold(st.m, st.s, tmax, tsum);
     if constexpr (STORE_P) {

@@ -358,14 +358,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (nch > 2) tmem_for_chunks(taddr + 64, nch - 2, [&](int c, float(&v)[32]) { fn(c + 2, v); });
           }
         };
-        float ymax = -INFINITY;
+        // the tile maximum as four partial maxima and the sum as four partial sums (column j
+        // into partial j % 4, columns in order, added pairwise at the end), as in the bf16
+        // epilogue
+        float ym[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         visit([&](int c, float(&v)[32]) {
           const int col0 = col_base + c * 32;
+          if (col0 + 32 <= args.V) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (col0 + j < args.V) ymax = fmaxf(ymax, v[j]);
+            for (int j = 0; j < 32; ++j) ym[j & 3] = fmaxf(ym[j & 3], v[j]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (col0 + j < args.V) ym[j & 3] = fmaxf(ym[j & 3], v[j]);
+          }
         });
-        float tsum = 0.0f;
+        const float ymax = fmaxf(fmaxf(ym[0], ym[1]), fmaxf(ym[2], ym[3]));
+        float ts[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         visit([&](int c, float(&v)[32]) {
           const int col0 = col_base + c * 32;
           const unsigned off = static_cast<unsigned>(y - col0);
@@ -375,9 +384,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int j = 1; j < 32; ++j) z = (static_cast<unsigned>(j) == off) ? v[j] : z;
             args.zy[row] = z;
           }
+          if (col0 + 32 <= args.V) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) tsum += (col0 + j < args.V) ? ex2_approx((v[j] - ymax) * kLog2e) : 0.0f;
+            for (int j = 0; j < 32; ++j) ts[j & 3] += ex2_approx((v[j] - ymax) * kLog2e);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) ts[j & 3] += (col0 + j < args.V) ? ex2_approx((v[j] - ymax) * kLog2e) : 0.0f;
+          }
         });
+        const float tsum = (ts[0] + ts[1]) + (ts[2] + ts[3]);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[acc]);

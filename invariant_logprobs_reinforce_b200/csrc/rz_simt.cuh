@@ -324,151 +324,251 @@ __global__ void __launch_bounds__(kSetupThreads)
   }
 }
 
-// kappa_t = coef_i * w_t with the unclipped ratio w_t = exp(lp_t - lp_rollout_t), for the
-// 4096 tokens of block `block0 + blockIdx.x`; per-block partial sums of kappa with a fixed
+// kappa_t = coef_i * w_t with the unclipped ratio w_t = exp(lp_t - lp_rollout_t) over the
+// 4096-token blocks [block0, block0 + nblk), per-block partial sums of kappa with a fixed
 // reduction order (each lane adds its 4 consecutive tokens in fp32, everything else in
-// fp64).  Warp w owns the block's tokens [512 w, 512 w + 512) as four windows of 128
-// (lane: 4 consecutive tokens, one 16-byte load per array).
+// fp64), and (the CTA that finishes last of all the call's blocks) their fixed-order sum,
+// the loss.  Warp w owns a block's tokens [512 w, 512 w + 512) as four windows of 128 (lane:
+// 4 consecutive tokens).
 //
-// Fast path (every response touching the block staged: at most 256): the responses'
-// starts relative to the block and their coefficients sit in shared memory; a lane
-// finds its first token's response by a short walk and then advances with one compare
-// per token (a boundary can only fall between two consecutive tokens).  Otherwise the
-// block walks the global offsets.
+// Persistent CTAs, a few per SM, each taking the blocks blockIdx.x, blockIdx.x + gridDim.x,
+// ...: thread 0 streams a whole block's lp, lp_rollout (and mask) into shared memory with
+// bulk copies, kKappaStages blocks ahead, so the memory system always has several blocks in
+// flight however long the arithmetic of one takes.  The responses touching a block (their
+// starts relative to the block and their coefficients, at most 256 staged) are fetched one
+// block ahead into registers and put into shared memory when the block begins; a lane finds
+// its first token's response by a short walk and then advances with one compare per token
+// (a boundary can only fall between two consecutive tokens).  A block that is not whole or
+// not 16-byte aligned, or that more than 256 responses touch, takes the general path from
+// global memory.  A block's partial is computed the same way whichever CTA takes it, so the
+// loss does not depend on the grid.
 // MASKED / CLIPPED: compiled variants with and without the token mask and the truncated-IS
 // cap, so the plain call carries neither per-token test (the arithmetic is the same).
+constexpr int kKappaStages = 3;
+constexpr int kKappaCtasPerSm = 2;
+
+template <bool MASKED>
+struct KappaSmem {
+  static constexpr int kStageBytes = kKappaBlockTokens * (8 + (MASKED ? 1 : 0));  // lp | lp_rollout | mask
+  static constexpr int kBytes = kKappaStages * kStageBytes + 8 * kKappaStages;     // + one barrier per stage
+};
+static_assert(KappaSmem<true>::kStageBytes % 16 == 0 && 4 * kKappaBlockTokens % 16 == 0, "bulk copy sizes");
+
+// Staged responses of one block, fetched into registers ahead of their use: thread t holds
+// entry t (start and coefficient of response i0 + t), thread 0 also entry 256's start.
+struct KappaStaging {
+  int i0, cnt;
+  int64_t o, o_last;
+  float c;
+};
+
+__device__ __forceinline__ void kappa_staging_fetch(const int64_t* __restrict__ off, const float* __restrict__ coef,
+                                                    int R, int first, KappaStaging& st) {
+  constexpr int64_t kFarAbs = int64_t{1} << 62;  // a start beyond every block
+  const int t = threadIdx.x;
+  st.i0 = min(max(first, 0), R - 1);
+  st.cnt = min(kKappaStagedOffsets, R - st.i0);
+  st.o = (t <= st.cnt && st.i0 + t < R) ? off[st.i0 + t] : kFarAbs;
+  st.c = t < st.cnt ? coef[st.i0 + t] : 0.0f;
+  st.o_last = (t == 0 && st.cnt == kKappaStagedOffsets && st.i0 + kKappaStagedOffsets < R)
+                  ? off[st.i0 + kKappaStagedOffsets]
+                  : kFarAbs;
+}
+
 template <bool MASKED, bool CLIPPED>
-__global__ void __launch_bounds__(kKappaThreads, 5)
+__global__ void __launch_bounds__(kKappaThreads, kKappaCtasPerSm)
     token_kappa_kernel(const float* __restrict__ lp, const float* __restrict__ lp_roll,
                        const int64_t* __restrict__ off, int R, const float* __restrict__ coef,
-                       const int* __restrict__ block_first, int64_t n, int block0, int vec_ok,
+                       const int* __restrict__ block_first, int64_t n, int block0, int nblk, int vec_ok,
                        const uint8_t* __restrict__ mask, float clip_max, float* __restrict__ kappa,
                        float* __restrict__ w_out, double* __restrict__ block_sums, int total_blocks,
-                       int* __restrict__ ticket, float* __restrict__ loss) {
+                       int* __restrict__ ticket, float* __restrict__ loss, int* status) {
+  using Smem = KappaSmem<MASKED>;
   constexpr int kFar = 1 << 30;  // a relative start beyond the block
+  extern __shared__ __align__(128) uint8_t kx_smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(kx_smem + kKappaStages * Smem::kStageBytes);
   __shared__ int s_rel[kKappaStagedOffsets + 1];  // start of staged response k, relative to the block
   __shared__ float s_coef[kKappaStagedOffsets];
   __shared__ double warp_sums[kKappaThreads / 32];
-  __shared__ double s_tree[kKappaThreads];
   __shared__ bool s_last;
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int blk = block0 + blockIdx.x;
-  const int64_t b0 = static_cast<int64_t>(blk) * kKappaBlockTokens;
-  const int nb = static_cast<int>(min(n - b0, static_cast<int64_t>(kKappaBlockTokens)));  // tokens in the block
-  const bool full = vec_ok && nb == kKappaBlockTokens;
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
   const int wrel = warp * (kKappaBlockTokens / 8);
-  float4 la[kKappaIters], lb[kKappaIters];
-  uint32_t mk[kKappaIters];
-  if (full) {
-#pragma unroll
-    for (int it = 0; it < kKappaIters; ++it) {
-      const int64_t t0 = b0 + wrel + it * 128 + lane * 4;
-      la[it] = __ldcs(reinterpret_cast<const float4*>(lp + t0));
-      lb[it] = __ldcs(reinterpret_cast<const float4*>(lp_roll + t0));
-      mk[it] = MASKED ? __ldcs(reinterpret_cast<const unsigned int*>(mask + t0)) : 0x01010101u;
-    }
+  const int my_blocks =
+      static_cast<int>(blockIdx.x) < nblk ? (nblk - static_cast<int>(blockIdx.x) + gridDim.x - 1) / gridDim.x : 0;
+  auto blk_of = [&](int k) { return block0 + static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x); };
+  auto streamed = [&](int blk) {
+    return vec_ok != 0 && static_cast<int64_t>(blk + 1) * kKappaBlockTokens <= n;
+  };
+  auto stage_ptr = [&](int k) { return kx_smem + (k % kKappaStages) * Smem::kStageBytes; };
+  const uint64_t pol = make_l2_policy<kL2EvictFirst>();
+  auto issue = [&](int k) {  // thread 0: bulk copies of this CTA's k-th block into its stage
+    const int blk = blk_of(k);
+    if (!streamed(blk)) return;
+    uint8_t* sp = stage_ptr(k);
+    uint64_t* bar = &full[k % kKappaStages];
+    const int64_t b0 = static_cast<int64_t>(blk) * kKappaBlockTokens;
+    mbar_arrive_expect_tx(bar, Smem::kStageBytes);
+    bulk_load_1d(sp, lp + b0, 4 * kKappaBlockTokens, bar, pol);
+    bulk_load_1d(sp + 4 * kKappaBlockTokens, lp_roll + b0, 4 * kKappaBlockTokens, bar, pol);
+    if constexpr (MASKED) bulk_load_1d(sp + 8 * kKappaBlockTokens, mask + b0, kKappaBlockTokens, bar, pol);
+  };
+  if (tid == 0) {
+    for (int s = 0; s < kKappaStages; ++s) mbar_init(&full[s], 1);
+    fence_mbarrier_init();
   }
-  // launched as a programmatic dependent of the setup kernel, the block's token loads above
-  // overlap the setup; everything below reads what the setup wrote
+  __syncthreads();
+  if (tid == 0)
+    for (int k = 0; k < min(kKappaStages, my_blocks); ++k) issue(k);
+  // launched as a programmatic dependent of the setup kernel, the copies above overlap the
+  // setup; everything below reads what the setup wrote
   grid_dependency_wait();
-  const int i0 = min(max(block_first[blk], 0), R - 1);
-  const int cnt = min(kKappaStagedOffsets, R - i0);
-  for (int k = threadIdx.x; k <= cnt; k += kKappaThreads) {
-    const int64_t o = (i0 + k < R) ? off[i0 + k] - b0 : kFar;
-    s_rel[k] = static_cast<int>(max(min(o, static_cast<int64_t>(kFar)), static_cast<int64_t>(-kFar)));
-    if (k < cnt) s_coef[k] = coef[i0 + k];
-  }
-  __syncthreads();
-  // the staged responses cover the block when the first starts at or before its first
-  // token and the one after the last staged starts at or after its end
-  const bool staged = s_rel[0] <= 0 && s_rel[cnt] >= nb;
 
-  double local = 0.0;
-  if (staged && full) {
-    // staged response k of the current token, the start of response k + 1 and coef_k in
-    // registers: a token that starts no new response reads no shared memory
-    int k = 0;
-    int next = s_rel[1];
-    float ck = s_coef[0];
-#pragma unroll
-    for (int it = 0; it < kKappaIters; ++it) {
-      const int tr = wrel + it * 128 + lane * 4;
-      if (next <= tr) {
-        do ++k; while (s_rel[k + 1] <= tr);
-        next = s_rel[k + 1];
-        ck = s_coef[k];
-      }
-      const float a4[4] = {la[it].x, la[it].y, la[it].z, la[it].w};
-      const float b4[4] = {lb[it].x, lb[it].y, lb[it].z, lb[it].w};
-      const uint32_t m4 = mk[it];
-      float w[4], kv[4];
-      float part = 0.0f;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        if (j > 0 && next <= tr + j) {  // responses are non-empty: at most one start per token
-          ++k;
-          next = s_rel[k + 1];
-          ck = s_coef[k];
-        }
-        w[j] = ex2_approx((a4[j] - b4[j]) * kLog2e);
-        const float g = CLIPPED ? fminf(w[j], clip_max) : w[j];
-        kv[j] = (!MASKED || ((m4 >> (8 * j)) & 0xffu)) ? ck * g : 0.0f;
-        part += kv[j];
-      }
-      const int64_t t0 = b0 + tr;
-      __stcs(reinterpret_cast<float4*>(kappa + t0), make_float4(kv[0], kv[1], kv[2], kv[3]));
-      if (w_out != nullptr) __stcs(reinterpret_cast<float4*>(w_out + t0), make_float4(w[0], w[1], w[2], w[3]));
-      local += static_cast<double>(part);
+  KappaStaging cur{};
+  int first_next = 0;
+  if (my_blocks > 0) kappa_staging_fetch(off, coef, R, block_first[blk_of(0)], cur);
+  if (my_blocks > 1) first_next = block_first[blk_of(1)];
+  bool aborted = false;
+  int k = 0;
+  for (; k < my_blocks; ++k) {
+    const int blk = blk_of(k);
+    const int64_t b0 = static_cast<int64_t>(blk) * kKappaBlockTokens;
+    const int nb = static_cast<int>(min(n - b0, static_cast<int64_t>(kKappaBlockTokens)));  // tokens in the block
+    // this block's responses into shared memory (every reader of the previous block's is
+    // past the barrier that ended it)
+    if (tid <= cur.cnt)
+      s_rel[tid] = static_cast<int>(max(min(cur.o - b0, static_cast<int64_t>(kFar)), static_cast<int64_t>(-kFar)));
+    if (tid < cur.cnt) s_coef[tid] = cur.c;
+    if (tid == 0 && cur.cnt == kKappaStagedOffsets)
+      s_rel[kKappaStagedOffsets] =
+          static_cast<int>(max(min(cur.o_last - b0, static_cast<int64_t>(kFar)), static_cast<int64_t>(-kFar)));
+    // the next block's responses, and the one after's first response, fetched now
+    KappaStaging nxt{};
+    int first_after = 0;
+    if (k + 1 < my_blocks) kappa_staging_fetch(off, coef, R, first_next, nxt);
+    if (k + 2 < my_blocks) first_after = block_first[blk_of(k + 2)];
+    const bool in_smem = streamed(blk);
+    bool ok = true;
+    if (in_smem) ok = mbar_wait(&full[k % kKappaStages], static_cast<uint32_t>((k / kKappaStages) & 1), nullptr);
+    if (!__syncthreads_and(ok)) {  // a copy that never landed: give up on the launch
+      aborted = true;
+      break;
     }
-  } else {
-    // general path: tail blocks, unaligned arrays, or more than 256 responses in the block
-    for (int it = 0; it < kKappaIters; ++it) {
-      const int64_t t0 = b0 + wrel + it * 128 + lane * 4;
-      float part = 0.0f;
-      if (t0 < b0 + nb) {
-        int i = find_response(off, R, t0);
-        for (int j = 0; j < 4 && t0 + j < b0 + nb; ++j) {
-          const int64_t t = t0 + j;
-          while (i + 1 < R && __ldg(off + i + 1) <= t) ++i;
-          const float w = ex2_approx((lp[t] - lp_roll[t]) * kLog2e);
-          const float g = CLIPPED ? fminf(w, clip_max) : w;
-          const float kv = (!MASKED || mask[t] != 0) ? __ldg(coef + i) * g : 0.0f;
-          kappa[t] = kv;
-          if (w_out != nullptr) w_out[t] = w;
-          part += kv;
+    const int cnt = cur.cnt;
+    // the staged responses cover the block when the first starts at or before its first
+    // token and the one after the last staged starts at or after its end
+    const bool staged = s_rel[0] <= 0 && s_rel[cnt] >= nb;
+    double local = 0.0;
+    if (staged && in_smem) {
+      const uint8_t* sp = stage_ptr(k);
+      const float* s_lp = reinterpret_cast<const float*>(sp);
+      const float* s_lr = reinterpret_cast<const float*>(sp + 4 * kKappaBlockTokens);
+      // staged response kr of the current token, the start of response kr + 1 and its coef
+      // in registers: a token that starts no new response reads no shared memory for it
+      int kr = 0;
+      int next = s_rel[1];
+      float ck = s_coef[0];
+#pragma unroll
+      for (int it = 0; it < kKappaIters; ++it) {
+        const int tr = wrel + it * 128 + lane * 4;
+        if (next <= tr) {
+          do ++kr; while (s_rel[kr + 1] <= tr);
+          next = s_rel[kr + 1];
+          ck = s_coef[kr];
         }
+        const float4 la = *reinterpret_cast<const float4*>(s_lp + tr);
+        const float4 lb = *reinterpret_cast<const float4*>(s_lr + tr);
+        const uint32_t m4 = MASKED ? *reinterpret_cast<const uint32_t*>(sp + 8 * kKappaBlockTokens + tr) : 0x01010101u;
+        const float a4[4] = {la.x, la.y, la.z, la.w};
+        const float b4[4] = {lb.x, lb.y, lb.z, lb.w};
+        float w[4], kv[4];
+        float part = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (j > 0 && next <= tr + j) {  // responses are non-empty: at most one start per token
+            ++kr;
+            next = s_rel[kr + 1];
+            ck = s_coef[kr];
+          }
+          w[j] = ex2_approx((a4[j] - b4[j]) * kLog2e);
+          const float g = CLIPPED ? fminf(w[j], clip_max) : w[j];
+          kv[j] = (!MASKED || ((m4 >> (8 * j)) & 0xffu)) ? ck * g : 0.0f;
+          part += kv[j];
+        }
+        const int64_t t0 = b0 + tr;
+        __stcs(reinterpret_cast<float4*>(kappa + t0), make_float4(kv[0], kv[1], kv[2], kv[3]));
+        if (w_out != nullptr) __stcs(reinterpret_cast<float4*>(w_out + t0), make_float4(w[0], w[1], w[2], w[3]));
+        local += static_cast<double>(part);
       }
-      local += static_cast<double>(part);
+    } else {
+      // general path: a partial or unaligned block, or more than 256 responses in the block
+      for (int it = 0; it < kKappaIters; ++it) {
+        const int64_t t0 = b0 + wrel + it * 128 + lane * 4;
+        float part = 0.0f;
+        if (t0 < b0 + nb) {
+          int i = find_response(off, R, t0);
+          for (int j = 0; j < 4 && t0 + j < b0 + nb; ++j) {
+            const int64_t t = t0 + j;
+            while (i + 1 < R && __ldg(off + i + 1) <= t) ++i;
+            const float w = ex2_approx((lp[t] - lp_roll[t]) * kLog2e);
+            const float g = CLIPPED ? fminf(w, clip_max) : w;
+            const float kv = (!MASKED || mask[t] != 0) ? __ldg(coef + i) * g : 0.0f;
+            kappa[t] = kv;
+            if (w_out != nullptr) w_out[t] = w;
+            part += kv;
+          }
+        }
+        local += static_cast<double>(part);
+      }
     }
+    // fixed-order block reduction: warp butterfly, then warp partials in warp order
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) local += __shfl_xor_sync(0xffffffffu, local, o);
+    if (lane == 0) warp_sums[warp] = local;
+    __syncthreads();
+    if (tid == 0) {
+      double sum = 0.0;
+      for (int w = 0; w < kKappaThreads / 32; ++w) sum += warp_sums[w];
+      block_sums[blk] = sum;
+    }
+    __syncthreads();  // the stage, the staged responses and warp_sums are free again
+    if (tid == 0 && k + kKappaStages < my_blocks) issue(k + kKappaStages);
+    cur = nxt;
+    first_next = first_after;
   }
-  // fixed-order block reduction: warp butterfly, then warp partials in warp order
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) local += __shfl_xor_sync(0xffffffffu, local, o);
-  if (lane == 0) warp_sums[warp] = local;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    double sum = 0.0;
-    for (int w = 0; w < kKappaThreads / 32; ++w) sum += warp_sums[w];
-    block_sums[blk] = sum;
+  if (aborted && tid == 0) {
+    atomicOr(status, kDevWaitTimeout);
+    // copies still in flight must land before the CTA's shared memory goes away
+    for (int j = k; j < min(k + kKappaStages, my_blocks); ++j)
+      if (streamed(blk_of(j))) mbar_wait(&full[j % kKappaStages], static_cast<uint32_t>((j / kKappaStages) & 1), nullptr);
+  }
+  // the CTA whose blocks complete the count over every launch of the call (the ticket is
+  // cleared with the status word) forms the loss; a CTA that gave up still counts its
+  // blocks, and the loss is then NaN
+  if (tid == 0) {
     __threadfence();
-    // the last of all total_blocks blocks (over every launch of the call; the ticket is
-    // cleared with the status word) forms the loss
-    s_last = atomicAdd(ticket, 1) == total_blocks - 1;
+    s_last = atomicAdd(ticket, my_blocks) + my_blocks == total_blocks;
   }
   __syncthreads();
   if (!s_last) return;
   __threadfence();
+  if (*reinterpret_cast<volatile const int*>(status) & kDevWaitTimeout) {
+    if (tid == 0) *loss = __int_as_float(0x7fc00000);
+    return;
+  }
   // loss = sum of the block partials in a fixed order: strided per thread, then a fixed tree
+  // (in the stage memory, whose copies have all landed)
+  double* s_tree = reinterpret_cast<double*>(kx_smem);
   double acc = 0.0;
-  for (int b = threadIdx.x; b < total_blocks; b += kKappaThreads) acc += __ldcg(block_sums + b);
-  s_tree[threadIdx.x] = acc;
+  for (int b = tid; b < total_blocks; b += kKappaThreads) acc += __ldcg(block_sums + b);
+  s_tree[tid] = acc;
   __syncthreads();
   for (int w = kKappaThreads >> 1; w > 0; w >>= 1) {
-    if (threadIdx.x < w) s_tree[threadIdx.x] += s_tree[threadIdx.x + w];
+    if (tid < w) s_tree[tid] += s_tree[tid + w];
     __syncthreads();
   }
-  if (threadIdx.x == 0) *loss = static_cast<float>(s_tree[0]);
+  if (tid == 0) *loss = static_cast<float>(s_tree[0]);
 }
 
 // ------------------------------------------------------------------------ backward
@@ -544,7 +644,7 @@ __global__ void __launch_bounds__(256)
 constexpr int kStatThreads = 256;
 constexpr int kStatTokens = 4096;  // tokens per block
 constexpr int kStatBins = 2048;    // 11 bits per radix pass
-constexpr int kStatCtasPerSm = 4;  // resident CTAs per SM of the persistent passes (register-limited)
+constexpr int kStatCtasPerSm = 2;  // resident CTAs per SM of the passes (their shared-memory stages)
 
 struct StatPartial {
   double k1, k2, k3;
@@ -623,31 +723,128 @@ __device__ __forceinline__ void load_stat_quads(const float* __restrict__ lp, co
   }
 }
 
-// Both passes loop over the 4096-token blocks blk = blockIdx.x, blockIdx.x + gridDim.x, ...
-// (one block per CTA when the grid covers them all): each block's fp64 partial is computed
-// the same way whichever CTA takes it, so the statistics do not depend on the grid, and a
-// CTA adds its shared histogram into the global one once, at the end (integer counts).
+// The same quads from a block streamed into shared memory (a whole block: no tail).
+__device__ __forceinline__ void load_stat_quads_smem(const float* s_lp, const float* s_lr, const uint8_t* s_mk,
+                                                     StatQuads& q) {
+#pragma unroll
+  for (int k = 0; k < kStatQuads; ++k) {
+    const int t = 4 * (threadIdx.x + k * kStatThreads);
+    const float4 x = *reinterpret_cast<const float4*>(s_lp + t);
+    const float4 y = *reinterpret_cast<const float4*>(s_lr + t);
+    q.a[k][0] = x.x, q.a[k][1] = x.y, q.a[k][2] = x.z, q.a[k][3] = x.w;
+    q.b[k][0] = y.x, q.b[k][1] = y.y, q.b[k][2] = y.z, q.b[k][3] = y.w;
+    const uint32_t m4 = s_mk != nullptr ? *reinterpret_cast<const uint32_t*>(s_mk + t) : 0x01010101u;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) q.on[k][i] = ((m4 >> (8 * i)) & 0xffu) != 0;
+  }
+}
+
+// Every statistics pass runs persistent CTAs over the 4096-token blocks blk = blockIdx.x,
+// blockIdx.x + gridDim.x, ...: thread 0 bulk-copies each whole, 16-byte-aligned block of lp,
+// lp_rollout (and the mask) into one of StatSmem::kStages shared-memory stages, that many blocks
+// ahead of its use, so several blocks are always in flight however long the arithmetic of
+// one takes (a partial or unaligned block is read from global memory instead).  body(blk, q)
+// runs on every thread with the block's tokens as quads; each block's partial is computed
+// the same way whichever CTA takes it, so the statistics do not depend on the grid.
+// Returns false when a copy never landed (status bit set; the CTA stops once the copies
+// still in flight have landed).
+// Stages: three blocks ahead (two with the mask, whose bytes would not leave room for two
+// CTAs per SM beside the 8 KB histogram).
+template <bool MASKED>
+struct StatSmem {
+  static constexpr int kStages = MASKED ? 2 : 3;
+  static constexpr int kStageBytes = kStatTokens * (8 + (MASKED ? 1 : 0));  // lp | lp_rollout | mask
+  static constexpr int kBytes = kStages * kStageBytes + 8 * kStages;
+};
+
+template <bool MASKED, class Body>
+__device__ __forceinline__ bool stat_stream_blocks(const float* __restrict__ lp, const float* __restrict__ lp_roll,
+                                                   const uint8_t* __restrict__ mask, int64_t n, bool vec, int nblk,
+                                                   uint8_t* smem, int* status, Body&& body) {
+  using Smem = StatSmem<MASKED>;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Smem::kStages * Smem::kStageBytes);
+  const int tid = threadIdx.x;
+  const int my = static_cast<int>(blockIdx.x) < nblk
+                     ? (nblk - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x)
+                     : 0;
+  auto blk_of = [&](int k) { return static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x); };
+  // only the last block of the array can be partial, and it is the last of its CTA, so a
+  // stage whose block is not streamed is never needed again
+  auto streamed = [&](int blk) { return vec && static_cast<int64_t>(blk + 1) * kStatTokens <= n; };
+  auto stage = [&](int k) { return smem + (k % Smem::kStages) * Smem::kStageBytes; };
+  const uint64_t pol = make_l2_policy<kL2EvictFirst>();
+  auto issue = [&](int k) {
+    const int blk = blk_of(k);
+    if (!streamed(blk)) return;
+    uint8_t* sp = stage(k);
+    uint64_t* bar = &full[k % Smem::kStages];
+    const int64_t b0 = static_cast<int64_t>(blk) * kStatTokens;
+    mbar_arrive_expect_tx(bar, Smem::kStageBytes);
+    bulk_load_1d(sp, lp + b0, 4 * kStatTokens, bar, pol);
+    bulk_load_1d(sp + 4 * kStatTokens, lp_roll + b0, 4 * kStatTokens, bar, pol);
+    if constexpr (MASKED) bulk_load_1d(sp + 8 * kStatTokens, mask + b0, kStatTokens, bar, pol);
+  };
+  if (tid == 0) {
+    for (int s = 0; s < Smem::kStages; ++s) mbar_init(&full[s], 1);
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  if (tid == 0)
+    for (int k = 0; k < min(Smem::kStages, my); ++k) issue(k);
+  int k = 0;
+  bool ok = true;
+  for (; k < my; ++k) {
+    const int blk = blk_of(k);
+    const bool in_smem = streamed(blk);
+    bool landed = true;
+    if (in_smem) landed = mbar_wait(&full[k % Smem::kStages], static_cast<uint32_t>((k / Smem::kStages) & 1), nullptr);
+    if (!__syncthreads_and(landed)) {
+      ok = false;
+      break;
+    }
+    StatQuads q;
+    if (in_smem) {
+      const uint8_t* sp = stage(k);
+      load_stat_quads_smem(reinterpret_cast<const float*>(sp), reinterpret_cast<const float*>(sp + 4 * kStatTokens),
+                           MASKED ? sp + 8 * kStatTokens : nullptr, q);
+    } else {
+      load_stat_quads(lp, lp_roll, MASKED ? mask : nullptr, n, vec, blk, q);
+    }
+    __syncthreads();  // every thread has its quads: the stage is free
+    if (tid == 0 && k + Smem::kStages < my) issue(k + Smem::kStages);
+    body(blk, q);
+  }
+  if (!ok && tid == 0) {
+    atomicOr(status, kDevWaitTimeout);
+    for (int j = k; j < min(k + Smem::kStages, my); ++j)
+      if (streamed(blk_of(j))) mbar_wait(&full[j % Smem::kStages], static_cast<uint32_t>((j / Smem::kStages) & 1), nullptr);
+  }
+  return ok;
+}
+
+// Pass 0: per block the KL sums k1, k2 (fp64), min / max of w, the deviation peak and the
+// count; the histogram of the deviation's first radix digit (its top 11 bits).
+template <bool MASKED>
 __global__ void __launch_bounds__(kStatThreads, kStatCtasPerSm)
     ratio_stats_pass0(const float* __restrict__ lp, const float* __restrict__ lp_roll, const uint8_t* __restrict__ mask,
-                      int64_t n, bool vec, int nblk, StatPartial* __restrict__ parts, unsigned* __restrict__ hist) {
+                      int64_t n, bool vec, int nblk, StatPartial* __restrict__ parts, unsigned* __restrict__ hist,
+                      int* status) {
+  extern __shared__ __align__(128) uint8_t st_smem[];
   __shared__ unsigned s_hist[kStatBins];
   __shared__ StatPartial s_part[kStatThreads / 32];
   for (int b = threadIdx.x; b < kStatBins; b += kStatThreads) s_hist[b] = 0u;
   __syncthreads();
-  for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x) {
-    StatQuads q;
-    load_stat_quads(lp, lp_roll, mask, n, vec, blk, q);
-    double k1 = 0.0, k2 = 0.0, k3 = 0.0;
+  stat_stream_blocks<MASKED>(lp, lp_roll, mask, n, vec, nblk, st_smem, status, [&](int blk, const StatQuads& q) {
+    double k1 = 0.0, k2 = 0.0;
     float wmin = INFINITY, wmax = -INFINITY, dmax = 0.0f;
     int cnt = 0;
 #pragma unroll
     for (int k = 0; k < kStatQuads; ++k) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const bool on = q.on[k][i];
-        if (on) {
-          // the KL estimators in fp64 (k3 cancels to second order); min / max / deviation
-          // on the ratio exactly as the loss stage computes it
+        if (q.on[k][i]) {
+          // the KL estimators in fp64; min / max / deviation on the ratio exactly as the
+          // loss stage computes it
           const double x = static_cast<double>(q.a[k][i]) - static_cast<double>(q.b[k][i]);
           const float w = ratio_of(q.a[k][i], q.b[k][i]);
           const float dev = fabsf(w - 1.0f);
@@ -665,20 +862,18 @@ __global__ void __launch_bounds__(kStatThreads, kStatCtasPerSm)
     for (int o = 16; o > 0; o >>= 1) {
       k1 += __shfl_xor_sync(0xffffffffu, k1, o);
       k2 += __shfl_xor_sync(0xffffffffu, k2, o);
-      k3 += __shfl_xor_sync(0xffffffffu, k3, o);
       wmin = fminf(wmin, __shfl_xor_sync(0xffffffffu, wmin, o));
       wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, o));
       dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, o));
       cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
     }
-    if ((threadIdx.x & 31) == 0) s_part[threadIdx.x >> 5] = StatPartial{k1, k2, k3, wmin, wmax, dmax, cnt};
+    if ((threadIdx.x & 31) == 0) s_part[threadIdx.x >> 5] = StatPartial{k1, k2, 0.0, wmin, wmax, dmax, cnt};
     __syncthreads();
     if (threadIdx.x == 0) {
       StatPartial acc = s_part[0];
       for (int w = 1; w < kStatThreads / 32; ++w) {
         acc.k1 += s_part[w].k1;
         acc.k2 += s_part[w].k2;
-        acc.k3 += s_part[w].k3;
         acc.w_min = fminf(acc.w_min, s_part[w].w_min);
         acc.w_max = fmaxf(acc.w_max, s_part[w].w_max);
         acc.dev_max = fmaxf(acc.dev_max, s_part[w].dev_max);
@@ -687,31 +882,30 @@ __global__ void __launch_bounds__(kStatThreads, kStatCtasPerSm)
       parts[blk] = acc;
     }
     __syncthreads();  // s_part is rewritten by the next block
-  }
+  });
+  __syncthreads();
   for (int b = threadIdx.x; b < kStatBins; b += kStatThreads)
     if (s_hist[b]) atomicAdd(&hist[b], s_hist[b]);
 }
 
-// Histogram of the next radix digit among the deviations whose higher bits equal `prefix`,
-// and half of the k3 sum: in every 4096-token block, each thread's quads k with k % 2 ==
+// Radix passes: the histogram of the next digit among the deviations whose higher bits
+// equal `prefix`, and half of the k3 sum: in every block, each thread's quads k with k % 2 ==
 // K3_HALF (the fp64 series is the heaviest arithmetic of the statistics; split evenly over
-// the two radix passes, which stream at copy speed with issue slots to spare, it costs every
-// SM the same).  The block's half-sum goes to k3_parts[2 blk + K3_HALF], formed the same way
-// whichever CTA takes the block (per-thread sums in token order, warp butterfly, warps in
-// order), so it does not depend on the grid.
-template <int K3_HALF>
+// the two radix passes it costs every SM the same).  The block's half-sum goes to
+// k3_parts[2 blk + K3_HALF], formed the same way whichever CTA takes the block (per-thread
+// sums in token order, warp butterfly, warps in order).
+template <bool MASKED, int K3_HALF>
 __global__ void __launch_bounds__(kStatThreads, kStatCtasPerSm)
     ratio_stats_pass(const float* __restrict__ lp, const float* __restrict__ lp_roll, const uint8_t* __restrict__ mask,
                      int64_t n, bool vec, int nblk, const unsigned* __restrict__ sel, int shift_hi, int shift,
-                     unsigned digit_mask, unsigned* __restrict__ hist, double* __restrict__ k3_parts) {
+                     unsigned digit_mask, unsigned* __restrict__ hist, double* __restrict__ k3_parts, int* status) {
+  extern __shared__ __align__(128) uint8_t st_smem[];
   __shared__ unsigned s_hist[kStatBins];
   __shared__ double s_k3[kStatThreads / 32];
   for (int b = threadIdx.x; b < kStatBins; b += kStatThreads) s_hist[b] = 0u;
   const unsigned prefix = sel[0];
   __syncthreads();
-  for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x) {
-    StatQuads q;
-    load_stat_quads(lp, lp_roll, mask, n, vec, blk, q);
+  stat_stream_blocks<MASKED>(lp, lp_roll, mask, n, vec, nblk, st_smem, status, [&](int blk, const StatQuads& q) {
     double k3 = 0.0;
 #pragma unroll
     for (int k = 0; k < kStatQuads; ++k) {
@@ -734,7 +928,8 @@ __global__ void __launch_bounds__(kStatThreads, kStatCtasPerSm)
       k3_parts[2 * static_cast<int64_t>(blk) + K3_HALF] = sum;
     }
     __syncthreads();  // s_k3 is rewritten by the next block
-  }
+  });
+  __syncthreads();
   for (int b = threadIdx.x; b < kStatBins; b += kStatThreads)
     if (s_hist[b]) atomicAdd(&hist[b], s_hist[b]);
 }
@@ -790,7 +985,7 @@ static_assert(2 * kSelectThreads >= kStatBins, "two bins per thread");
 __global__ void __launch_bounds__(kSelectThreads)
     ratio_stats_select(unsigned* __restrict__ hist, int nbins, int digit_bits, unsigned* __restrict__ sel,
                        const StatPartial* __restrict__ acc_in, int last, double* __restrict__ stats,
-                       const double* __restrict__ k3_parts, int nk3) {
+                       const double* __restrict__ k3_parts, int nk3, const int* status) {
   __shared__ unsigned s_warp[kSelectThreads / 32];
   __shared__ double s_k3[kSelectThreads];
   if (last) {  // the k3 sum of all block halves: strided per thread, then a fixed tree
@@ -848,6 +1043,10 @@ __global__ void __launch_bounds__(kSelectThreads)
   sel[0] = med_bits;
   sel[1] = rank - below;
   if (!last) return;
+  if (*reinterpret_cast<volatile const int*>(status) & kDevWaitTimeout) {  // a pass gave up: no statistics
+    for (int i = 0; i < 9; ++i) stats[i] = __longlong_as_double(0x7ff8000000000000ll);
+    return;
+  }
   const StatPartial acc = *acc_in;
   const double m = acc.count > 0 ? static_cast<double>(acc.count) : 1.0;
   const double med = static_cast<double>(__uint_as_float(med_bits));
