@@ -259,13 +259,28 @@ int forward_group_m(int32_t d, int elem_bytes) {
 }
 int first_if_few(int consumer_tiles) { return consumer_tiles <= kFewConsumerTiles ? kL2EvictFirst : kL2Normal; }
 
-// Backward contractions with more than kFewConsumerTiles output tiles per row block (d >
-// 3072) run their N tiles in balanced groups of at most that many: a wave then streams
-// only its group's slice of W (dH) or H (dW), and a dZ row block has only the group's
-// tiles as consumers, at the price of reading dZ once per group.
+// dH with more than kFewConsumerTiles output tiles per row block (d > 3072) runs its N tiles
+// in balanced groups of at most that many: a wave then streams only its group's slice of
+// W, and a dZ row block has only the group's tiles as consumers, at the price of reading dZ
+// once per group (dW groups by the size of its slice of H, dw_group_n).
 int backward_group_n(int n_tiles) {
   if (n_tiles <= kFewConsumerTiles) return n_tiles;
   const int groups = (n_tiles + kFewConsumerTiles - 1) / kFewConsumerTiles;
+  return (n_tiles + groups - 1) / groups;
+}
+
+// dW's column tiles run in balanced groups whose slice of the chunk's H (kept in L2 with
+// evict-last while the group's waves stream dZ past it) takes at most 48 MB, and at most
+// kFewConsumerTiles tiles: at d = 2560 and 16384-row chunks two groups of 5 (42 MB each)
+// instead of one of 10 (84 MB), at the price of reading dZ once per group.  Measured on one
+// box: dW 233 vs 240-243 ms per step, the step 767-768 vs 778-783 ms (less DRAM traffic, so a
+// higher clock under the power cap).
+constexpr uint64_t kDwSliceBytes = 48ull << 20;
+int dw_group_n(int n_tiles, int64_t rows) {
+  const uint64_t tile_bytes = static_cast<uint64_t>(std::max<int64_t>(rows, 1)) * BN * 2;
+  const int cap = static_cast<int>(
+      std::min<uint64_t>(kFewConsumerTiles, std::max<uint64_t>(1, kDwSliceBytes / tile_bytes)));
+  const int groups = (n_tiles + cap - 1) / cap;
   return (n_tiles + groups - 1) / groups;
 }
 
@@ -705,7 +720,7 @@ rz_status run_backward_chunk(const rz_bf16* H, const rz_bf16* W, const int32_t* 
     e.out_rows = V;
     e.accumulate = c0 > 0 ? 1 : 0;
     GemmSched s = make_sched(V, d, 1, 1, rows);
-    s.group_n = backward_group_n(s.n_tiles);
+    s.group_n = dw_group_n(s.n_tiles, rows);
     s.l2_pol_a = first_if_few(s.group_n);  // dZ^T
     // the group's columns of the chunk's H
     s.l2_pol_b = keep_if_fits(static_cast<uint64_t>(rows) * std::min<int64_t>(d, s.group_n * BN) * 2);
@@ -1173,24 +1188,6 @@ size_t stats_k3_off(int64_t n) { return align_up(stats_acc_off(n) + sizeof(StatP
 constexpr int kNormBlocks = 1184;  // 8 per SM on 148 SMs; fixed, so the partial order is fixed
 }  // namespace
 
-// The statistics passes' bulk-copy stages exceed the default shared-memory limit: raised
-// once per device and mask variant.
-cudaError_t ensure_stat_smem_attr(bool masked, const void* p0, const void* p1, const void* p2, int smem) {
-  static std::atomic<uint64_t> done[2];
-  int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
-  if (err != cudaSuccess) return err;
-  std::atomic<uint64_t>& word = done[masked ? 1 : 0];
-  const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
-  if (bit != 0 && (word.load(std::memory_order_acquire) & bit)) return cudaSuccess;
-  for (const void* f : {p0, p1, p2}) {
-    err = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (err != cudaSuccess) return err;
-  }
-  if (bit != 0) word.fetch_or(bit, std::memory_order_acq_rel);
-  return cudaSuccess;
-}
-
 RZ_API size_t rz_workspace_bytes_ratio_stats(int64_t n_tok, int32_t n_resp) {
   if (n_tok < 1 || n_tok >= (int64_t{1} << 31) || n_resp < 1) return 0;
   return align_up(stats_k3_off(n_tok) + sizeof(double) * 2 * stat_blocks(n_tok), kAlign);
@@ -1214,32 +1211,23 @@ RZ_API rz_status rz_ratio_stats(const float* lp, const float* lp_rollout, const 
   if (cudaMemsetAsync(sel, 0, 16, st) != cudaSuccess) return RZ_ERR_CUDA;
   const int nb = stat_blocks(n_tok);
   StatPartial* acc = at<StatPartial>(workspace, stats_acc_off(n_tok));
-  int* status = at<int>(workspace, 0);
-  // whole blocks are bulk-copied into shared memory: 16-byte aligned arrays only (otherwise
-  // every block is read from global memory)
-  const bool vec = aligned(lp, 16) && aligned(lp_rollout, 16) && (token_mask == nullptr || aligned(token_mask, 16));
+  const bool vec = aligned(lp, 16) && aligned(lp_rollout, 16);
+  // pass 0 (arithmetic-heavy, few histogram bins) runs one CTA per token block; the radix
+  // passes run persistent CTAs, a few per SM, that flush their histograms once
   const int sms = sm_count();
   if (sms <= 0) return RZ_ERR_CUDA;
   const int grid = std::min(nb, kStatCtasPerSm * sms);
+  ratio_stats_pass0<<<nb, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, vec, nb, parts, hist);
+  ratio_stats_reduce<<<1, 1024, 0, st>>>(parts, nb, acc, sel);
   double* k3_parts = at<double>(workspace, stats_k3_off(n_tok));
   const int nk3 = 2 * nb;  // two k3 half-sums per token block, one from each radix pass
-  const bool masked = token_mask != nullptr;
-  auto pass0 = masked ? ratio_stats_pass0<true> : ratio_stats_pass0<false>;
-  auto pass1 = masked ? ratio_stats_pass<true, 0> : ratio_stats_pass<false, 0>;
-  auto pass2 = masked ? ratio_stats_pass<true, 1> : ratio_stats_pass<false, 1>;
-  const int smem = masked ? StatSmem<true>::kBytes : StatSmem<false>::kBytes;
-  if (ensure_stat_smem_attr(masked, reinterpret_cast<const void*>(pass0), reinterpret_cast<const void*>(pass1),
-                            reinterpret_cast<const void*>(pass2), smem) != cudaSuccess)
-    return RZ_ERR_CUDA;
-  pass0<<<grid, kStatThreads, smem, st>>>(lp, lp_rollout, token_mask, n_tok, vec, nb, parts, hist, status);
-  ratio_stats_reduce<<<1, 1024, 0, st>>>(parts, nb, acc, sel);
-  ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, kStatBins, 11, sel, acc, 0, stats_out, k3_parts, nk3, status);
-  pass1<<<grid, kStatThreads, smem, st>>>(lp, lp_rollout, token_mask, n_tok, vec, nb, sel, 21, 10, 0x7ffu, hist,
-                                          k3_parts, status);
-  ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, kStatBins, 11, sel, acc, 0, stats_out, k3_parts, nk3, status);
-  pass2<<<grid, kStatThreads, smem, st>>>(lp, lp_rollout, token_mask, n_tok, vec, nb, sel, 10, 0, 0x3ffu, hist,
-                                          k3_parts, status);
-  ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, 1024, 10, sel, acc, 1, stats_out, k3_parts, nk3, status);
+  ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, kStatBins, 11, sel, acc, 0, stats_out, k3_parts, nk3);
+  ratio_stats_pass<0><<<grid, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, vec, nb, sel, 21, 10, 0x7ffu,
+                                                     hist, k3_parts);
+  ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, kStatBins, 11, sel, acc, 0, stats_out, k3_parts, nk3);
+  ratio_stats_pass<1><<<grid, kStatThreads, 0, st>>>(lp, lp_rollout, token_mask, n_tok, vec, nb, sel, 10, 0, 0x3ffu,
+                                                     hist, k3_parts);
+  ratio_stats_select<<<1, kSelectThreads, 0, st>>>(hist, 1024, 10, sel, acc, 1, stats_out, k3_parts, nk3);
   if (resp_mean_ratio_out != nullptr)
     response_mean_ratio_kernel<<<static_cast<unsigned>(ceil_div(n_resp, 8)), 256, 0, st>>>(
         lp, lp_rollout, token_mask, seg_offsets, n_resp, resp_mean_ratio_out);

@@ -358,25 +358,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (nch > 2) tmem_for_chunks(taddr + 64, nch - 2, [&](int c, float(&v)[32]) { fn(c + 2, v); });
           }
         };
-        // the tile maximum as four partial maxima and the sum as four partial sums (column j
-        // into partial j % 4, columns in order, added pairwise at the end), as in the bf16
-        // epilogue
-        float ym[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        // one pass over the tile, chunk by chunk in column order: the chunk's maximum (four
+        // partial maxima, column j into partial j % 4), the tile's running maximum, the running
+        // sum rescaled to it, then the chunk's exponentials as four partial sums added
+        // pairwise; every TMEM column is read once.  The raw logit of the sampled token is
+        // kept on the way.
+        float tmax = -INFINITY, tsum = 0.0f;
         visit([&](int c, float(&v)[32]) {
           const int col0 = col_base + c * 32;
-          if (col0 + 32 <= args.V) {
+          const bool whole = col0 + 32 <= args.V;
+          float cm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          if (whole) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) ym[j & 3] = fmaxf(ym[j & 3], v[j]);
+            for (int j = 0; j < 32; ++j) cm[j & 3] = fmaxf(cm[j & 3], v[j]);
           } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-              if (col0 + j < args.V) ym[j & 3] = fmaxf(ym[j & 3], v[j]);
+              if (col0 + j < args.V) cm[j & 3] = fmaxf(cm[j & 3], v[j]);
           }
-        });
-        const float ymax = fmaxf(fmaxf(ym[0], ym[1]), fmaxf(ym[2], ym[3]));
-        float ts[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-        visit([&](int c, float(&v)[32]) {
-          const int col0 = col_base + c * 32;
+          // every visited chunk holds a column < V, so m_new is finite from the first chunk on
+          const float m_new = fmaxf(tmax, fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3])));
           const unsigned off = static_cast<unsigned>(y - col0);
           if (off < 32u) {
             float z = v[0];
@@ -384,19 +385,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int j = 1; j < 32; ++j) z = (static_cast<unsigned>(j) == off) ? v[j] : z;
             args.zy[row] = z;
           }
-          if (col0 + 32 <= args.V) {
+          float ts[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+          if (whole) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) ts[j & 3] += ex2_approx((v[j] - ymax) * kLog2e);
+            for (int j = 0; j < 32; ++j) ts[j & 3] += ex2_approx((v[j] - m_new) * kLog2e);
           } else {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) ts[j & 3] += (col0 + j < args.V) ? ex2_approx((v[j] - ymax) * kLog2e) : 0.0f;
+            for (int j = 0; j < 32; ++j) ts[j & 3] += (col0 + j < args.V) ? ex2_approx((v[j] - m_new) * kLog2e) : 0.0f;
           }
+          // first chunk: tmax = -inf, so the old sum (0) is scaled by 2^-inf = 0
+          tsum = __fmaf_rn(tsum, ex2_approx(__fmul_rn(tmax - m_new, kLog2e)), (ts[0] + ts[1]) + (ts[2] + ts[3]));
+          tmax = m_new;
         });
-        const float tsum = (ts[0] + ts[1]) + (ts[2] + ts[3]);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[acc]);
-        lse_fold(m, s, ymax, tsum);
+        lse_fold(m, s, tmax, tsum);
       }
       if (aborted) break;
       if (row < args.rows) {

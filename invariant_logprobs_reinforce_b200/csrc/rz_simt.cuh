@@ -394,7 +394,7 @@ __global__ void __launch_bounds__(kKappaThreads, kKappaCtasPerSm)
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
-  const int wrel = warp * (kKappaBlockTokens / 8);
+  const int wrel = warp * (kKappaBlockTokens / (kKappaThreads / 32));
   const int my_blocks =
       static_cast<int>(blockIdx.x) < nblk ? (nblk - static_cast<int>(blockIdx.x) + gridDim.x - 1) / gridDim.x : 0;
   auto blk_of = [&](int k) { return block0 + static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x); };
@@ -644,7 +644,7 @@ __global__ void __launch_bounds__(256)
 constexpr int kStatThreads = 256;
 constexpr int kStatTokens = 4096;  // tokens per block
 constexpr int kStatBins = 2048;    // 11 bits per radix pass
-constexpr int kStatCtasPerSm = 2;  // resident CTAs per SM of the passes (their shared-memory stages)
+constexpr int kStatCtasPerSm = 4;  // resident CTAs per SM of the persistent passes (register-limited)
 
 struct StatPartial {
   double k1, k2, k3;
@@ -723,128 +723,31 @@ __device__ __forceinline__ void load_stat_quads(const float* __restrict__ lp, co
   }
 }
 
-// The same quads from a block streamed into shared memory (a whole block: no tail).
-__device__ __forceinline__ void load_stat_quads_smem(const float* s_lp, const float* s_lr, const uint8_t* s_mk,
-                                                     StatQuads& q) {
-#pragma unroll
-  for (int k = 0; k < kStatQuads; ++k) {
-    const int t = 4 * (threadIdx.x + k * kStatThreads);
-    const float4 x = *reinterpret_cast<const float4*>(s_lp + t);
-    const float4 y = *reinterpret_cast<const float4*>(s_lr + t);
-    q.a[k][0] = x.x, q.a[k][1] = x.y, q.a[k][2] = x.z, q.a[k][3] = x.w;
-    q.b[k][0] = y.x, q.b[k][1] = y.y, q.b[k][2] = y.z, q.b[k][3] = y.w;
-    const uint32_t m4 = s_mk != nullptr ? *reinterpret_cast<const uint32_t*>(s_mk + t) : 0x01010101u;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) q.on[k][i] = ((m4 >> (8 * i)) & 0xffu) != 0;
-  }
-}
-
-// Every statistics pass runs persistent CTAs over the 4096-token blocks blk = blockIdx.x,
-// blockIdx.x + gridDim.x, ...: thread 0 bulk-copies each whole, 16-byte-aligned block of lp,
-// lp_rollout (and the mask) into one of StatSmem::kStages shared-memory stages, that many blocks
-// ahead of its use, so several blocks are always in flight however long the arithmetic of
-// one takes (a partial or unaligned block is read from global memory instead).  body(blk, q)
-// runs on every thread with the block's tokens as quads; each block's partial is computed
-// the same way whichever CTA takes it, so the statistics do not depend on the grid.
-// Returns false when a copy never landed (status bit set; the CTA stops once the copies
-// still in flight have landed).
-// Stages: three blocks ahead (two with the mask, whose bytes would not leave room for two
-// CTAs per SM beside the 8 KB histogram).
-template <bool MASKED>
-struct StatSmem {
-  static constexpr int kStages = MASKED ? 2 : 3;
-  static constexpr int kStageBytes = kStatTokens * (8 + (MASKED ? 1 : 0));  // lp | lp_rollout | mask
-  static constexpr int kBytes = kStages * kStageBytes + 8 * kStages;
-};
-
-template <bool MASKED, class Body>
-__device__ __forceinline__ bool stat_stream_blocks(const float* __restrict__ lp, const float* __restrict__ lp_roll,
-                                                   const uint8_t* __restrict__ mask, int64_t n, bool vec, int nblk,
-                                                   uint8_t* smem, int* status, Body&& body) {
-  using Smem = StatSmem<MASKED>;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Smem::kStages * Smem::kStageBytes);
-  const int tid = threadIdx.x;
-  const int my = static_cast<int>(blockIdx.x) < nblk
-                     ? (nblk - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x)
-                     : 0;
-  auto blk_of = [&](int k) { return static_cast<int>(blockIdx.x) + k * static_cast<int>(gridDim.x); };
-  // only the last block of the array can be partial, and it is the last of its CTA, so a
-  // stage whose block is not streamed is never needed again
-  auto streamed = [&](int blk) { return vec && static_cast<int64_t>(blk + 1) * kStatTokens <= n; };
-  auto stage = [&](int k) { return smem + (k % Smem::kStages) * Smem::kStageBytes; };
-  const uint64_t pol = make_l2_policy<kL2EvictFirst>();
-  auto issue = [&](int k) {
-    const int blk = blk_of(k);
-    if (!streamed(blk)) return;
-    uint8_t* sp = stage(k);
-    uint64_t* bar = &full[k % Smem::kStages];
-    const int64_t b0 = static_cast<int64_t>(blk) * kStatTokens;
-    mbar_arrive_expect_tx(bar, Smem::kStageBytes);
-    bulk_load_1d(sp, lp + b0, 4 * kStatTokens, bar, pol);
-    bulk_load_1d(sp + 4 * kStatTokens, lp_roll + b0, 4 * kStatTokens, bar, pol);
-    if constexpr (MASKED) bulk_load_1d(sp + 8 * kStatTokens, mask + b0, kStatTokens, bar, pol);
-  };
-  if (tid == 0) {
-    for (int s = 0; s < Smem::kStages; ++s) mbar_init(&full[s], 1);
-    fence_mbarrier_init();
-  }
-  __syncthreads();
-  if (tid == 0)
-    for (int k = 0; k < min(Smem::kStages, my); ++k) issue(k);
-  int k = 0;
-  bool ok = true;
-  for (; k < my; ++k) {
-    const int blk = blk_of(k);
-    const bool in_smem = streamed(blk);
-    bool landed = true;
-    if (in_smem) landed = mbar_wait(&full[k % Smem::kStages], static_cast<uint32_t>((k / Smem::kStages) & 1), nullptr);
-    if (!__syncthreads_and(landed)) {
-      ok = false;
-      break;
-    }
-    StatQuads q;
-    if (in_smem) {
-      const uint8_t* sp = stage(k);
-      load_stat_quads_smem(reinterpret_cast<const float*>(sp), reinterpret_cast<const float*>(sp + 4 * kStatTokens),
-                           MASKED ? sp + 8 * kStatTokens : nullptr, q);
-    } else {
-      load_stat_quads(lp, lp_roll, MASKED ? mask : nullptr, n, vec, blk, q);
-    }
-    __syncthreads();  // every thread has its quads: the stage is free
-    if (tid == 0 && k + Smem::kStages < my) issue(k + Smem::kStages);
-    body(blk, q);
-  }
-  if (!ok && tid == 0) {
-    atomicOr(status, kDevWaitTimeout);
-    for (int j = k; j < min(k + Smem::kStages, my); ++j)
-      if (streamed(blk_of(j))) mbar_wait(&full[j % Smem::kStages], static_cast<uint32_t>((j / Smem::kStages) & 1), nullptr);
-  }
-  return ok;
-}
-
-// Pass 0: per block the KL sums k1, k2 (fp64), min / max of w, the deviation peak and the
-// count; the histogram of the deviation's first radix digit (its top 11 bits).
-template <bool MASKED>
+// Both passes loop over the 4096-token blocks blk = blockIdx.x, blockIdx.x + gridDim.x, ...
+// (one block per CTA when the grid covers them all): each block's fp64 partial is computed
+// the same way whichever CTA takes it, so the statistics do not depend on the grid, and a
+// CTA adds its shared histogram into the global one once, at the end (integer counts).
 __global__ void __launch_bounds__(kStatThreads, kStatCtasPerSm)
     ratio_stats_pass0(const float* __restrict__ lp, const float* __restrict__ lp_roll, const uint8_t* __restrict__ mask,
-                      int64_t n, bool vec, int nblk, StatPartial* __restrict__ parts, unsigned* __restrict__ hist,
-                      int* status) {
-  extern __shared__ __align__(128) uint8_t st_smem[];
+                      int64_t n, bool vec, int nblk, StatPartial* __restrict__ parts, unsigned* __restrict__ hist) {
   __shared__ unsigned s_hist[kStatBins];
   __shared__ StatPartial s_part[kStatThreads / 32];
   for (int b = threadIdx.x; b < kStatBins; b += kStatThreads) s_hist[b] = 0u;
   __syncthreads();
-  stat_stream_blocks<MASKED>(lp, lp_roll, mask, n, vec, nblk, st_smem, status, [&](int blk, const StatQuads& q) {
-    double k1 = 0.0, k2 = 0.0;
+  for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x) {
+    StatQuads q;
+    load_stat_quads(lp, lp_roll, mask, n, vec, blk, q);
+    double k1 = 0.0, k2 = 0.0, k3 = 0.0;
     float wmin = INFINITY, wmax = -INFINITY, dmax = 0.0f;
     int cnt = 0;
 #pragma unroll
     for (int k = 0; k < kStatQuads; ++k) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        if (q.on[k][i]) {
-          // the KL estimators in fp64; min / max / deviation on the ratio exactly as the
-          // loss stage computes it
+        const bool on = q.on[k][i];
+        if (on) {
+          // the KL estimators in fp64 (k3 cancels to second order); min / max / deviation
+          // on the ratio exactly as the loss stage computes it
           const double x = static_cast<double>(q.a[k][i]) - static_cast<double>(q.b[k][i]);
           const float w = ratio_of(q.a[k][i], q.b[k][i]);
           const float dev = fabsf(w - 1.0f);
@@ -862,18 +765,20 @@ __global__ void __launch_bounds__(kStatThreads, kStatCtasPerSm)
     for (int o = 16; o > 0; o >>= 1) {
       k1 += __shfl_xor_sync(0xffffffffu, k1, o);
       k2 += __shfl_xor_sync(0xffffffffu, k2, o);
+      k3 += __shfl_xor_sync(0xffffffffu, k3, o);
       wmin = fminf(wmin, __shfl_xor_sync(0xffffffffu, wmin, o));
       wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, o));
       dmax = fmaxf(dmax, __shfl_xor_sync(0xffffffffu, dmax, o));
       cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
     }
-    if ((threadIdx.x & 31) == 0) s_part[threadIdx.x >> 5] = StatPartial{k1, k2, 0.0, wmin, wmax, dmax, cnt};
+    if ((threadIdx.x & 31) == 0) s_part[threadIdx.x >> 5] = StatPartial{k1, k2, k3, wmin, wmax, dmax, cnt};
     __syncthreads();
     if (threadIdx.x == 0) {
       StatPartial acc = s_part[0];
       for (int w = 1; w < kStatThreads / 32; ++w) {
         acc.k1 += s_part[w].k1;
         acc.k2 += s_part[w].k2;
+        acc.k3 += s_part[w].k3;
         acc.w_min = fminf(acc.w_min, s_part[w].w_min);
         acc.w_max = fmaxf(acc.w_max, s_part[w].w_max);
         acc.dev_max = fmaxf(acc.dev_max, s_part[w].dev_max);
@@ -882,30 +787,31 @@ __global__ void __launch_bounds__(kStatThreads, kStatCtasPerSm)
       parts[blk] = acc;
     }
     __syncthreads();  // s_part is rewritten by the next block
-  });
-  __syncthreads();
+  }
   for (int b = threadIdx.x; b < kStatBins; b += kStatThreads)
     if (s_hist[b]) atomicAdd(&hist[b], s_hist[b]);
 }
 
-// Radix passes: the histogram of the next digit among the deviations whose higher bits
-// equal `prefix`, and half of the k3 sum: in every block, each thread's quads k with k % 2 ==
+// Histogram of the next radix digit among the deviations whose higher bits equal `prefix`,
+// and half of the k3 sum: in every 4096-token block, each thread's quads k with k % 2 ==
 // K3_HALF (the fp64 series is the heaviest arithmetic of the statistics; split evenly over
-// the two radix passes it costs every SM the same).  The block's half-sum goes to
-// k3_parts[2 blk + K3_HALF], formed the same way whichever CTA takes the block (per-thread
-// sums in token order, warp butterfly, warps in order).
-template <bool MASKED, int K3_HALF>
+// the two radix passes, which stream at copy speed with issue slots to spare, it costs every
+// SM the same).  The block's half-sum goes to k3_parts[2 blk + K3_HALF], formed the same way
+// whichever CTA takes the block (per-thread sums in token order, warp butterfly, warps in
+// order), so it does not depend on the grid.
+template <int K3_HALF>
 __global__ void __launch_bounds__(kStatThreads, kStatCtasPerSm)
     ratio_stats_pass(const float* __restrict__ lp, const float* __restrict__ lp_roll, const uint8_t* __restrict__ mask,
                      int64_t n, bool vec, int nblk, const unsigned* __restrict__ sel, int shift_hi, int shift,
-                     unsigned digit_mask, unsigned* __restrict__ hist, double* __restrict__ k3_parts, int* status) {
-  extern __shared__ __align__(128) uint8_t st_smem[];
+                     unsigned digit_mask, unsigned* __restrict__ hist, double* __restrict__ k3_parts) {
   __shared__ unsigned s_hist[kStatBins];
   __shared__ double s_k3[kStatThreads / 32];
   for (int b = threadIdx.x; b < kStatBins; b += kStatThreads) s_hist[b] = 0u;
   const unsigned prefix = sel[0];
   __syncthreads();
-  stat_stream_blocks<MASKED>(lp, lp_roll, mask, n, vec, nblk, st_smem, status, [&](int blk, const StatQuads& q) {
+  for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x) {
+    StatQuads q;
+    load_stat_quads(lp, lp_roll, mask, n, vec, blk, q);
     double k3 = 0.0;
 #pragma unroll
     for (int k = 0; k < kStatQuads; ++k) {
@@ -928,8 +834,7 @@ __global__ void __launch_bounds__(kStatThreads, kStatCtasPerSm)
       k3_parts[2 * static_cast<int64_t>(blk) + K3_HALF] = sum;
     }
     __syncthreads();  // s_k3 is rewritten by the next block
-  });
-  __syncthreads();
+  }
   for (int b = threadIdx.x; b < kStatBins; b += kStatThreads)
     if (s_hist[b]) atomicAdd(&hist[b], s_hist[b]);
 }
@@ -985,7 +890,7 @@ static_assert(2 * kSelectThreads >= kStatBins, "two bins per thread");
 __global__ void __launch_bounds__(kSelectThreads)
     ratio_stats_select(unsigned* __restrict__ hist, int nbins, int digit_bits, unsigned* __restrict__ sel,
                        const StatPartial* __restrict__ acc_in, int last, double* __restrict__ stats,
-                       const double* __restrict__ k3_parts, int nk3, const int* status) {
+                       const double* __restrict__ k3_parts, int nk3) {
   __shared__ unsigned s_warp[kSelectThreads / 32];
   __shared__ double s_k3[kSelectThreads];
   if (last) {  // the k3 sum of all block halves: strided per thread, then a fixed tree
@@ -1043,10 +948,6 @@ __global__ void __launch_bounds__(kSelectThreads)
   sel[0] = med_bits;
   sel[1] = rank - below;
   if (!last) return;
-  if (*reinterpret_cast<volatile const int*>(status) & kDevWaitTimeout) {  // a pass gave up: no statistics
-    for (int i = 0; i < 9; ++i) stats[i] = __longlong_as_double(0x7ff8000000000000ll);
-    return;
-  }
   const StatPartial acc = *acc_in;
   const double m = acc.count > 0 ? static_cast<double>(acc.count) : 1.0;
   const double med = static_cast<double>(__uint_as_float(med_bits));

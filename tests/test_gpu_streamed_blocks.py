@@ -1,8 +1,8 @@
 """The loss stage and the ratio statistics at a size where every persistent CTA takes many
 4096-token blocks (about 2^23 tokens: seven or more blocks per CTA, so every shared-memory
 stage is refilled several times), with a ragged last block: the bulk-copied path (16-byte
-aligned inputs) against the path that reads global memory (the same values one element
-into a fresh buffer) bit for bit, with and without a token mask, and both against the fp64
+aligned inputs) against the path that reads global memory (the same values 4 bytes into a
+fresh buffer) bit for bit, with and without a token mask, and both against the fp64
 oracle."""
 import numpy as np
 import pytest
@@ -48,10 +48,11 @@ def _t(x):
 
 
 def _shifted(x, dtype):
-    """x one element into a fresh buffer: aligned to the element, not to 16 bytes."""
-    buf = torch.zeros(x.numel() + 1, dtype=dtype, device="cuda")
-    buf[1:] = x
-    return buf[1:]
+    """x 4 bytes into a fresh buffer: 4-byte aligned (what the calls require), not 16-byte."""
+    k = 4 // x.element_size()
+    buf = torch.zeros(x.numel() + k, dtype=dtype, device="cuda")
+    buf[k:] = x
+    return buf[k:]
 
 
 @pytest.mark.parametrize("masked", [False, True])
