@@ -95,15 +95,29 @@ __global__ void merge_lse_kernel(const float* __restrict__ part_m, const float* 
 // below.  flags[0] is the unsorted-ids flag; flags[1] and flags[2] are the tickets of the
 // setup kernel and of the ratio / kappa kernel (all cleared with the status word).
 
-// Per response (one warp each): the number of tokens whose mask byte is non-zero.
+// Per response (one warp each): the number of tokens whose mask byte is non-zero.  The
+// 16-byte-aligned middle of the response's mask is read 16 bytes per lane (nonzero bytes
+// counted four at a time: __vcmpne4 sets a byte to 0xff where it is nonzero), the ragged ends
+// byte by byte; the count is an integer, so the split does not change it.
+__device__ __forceinline__ int nonzero_bytes(uint32_t x) { return __popc(__vcmpne4(x, 0u)) >> 3; }
+
 __global__ void __launch_bounds__(256)
     masked_count_kernel(const uint8_t* __restrict__ mask, const int64_t* __restrict__ off, int R,
                         int* __restrict__ counted) {
   const int i = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (i >= R) return;
+  const int64_t o0 = off[i], o1 = off[i + 1];
+  const uint64_t base = reinterpret_cast<uint64_t>(mask);
+  const int64_t a0 = min(o1, o0 + static_cast<int64_t>((16u - ((base + static_cast<uint64_t>(o0)) & 15u)) & 15u));
+  const int64_t a1 = a0 + ((o1 - a0) & ~int64_t{15});
   int c = 0;
-  for (int64_t t = off[i] + lane; t < off[i + 1]; t += 32) c += mask[t] != 0;
+  for (int64_t t = o0 + lane; t < a0; t += 32) c += mask[t] != 0;
+  for (int64_t t = a0 + 16 * lane; t < a1; t += 16 * 32) {
+    const uint4 v = __ldcs(reinterpret_cast<const uint4*>(mask + t));
+    c += nonzero_bytes(v.x) + nonzero_bytes(v.y) + nonzero_bytes(v.z) + nonzero_bytes(v.w);
+  }
+  for (int64_t t = a1 + lane; t < o1; t += 32) c += mask[t] != 0;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
   if (lane == 0) counted[i] = c;
