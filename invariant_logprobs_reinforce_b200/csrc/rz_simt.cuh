@@ -350,7 +350,9 @@ __global__ void __launch_bounds__(kSetupThreads)
 // bulk copies, kKappaStages blocks ahead, so the memory system always has several blocks in
 // flight however long the arithmetic of one takes.  The responses touching a block (their
 // starts relative to the block and their coefficients, at most 256 staged) are fetched one
-// block ahead into registers and put into shared memory when the block begins; a lane finds
+// block ahead into registers and put into shared memory when the block begins (two buffers by
+// block parity, so that one barrier per block suffices: after it, thread 0 adds the previous
+// block's warp partials and refills the previous block's stage); a lane finds
 // its first token's response by a short walk and then advances with one compare per token
 // (a boundary can only fall between two consecutive tokens).  A block that is not whole or
 // not 16-byte aligned, or that more than 256 responses touch, takes the general path from
@@ -401,9 +403,10 @@ __global__ void __launch_bounds__(kKappaThreads, kKappaCtasPerSm)
   constexpr int kFar = 1 << 30;  // a relative start beyond the block
   extern __shared__ __align__(128) uint8_t kx_smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(kx_smem + kKappaStages * Smem::kStageBytes);
-  __shared__ int s_rel[kKappaStagedOffsets + 1];  // start of staged response k, relative to the block
-  __shared__ float s_coef[kKappaStagedOffsets];
-  __shared__ double warp_sums[kKappaThreads / 32];
+  // double-buffered by block parity, so that one barrier per block suffices
+  __shared__ int s_rel[2][kKappaStagedOffsets + 1];  // start of staged response k, relative to the block
+  __shared__ float s_coef[2][kKappaStagedOffsets];
+  __shared__ double warp_sums[2][kKappaThreads / 32];
   __shared__ bool s_last;
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -449,13 +452,14 @@ __global__ void __launch_bounds__(kKappaThreads, kKappaCtasPerSm)
     const int blk = blk_of(k);
     const int64_t b0 = static_cast<int64_t>(blk) * kKappaBlockTokens;
     const int nb = static_cast<int>(min(n - b0, static_cast<int64_t>(kKappaBlockTokens)));  // tokens in the block
-    // this block's responses into shared memory (every reader of the previous block's is
-    // past the barrier that ended it)
+    // this block's responses into the staging buffer of its parity (its last readers, block
+    // k - 2, are past the barrier of block k - 1)
+    const int pb = k & 1;
     if (tid <= cur.cnt)
-      s_rel[tid] = static_cast<int>(max(min(cur.o - b0, static_cast<int64_t>(kFar)), static_cast<int64_t>(-kFar)));
-    if (tid < cur.cnt) s_coef[tid] = cur.c;
+      s_rel[pb][tid] = static_cast<int>(max(min(cur.o - b0, static_cast<int64_t>(kFar)), static_cast<int64_t>(-kFar)));
+    if (tid < cur.cnt) s_coef[pb][tid] = cur.c;
     if (tid == 0 && cur.cnt == kKappaStagedOffsets)
-      s_rel[kKappaStagedOffsets] =
+      s_rel[pb][kKappaStagedOffsets] =
           static_cast<int>(max(min(cur.o_last - b0, static_cast<int64_t>(kFar)), static_cast<int64_t>(-kFar)));
     // the next block's responses, and the one after's first response, fetched now
     KappaStaging nxt{};
@@ -465,14 +469,24 @@ __global__ void __launch_bounds__(kKappaThreads, kKappaCtasPerSm)
     const bool in_smem = streamed(blk);
     bool ok = true;
     if (in_smem) ok = mbar_wait(&full[k % kKappaStages], static_cast<uint32_t>((k / kKappaStages) & 1), nullptr);
+    // the one barrier of a block: its staging is visible, and every thread is done with block
+    // k - 1 (its stage may be refilled, its warp partials added)
     if (!__syncthreads_and(ok)) {  // a copy that never landed: give up on the launch
       aborted = true;
       break;
     }
+    if (tid == 0 && k > 0) {
+      double sum = 0.0;
+      for (int w = 0; w < kKappaThreads / 32; ++w) sum += warp_sums[pb ^ 1][w];
+      block_sums[blk_of(k - 1)] = sum;
+      if (k - 1 + kKappaStages < my_blocks) issue(k - 1 + kKappaStages);
+    }
+    const int* rel = s_rel[pb];
+    const float* cf = s_coef[pb];
     const int cnt = cur.cnt;
     // the staged responses cover the block when the first starts at or before its first
     // token and the one after the last staged starts at or after its end
-    const bool staged = s_rel[0] <= 0 && s_rel[cnt] >= nb;
+    const bool staged = rel[0] <= 0 && rel[cnt] >= nb;
     double local = 0.0;
     if (staged && in_smem) {
       const uint8_t* sp = stage_ptr(k);
@@ -481,15 +495,15 @@ __global__ void __launch_bounds__(kKappaThreads, kKappaCtasPerSm)
       // staged response kr of the current token, the start of response kr + 1 and its coef
       // in registers: a token that starts no new response reads no shared memory for it
       int kr = 0;
-      int next = s_rel[1];
-      float ck = s_coef[0];
+      int next = rel[1];
+      float ck = cf[0];
 #pragma unroll
       for (int it = 0; it < kKappaIters; ++it) {
         const int tr = wrel + it * 128 + lane * 4;
         if (next <= tr) {
-          do ++kr; while (s_rel[kr + 1] <= tr);
-          next = s_rel[kr + 1];
-          ck = s_coef[kr];
+          do ++kr; while (rel[kr + 1] <= tr);
+          next = rel[kr + 1];
+          ck = cf[kr];
         }
         const float4 la = *reinterpret_cast<const float4*>(s_lp + tr);
         const float4 lb = *reinterpret_cast<const float4*>(s_lr + tr);
@@ -502,8 +516,8 @@ __global__ void __launch_bounds__(kKappaThreads, kKappaCtasPerSm)
         for (int j = 0; j < 4; ++j) {
           if (j > 0 && next <= tr + j) {  // responses are non-empty: at most one start per token
             ++kr;
-            next = s_rel[kr + 1];
-            ck = s_coef[kr];
+            next = rel[kr + 1];
+            ck = cf[kr];
           }
           w[j] = ex2_approx((a4[j] - b4[j]) * kLog2e);
           const float g = CLIPPED ? fminf(w[j], clip_max) : w[j];
@@ -539,22 +553,22 @@ __global__ void __launch_bounds__(kKappaThreads, kKappaCtasPerSm)
     // fixed-order block reduction: warp butterfly, then warp partials in warp order
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) local += __shfl_xor_sync(0xffffffffu, local, o);
-    if (lane == 0) warp_sums[warp] = local;
-    __syncthreads();
-    if (tid == 0) {
-      double sum = 0.0;
-      for (int w = 0; w < kKappaThreads / 32; ++w) sum += warp_sums[w];
-      block_sums[blk] = sum;
-    }
-    __syncthreads();  // the stage, the staged responses and warp_sums are free again
-    if (tid == 0 && k + kKappaStages < my_blocks) issue(k + kKappaStages);
+    if (lane == 0) warp_sums[pb][warp] = local;  // added in warp order after the next barrier
     cur = nxt;
     first_next = first_after;
   }
+  __syncthreads();
+  if (!aborted && tid == 0 && my_blocks > 0) {  // the last block's partial
+    double sum = 0.0;
+    for (int w = 0; w < kKappaThreads / 32; ++w) sum += warp_sums[(my_blocks - 1) & 1][w];
+    block_sums[blk_of(my_blocks - 1)] = sum;
+  }
   if (aborted && tid == 0) {
     atomicOr(status, kDevWaitTimeout);
-    // copies still in flight must land before the CTA's shared memory goes away
-    for (int j = k; j < min(k + kKappaStages, my_blocks); ++j)
+    // copies still in flight must land before the CTA's shared memory goes away: block j < k
+    // + kKappaStages - 1 was issued by the time the barrier of block k gave up
+    const int issued_end = min(k == 0 ? kKappaStages : k - 1 + kKappaStages, my_blocks);
+    for (int j = k; j < issued_end; ++j)
       if (streamed(blk_of(j))) mbar_wait(&full[j % kKappaStages], static_cast<uint32_t>((j / kKappaStages) & 1), nullptr);
   }
   // the CTA whose blocks complete the count over every launch of the call (the ticket is
