@@ -563,7 +563,8 @@ rz_status run_kappa(const float* lp, const float* lp_roll, const int64_t* off, i
   const int sms = sm_count();
   if (sms <= 0) return RZ_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(std::max(1, std::min(nblk, kKappaCtasPerSm * sms))));
+  const int ctas = masked ? KappaSmem<true>::kCtasPerSm : KappaSmem<false>::kCtasPerSm;
+  cfg.gridDim = dim3(static_cast<unsigned>(std::max(1, std::min(nblk, ctas * sms))));
   cfg.blockDim = dim3(kKappaThreads);
   cfg.dynamicSmemBytes = static_cast<size_t>(smem);
   cfg.stream = stream;

@@ -347,7 +347,7 @@ __global__ void __launch_bounds__(kSetupThreads)
 //
 // Persistent CTAs, a few per SM, each taking the blocks blockIdx.x, blockIdx.x + gridDim.x,
 // ...: thread 0 streams a whole block's lp, lp_rollout (and mask) into shared memory with
-// bulk copies, kKappaStages blocks ahead, so the memory system always has several blocks in
+// bulk copies, KappaSmem::kStages blocks ahead, so the memory system always has several blocks in
 // flight however long the arithmetic of one takes.  The responses touching a block (their
 // starts relative to the block and their coefficients, at most 256 staged) are fetched one
 // block ahead into registers and put into shared memory when the block begins (two buffers by
@@ -360,13 +360,16 @@ __global__ void __launch_bounds__(kSetupThreads)
 // loss does not depend on the grid.
 // MASKED / CLIPPED: compiled variants with and without the token mask and the truncated-IS
 // cap, so the plain call carries neither per-token test (the arithmetic is the same).
-constexpr int kKappaStages = 3;
-constexpr int kKappaCtasPerSm = 2;
+constexpr int kKappaMaxStages = 3;
 
+// Unmasked: three CTAs per SM with two stages each; masked (a ninth byte per token): two CTAs
+// with three stages (three CTAs would not fit).  Six blocks in flight per SM either way.
 template <bool MASKED>
 struct KappaSmem {
+  static constexpr int kStages = MASKED ? 3 : 2;
+  static constexpr int kCtasPerSm = MASKED ? 2 : 3;
   static constexpr int kStageBytes = kKappaBlockTokens * (8 + (MASKED ? 1 : 0));  // lp | lp_rollout | mask
-  static constexpr int kBytes = kKappaStages * kStageBytes + 8 * kKappaStages;     // + one barrier per stage
+  static constexpr int kBytes = kStages * kStageBytes + 8 * kStages;              // + one barrier per stage
 };
 static_assert(KappaSmem<true>::kStageBytes % 16 == 0 && 4 * kKappaBlockTokens % 16 == 0, "bulk copy sizes");
 
@@ -392,7 +395,7 @@ __device__ __forceinline__ void kappa_staging_fetch(const int64_t* __restrict__ 
 }
 
 template <bool MASKED, bool CLIPPED>
-__global__ void __launch_bounds__(kKappaThreads, kKappaCtasPerSm)
+__global__ void __launch_bounds__(kKappaThreads, KappaSmem<MASKED>::kCtasPerSm)
     token_kappa_kernel(const float* __restrict__ lp, const float* __restrict__ lp_roll,
                        const int64_t* __restrict__ off, int R, const float* __restrict__ coef,
                        const int* __restrict__ block_first, int64_t n, int block0, int nblk, int vec_ok,
@@ -400,9 +403,10 @@ __global__ void __launch_bounds__(kKappaThreads, kKappaCtasPerSm)
                        float* __restrict__ w_out, double* __restrict__ block_sums, int total_blocks,
                        int* __restrict__ ticket, float* __restrict__ loss, int* status) {
   using Smem = KappaSmem<MASKED>;
+  constexpr int kS = Smem::kStages;
   constexpr int kFar = 1 << 30;  // a relative start beyond the block
   extern __shared__ __align__(128) uint8_t kx_smem[];
-  uint64_t* full = reinterpret_cast<uint64_t*>(kx_smem + kKappaStages * Smem::kStageBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(kx_smem + kS * Smem::kStageBytes);
   // double-buffered by block parity, so that one barrier per block suffices
   __shared__ int s_rel[2][kKappaStagedOffsets + 1];  // start of staged response k, relative to the block
   __shared__ float s_coef[2][kKappaStagedOffsets];
@@ -418,13 +422,13 @@ __global__ void __launch_bounds__(kKappaThreads, kKappaCtasPerSm)
   auto streamed = [&](int blk) {
     return vec_ok != 0 && static_cast<int64_t>(blk + 1) * kKappaBlockTokens <= n;
   };
-  auto stage_ptr = [&](int k) { return kx_smem + (k % kKappaStages) * Smem::kStageBytes; };
+  auto stage_ptr = [&](int k) { return kx_smem + (k % kS) * Smem::kStageBytes; };
   const uint64_t pol = make_l2_policy<kL2EvictFirst>();
   auto issue = [&](int k) {  // thread 0: bulk copies of this CTA's k-th block into its stage
     const int blk = blk_of(k);
     if (!streamed(blk)) return;
     uint8_t* sp = stage_ptr(k);
-    uint64_t* bar = &full[k % kKappaStages];
+    uint64_t* bar = &full[k % kS];
     const int64_t b0 = static_cast<int64_t>(blk) * kKappaBlockTokens;
     mbar_arrive_expect_tx(bar, Smem::kStageBytes);
     bulk_load_1d(sp, lp + b0, 4 * kKappaBlockTokens, bar, pol);
@@ -432,12 +436,12 @@ __global__ void __launch_bounds__(kKappaThreads, kKappaCtasPerSm)
     if constexpr (MASKED) bulk_load_1d(sp + 8 * kKappaBlockTokens, mask + b0, kKappaBlockTokens, bar, pol);
   };
   if (tid == 0) {
-    for (int s = 0; s < kKappaStages; ++s) mbar_init(&full[s], 1);
+    for (int s = 0; s < kS; ++s) mbar_init(&full[s], 1);
     fence_mbarrier_init();
   }
   __syncthreads();
   if (tid == 0)
-    for (int k = 0; k < min(kKappaStages, my_blocks); ++k) issue(k);
+    for (int k = 0; k < min(kS, my_blocks); ++k) issue(k);
   // launched as a programmatic dependent of the setup kernel, the copies above overlap the
   // setup; everything below reads what the setup wrote
   grid_dependency_wait();
@@ -468,7 +472,7 @@ __global__ void __launch_bounds__(kKappaThreads, kKappaCtasPerSm)
     if (k + 2 < my_blocks) first_after = block_first[blk_of(k + 2)];
     const bool in_smem = streamed(blk);
     bool ok = true;
-    if (in_smem) ok = mbar_wait(&full[k % kKappaStages], static_cast<uint32_t>((k / kKappaStages) & 1), nullptr);
+    if (in_smem) ok = mbar_wait(&full[k % kS], static_cast<uint32_t>((k / kS) & 1), nullptr);
     // the one barrier of a block: its staging is visible, and every thread is done with block
     // k - 1 (its stage may be refilled, its warp partials added)
     if (!__syncthreads_and(ok)) {  // a copy that never landed: give up on the launch
@@ -479,7 +483,7 @@ __global__ void __launch_bounds__(kKappaThreads, kKappaCtasPerSm)
       double sum = 0.0;
       for (int w = 0; w < kKappaThreads / 32; ++w) sum += warp_sums[pb ^ 1][w];
       block_sums[blk_of(k - 1)] = sum;
-      if (k - 1 + kKappaStages < my_blocks) issue(k - 1 + kKappaStages);
+      if (k - 1 + kS < my_blocks) issue(k - 1 + kS);
     }
     const int* rel = s_rel[pb];
     const float* cf = s_coef[pb];
@@ -566,10 +570,10 @@ __global__ void __launch_bounds__(kKappaThreads, kKappaCtasPerSm)
   if (aborted && tid == 0) {
     atomicOr(status, kDevWaitTimeout);
     // copies still in flight must land before the CTA's shared memory goes away: block j < k
-    // + kKappaStages - 1 was issued by the time the barrier of block k gave up
-    const int issued_end = min(k == 0 ? kKappaStages : k - 1 + kKappaStages, my_blocks);
+    // + kS - 1 was issued by the time the barrier of block k gave up
+    const int issued_end = min(k == 0 ? kS : k - 1 + kS, my_blocks);
     for (int j = k; j < issued_end; ++j)
-      if (streamed(blk_of(j))) mbar_wait(&full[j % kKappaStages], static_cast<uint32_t>((j / kKappaStages) & 1), nullptr);
+      if (streamed(blk_of(j))) mbar_wait(&full[j % kS], static_cast<uint32_t>((j / kS) & 1), nullptr);
   }
   // the CTA whose blocks complete the count over every launch of the call (the ticket is
   // cleared with the status word) forms the loss; a CTA that gave up still counts its
